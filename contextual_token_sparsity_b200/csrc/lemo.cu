@@ -1,0 +1,332 @@
+// lemo.cu - host side of liblemo.so: argument checks, workspace layout,
+// tensor-map encoding and launches.  The kernels live in the included .cuh
+// files; everything is one translation unit so that the device error word is
+// a single symbol per device.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "lemo.h"
+#include "common.cuh"
+#include "move.cuh"
+#include "score.cuh"
+#include "select.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int32_t kMaxSeqlen = 1 << 22;
+constexpr int64_t kDefaultSpinNs = 2000000000LL;
+
+std::mutex g_mu;
+int g_sms[kMaxDevices];              // 0 = not queried yet
+bool g_score_attr[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+int g_skip_publish_tile = -1;
+int64_t g_spin_ns = kDefaultSpinNs;
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Number of SMs of the current device (cached).  Returns 0 on failure.
+int device_sms(int* dev_out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+    *dev_out = dev;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_sms[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+        g_sms[dev] = n;
+    }
+    return g_sms[dev];
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    return g_encode;
+}
+
+lemo_status launch_status() {
+    return cudaGetLastError() == cudaSuccess ? LEMO_OK : LEMO_ERR_CUDA;
+}
+
+// Shape checks common to scoring and selection.
+lemo_status check_shape(const lemo_shape* s, bool scoring) {
+    if (!s || !s->cu_seqlens) return LEMO_ERR_INVALID_ARG;
+    if (s->batch < 1 || s->total_L < 0 || s->max_seqlen < 0) return LEMO_ERR_INVALID_ARG;
+    if (s->max_seqlen > kMaxSeqlen) return LEMO_ERR_UNSUPPORTED;
+    if (s->total_L > 0 && s->max_seqlen == 0) return LEMO_ERR_INVALID_ARG;
+    if (s->block <= 0) return LEMO_ERR_INVALID_ARG;
+    if (s->block != 64 && s->block != 128) return LEMO_ERR_UNSUPPORTED;
+    if (!aligned(s->cu_seqlens, 4)) return LEMO_ERR_INVALID_ARG;
+    if (scoring) {
+        if (s->H < 1 || s->dh < 1) return LEMO_ERR_INVALID_ARG;
+        if (s->dh != 64 && s->dh != 128) return LEMO_ERR_UNSUPPORTED;
+        if ((int64_t)s->H * s->dh > (1 << 20)) return LEMO_ERR_UNSUPPORTED;
+    }
+    return LEMO_OK;
+}
+
+lemo::WsLayout layout_of(const lemo_shape* s) {
+    return lemo::ws_layout(s->batch, s->total_L, s->max_seqlen, s->block);
+}
+
+lemo_status check_ws(const lemo_shape* s, const void* ws, size_t ws_bytes) {
+    if (!ws || !aligned(ws, 256)) return LEMO_ERR_INVALID_ARG;
+    if (ws_bytes < layout_of(s).total) return LEMO_ERR_INVALID_ARG;
+    return LEMO_OK;
+}
+
+void launch_plan(const lemo_shape* s, char* ws, const lemo::WsLayout& lay, int32_t* zero_word,
+                 cudaStream_t st) {
+    lemo::plan_kernel<<<1, 1024, 0, st>>>(s->cu_seqlens, s->batch, s->total_L, s->max_seqlen,
+                                          s->block, ws, lay, zero_word);
+}
+
+bool encode_rows(CUtensorMap* tm, const uint16_t* base, int64_t rows, int64_t width,
+                 uint32_t box_rows) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)width, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)(width * 2)};
+    const cuuint32_t box[2] = {(cuuint32_t)lemo::score::KB, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(base), dims,
+               strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+// Persistent grid of the row-copy kernels: as many CTAs as fit on the SMs
+// at once (one full wave), so no CTA waits for a second wave.
+int g_move_ctas[kMaxDevices][2];
+
+template <typename Kernel>
+int move_grid(int dev, int sms, int which, Kernel kernel) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_move_ctas[dev][which] == 0) {
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, lemo::kMoveThreads, 0) !=
+                cudaSuccess ||
+            per_sm < 1)
+            per_sm = 1;
+        g_move_ctas[dev][which] = per_sm;
+    }
+    return sms * g_move_ctas[dev][which];
+}
+
+lemo_status check_move(const void* x, int64_t ld_x, int64_t x_rows, int32_t d, const void* y,
+                       int64_t ld_y, const int32_t* kept_idx, const int32_t* kept_total) {
+    if (!x || !y || !kept_idx || !kept_total) return LEMO_ERR_INVALID_ARG;
+    if (d <= 0 || x_rows < 0) return LEMO_ERR_INVALID_ARG;
+    if (d % 8 != 0) return LEMO_ERR_UNSUPPORTED;
+    if (ld_x < d || ld_y < d || ld_x % 8 != 0 || ld_y % 8 != 0) return LEMO_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(y, 16) || !aligned(kept_idx, 4) || !aligned(kept_total, 4))
+        return LEMO_ERR_INVALID_ARG;
+    return LEMO_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* lemo_status_string(lemo_status st) {
+    switch (st) {
+        case LEMO_OK: return "LEMO_OK";
+        case LEMO_ERR_INVALID_ARG: return "LEMO_ERR_INVALID_ARG";
+        case LEMO_ERR_UNSUPPORTED: return "LEMO_ERR_UNSUPPORTED";
+        case LEMO_ERR_CUDA: return "LEMO_ERR_CUDA";
+        case LEMO_ERR_CAPACITY: return "LEMO_ERR_CAPACITY";
+        case LEMO_ERR_TIMEOUT: return "LEMO_ERR_TIMEOUT";
+    }
+    return "LEMO_ERR_UNKNOWN";
+}
+
+size_t lemo_workspace_size(const lemo_shape* shape) {
+    if (check_shape(shape, false) != LEMO_OK) return 0;
+    return layout_of(shape).total;
+}
+
+int64_t lemo_block_max_elems(int32_t batch, const int32_t* lengths_host, int32_t block) {
+    if (batch < 1 || !lengths_host || block <= 0) return 0;
+    int64_t n = 0;
+    for (int s = 0; s < batch; ++s) {
+        if (lengths_host[s] < 0) return 0;
+        const int64_t nb = (lengths_host[s] + (int64_t)block - 1) / block;
+        n += nb * nb;
+    }
+    return n;
+}
+
+lemo_status lemo_score_blocks(const lemo_shape* shape, const uint16_t* q, const uint16_t* k,
+                              float scale, float* block_max, float* block_scores, void* ws,
+                              size_t ws_bytes, lemo_stream stream) {
+    lemo_status e = check_shape(shape, true);
+    if (e != LEMO_OK) return e;
+    if (!q || !k || !block_scores) return LEMO_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(block_scores, 4) ||
+        (block_max && !aligned(block_max, 4)))
+        return LEMO_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || scale == __builtin_inff()) return LEMO_ERR_INVALID_ARG;
+    if ((e = check_ws(shape, ws, ws_bytes)) != LEMO_OK) return e;
+    int dev = 0;
+    const int sms = device_sms(&dev);
+    if (sms <= 0) return LEMO_ERR_CUDA;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const lemo::WsLayout lay = layout_of(shape);
+    char* w = static_cast<char*>(ws);
+    float* mblk = block_max ? block_max : reinterpret_cast<float*>(w + lay.mblk);
+
+    launch_plan(shape, w, lay, nullptr, st);
+    if ((e = launch_status()) != LEMO_OK) return e;
+    if (shape->total_L > 0) {
+        namespace sc = lemo::score;
+        CUtensorMap tm_q, tm_k;
+        const int64_t width = (int64_t)shape->H * shape->dh;
+        if (!encode_rows(&tm_q, q, shape->total_L, width, sc::BM) ||
+            !encode_rows(&tm_k, k, shape->total_L, width, sc::BN))
+            return LEMO_ERR_CUDA;
+        {
+            std::lock_guard<std::mutex> lk(g_mu);
+            if (!g_score_attr[dev]) {
+                if (cudaFuncSetAttribute(sc::score_tiles_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         sc::SMEM_BYTES) != cudaSuccess)
+                    return LEMO_ERR_CUDA;
+                g_score_attr[dev] = true;
+            }
+        }
+        sc::Args a;
+        a.cu = shape->cu_seqlens;
+        a.batch = shape->batch;
+        a.H = shape->H;
+        a.dh = shape->dh;
+        a.block = shape->block;
+        a.out_scale = scale / (float)shape->H;
+        a.mblk = mblk;
+        a.ws = w;
+        a.lay = lay;
+        a.spin_limit_ns = (uint64_t)g_spin_ns;
+        sc::score_tiles_kernel<<<sms, sc::THREADS, sc::SMEM_BYTES, st>>>(tm_q, tm_k, a);
+        if ((e = launch_status()) != LEMO_OK) return e;
+        sc::column_sum_kernel<<<sms, 256, 0, st>>>(mblk, w, lay, shape->batch, block_scores);
+        if ((e = launch_status()) != LEMO_OK) return e;
+    }
+    return LEMO_OK;
+}
+
+lemo_status lemo_select(const lemo_shape* shape, const float* block_scores, float threshold,
+                        uint8_t* block_mask, int32_t* kept_idx, int32_t* cu_kept,
+                        int32_t* kept_total, void* ws, size_t ws_bytes, lemo_stream stream) {
+    lemo_status e = check_shape(shape, false);
+    if (e != LEMO_OK) return e;
+    if (!block_scores || !block_mask || !kept_idx || !cu_kept || !kept_total)
+        return LEMO_ERR_INVALID_ARG;
+    if (!aligned(block_scores, 4) || !aligned(kept_idx, 4) || !aligned(cu_kept, 4) ||
+        !aligned(kept_total, 4))
+        return LEMO_ERR_INVALID_ARG;
+    if ((e = check_ws(shape, ws, ws_bytes)) != LEMO_OK) return e;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const lemo::WsLayout lay = layout_of(shape);
+    char* w = static_cast<char*>(ws);
+    launch_plan(shape, w, lay, kept_total, st);
+    if ((e = launch_status()) != LEMO_OK) return e;
+    lemo::SelectArgs a;
+    a.cu = shape->cu_seqlens;
+    a.batch = shape->batch;
+    a.total_L = shape->total_L;
+    a.block = shape->block;
+    a.scores = block_scores;
+    a.theta = threshold;
+    a.mask = block_mask;
+    a.kept_idx = kept_idx;
+    a.cu_kept = cu_kept;
+    a.kept_total = kept_total;
+    a.ws = w;
+    a.lay = lay;
+    a.skip_publish_tile = g_skip_publish_tile;
+    a.spin_limit_ns = (uint64_t)g_spin_ns;
+    lemo::select_kernel<<<(unsigned)lay.n_lookback, lemo::kSelectThreads, 0, st>>>(a);
+    return launch_status();
+}
+
+lemo_status lemo_gather_pad(const uint16_t* x, int64_t ld_x, int64_t x_rows, int32_t d,
+                            const int32_t* kept_idx, const int32_t* kept_total, int32_t pad_to,
+                            uint16_t* y, int64_t ld_y, int64_t y_rows_capacity,
+                            lemo_stream stream) {
+    lemo_status e = check_move(x, ld_x, x_rows, d, y, ld_y, kept_idx, kept_total);
+    if (e != LEMO_OK) return e;
+    if (pad_to < 1 || y_rows_capacity < 0) return LEMO_ERR_INVALID_ARG;
+    int dev = 0;
+    const int sms = device_sms(&dev);
+    if (sms <= 0) return LEMO_ERR_CUDA;
+    lemo::MoveArgs a;
+    a.src = reinterpret_cast<const uint4*>(x);
+    a.dst = reinterpret_cast<uint4*>(y);
+    a.ld_src = ld_x / 8;
+    a.ld_dst = ld_y / 8;
+    a.x_rows = x_rows;
+    a.dvec = d / 8;
+    a.kept_idx = kept_idx;
+    a.kept_total = kept_total;
+    a.pad_to = pad_to;
+    a.cap = y_rows_capacity;
+    lemo::gather_pad_kernel<<<move_grid(dev, sms, 0, lemo::gather_pad_kernel), lemo::kMoveThreads, 0,
+                              reinterpret_cast<cudaStream_t>(stream)>>>(a);
+    return launch_status();
+}
+
+lemo_status lemo_scatter_residual(uint16_t* x, int64_t ld_x, int64_t x_rows, int32_t d,
+                                  const uint16_t* y, int64_t ld_y, const int32_t* kept_idx,
+                                  const int32_t* kept_total, lemo_stream stream) {
+    lemo_status e = check_move(x, ld_x, x_rows, d, y, ld_y, kept_idx, kept_total);
+    if (e != LEMO_OK) return e;
+    int dev = 0;
+    const int sms = device_sms(&dev);
+    if (sms <= 0) return LEMO_ERR_CUDA;
+    lemo::MoveArgs a;
+    a.src = reinterpret_cast<const uint4*>(y);
+    a.dst = reinterpret_cast<uint4*>(x);
+    a.ld_src = ld_y / 8;
+    a.ld_dst = ld_x / 8;
+    a.x_rows = x_rows;
+    a.dvec = d / 8;
+    a.kept_idx = kept_idx;
+    a.kept_total = kept_total;
+    a.pad_to = 1;
+    a.cap = 0;
+    lemo::scatter_residual_kernel<<<move_grid(dev, sms, 1, lemo::scatter_residual_kernel),
+                                    lemo::kMoveThreads, 0,
+                                    reinterpret_cast<cudaStream_t>(stream)>>>(a);
+    return launch_status();
+}
+
+lemo_status lemo_get_error(lemo_stream stream) {
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return LEMO_ERR_CUDA;
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbol(&v, lemo::g_error, sizeof(v)) != cudaSuccess) return LEMO_ERR_CUDA;
+    if (v != 0) {
+        const unsigned int z = 0;
+        if (cudaMemcpyToSymbol(lemo::g_error, &z, sizeof(z)) != cudaSuccess) return LEMO_ERR_CUDA;
+    }
+    return static_cast<lemo_status>(v);
+}
+
+void lemo_set_test_hooks(int32_t select_skip_publish_tile, int64_t spin_limit_ns) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_skip_publish_tile = select_skip_publish_tile < 0 ? -1 : select_skip_publish_tile;
+    g_spin_ns = spin_limit_ns > 0 ? spin_limit_ns : kDefaultSpinNs;
+}
+
+}  // extern "C"

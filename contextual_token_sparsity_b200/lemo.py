@@ -1,0 +1,157 @@
+"""ctypes binding of liblemo.so (C ABI in include/lemo.h), same entry-point names.
+
+Argument marshalling only: tensors become device pointers, the stream is the
+current torch stream unless one is given, and a non-OK status raises
+``LemoError``.  Every step of the path runs in the library's CUDA kernels;
+there is no CPU fallback - if the library is missing, every call raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "liblemo.so")
+
+STATUS = {0: "LEMO_OK", 1: "LEMO_ERR_INVALID_ARG", 2: "LEMO_ERR_UNSUPPORTED", 3: "LEMO_ERR_CUDA",
+          4: "LEMO_ERR_CAPACITY", 5: "LEMO_ERR_TIMEOUT"}
+LEMO_OK = 0
+LEMO_ERR_INVALID_ARG = 1
+LEMO_ERR_UNSUPPORTED = 2
+LEMO_ERR_CUDA = 3
+LEMO_ERR_CAPACITY = 4
+LEMO_ERR_TIMEOUT = 5
+
+
+class LemoError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = int(status)
+        super().__init__(f"{where}: {STATUS.get(self.status, self.status)}")
+
+
+class lemo_shape(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32),
+        ("cu_seqlens", ctypes.c_void_p),
+        ("total_L", ctypes.c_int32),
+        ("max_seqlen", ctypes.c_int32),
+        ("H", ctypes.c_int32),
+        ("dh", ctypes.c_int32),
+        ("block", ctypes.c_int32),
+    ]
+
+
+_P = ctypes.c_void_p
+_I32 = ctypes.c_int32
+_I64 = ctypes.c_int64
+_SIGS = {
+    "lemo_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "lemo_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(lemo_shape)]),
+    "lemo_block_max_elems": (_I64, [_I32, _P, _I32]),
+    "lemo_score_blocks": (ctypes.c_int, [ctypes.POINTER(lemo_shape), _P, _P, ctypes.c_float, _P,
+                                         _P, _P, ctypes.c_size_t, _P]),
+    "lemo_select": (ctypes.c_int, [ctypes.POINTER(lemo_shape), _P, ctypes.c_float, _P, _P, _P,
+                                   _P, _P, ctypes.c_size_t, _P]),
+    "lemo_gather_pad": (ctypes.c_int, [_P, _I64, _I64, _I32, _P, _P, _I32, _P, _I64, _I64, _P]),
+    "lemo_scatter_residual": (ctypes.c_int, [_P, _I64, _I64, _I32, _P, _I64, _P, _P, _P]),
+    "lemo_get_error": (ctypes.c_int, [_P]),
+    "lemo_set_test_hooks": (None, [_I32, _I64]),
+}
+
+_lib = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load liblemo.so (once) and declare its signatures.  Raises if absent."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise RuntimeError(f"liblemo.so not found at {path}; build it with "
+                               "`python -m contextual_token_sparsity_b200.build`")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(st: int, where: str):
+    if st != LEMO_OK:
+        raise LemoError(st, where)
+
+
+def make_shape(cu_seqlens, total_L: int, max_seqlen: int, H: int = 1, dh: int = 64,
+               block: int = 64) -> lemo_shape:
+    """lemo_shape for a packed batch; ``cu_seqlens`` is a device int32 tensor."""
+    return lemo_shape(int(cu_seqlens.numel()) - 1, _ptr(cu_seqlens), int(total_L),
+                      int(max_seqlen), int(H), int(dh), int(block))
+
+
+def lemo_workspace_size(shape: lemo_shape) -> int:
+    return int(load().lemo_workspace_size(ctypes.byref(shape)))
+
+
+def lemo_block_max_elems(lengths, block: int) -> int:
+    arr = (ctypes.c_int32 * len(lengths))(*[int(v) for v in lengths])
+    return int(load().lemo_block_max_elems(len(lengths), ctypes.cast(arr, ctypes.c_void_p), block))
+
+
+def lemo_score_blocks(shape, q, k, scale, block_max, block_scores, ws, stream=None):
+    _check(load().lemo_score_blocks(ctypes.byref(shape), _ptr(q), _ptr(k), float(scale),
+                                    _ptr(block_max), _ptr(block_scores), _ptr(ws),
+                                    ws.numel() * ws.element_size(), _stream(stream)),
+           "lemo_score_blocks")
+
+
+def lemo_select(shape, block_scores, threshold, block_mask, kept_idx, cu_kept, kept_total, ws,
+                stream=None):
+    _check(load().lemo_select(ctypes.byref(shape), _ptr(block_scores), float(threshold),
+                              _ptr(block_mask), _ptr(kept_idx), _ptr(cu_kept), _ptr(kept_total),
+                              _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "lemo_select")
+
+
+def lemo_gather_pad(x, kept_idx, kept_total, pad_to, y, stream=None, d=None):
+    """x [rows, ld_x] and y [capacity, ld_y] bf16/int16 2-D tensors (row-major)."""
+    d = x.shape[1] if d is None else d
+    _check(load().lemo_gather_pad(_ptr(x), x.stride(0), x.shape[0], int(d), _ptr(kept_idx),
+                                  _ptr(kept_total), int(pad_to), _ptr(y), y.stride(0),
+                                  y.shape[0], _stream(stream)),
+           "lemo_gather_pad")
+
+
+def lemo_scatter_residual(x, y, kept_idx, kept_total, stream=None, d=None):
+    d = x.shape[1] if d is None else d
+    _check(load().lemo_scatter_residual(_ptr(x), x.stride(0), x.shape[0], int(d), _ptr(y),
+                                        y.stride(0), _ptr(kept_idx), _ptr(kept_total),
+                                        _stream(stream)),
+           "lemo_scatter_residual")
+
+
+def lemo_get_error(stream=None) -> int:
+    """Synchronise the stream; return (and clear) the device error status."""
+    return int(load().lemo_get_error(_stream(stream)))
+
+
+def lemo_set_test_hooks(select_skip_publish_tile: int = -1, spin_limit_ns: int = 0):
+    load().lemo_set_test_hooks(int(select_skip_publish_tile), int(spin_limit_ns))

@@ -41,9 +41,12 @@ def to_bf16_bits(a) -> np.ndarray:
     """float -> bf16 bit patterns: first to float32 (numpy rounding), then
     the float32 pattern is rounded to its upper 16 bits, ties to even."""
     f = np.ascontiguousarray(a, dtype=np.float32)
-    u = f.view(np.uint32).astype(np.uint64)
-    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
-    return u.astype(np.uint16)
+    u = f.view(np.uint32)
+    r = (u >> 16) & np.uint32(1)
+    r += np.uint32(0x7FFF)
+    r += u  # cannot wrap for finite values (only NaN patterns are that large)
+    r >>= np.uint32(16)
+    return r.astype(np.uint16)
 
 
 def bf16_bits_to_f32(bits) -> np.ndarray:

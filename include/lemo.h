@@ -1,0 +1,234 @@
+/*
+ * lemo.h - C ABI of liblemo.so, the sm_100a (B200) implementation of the
+ * per-layer hot path of contextual token sparsity:
+ *
+ *   block scoring -> threshold -> compaction -> gather (selective load)
+ *   -> [caller's sublayer] -> scatter with in-place residual add.
+ *
+ * The method is that of "Jenga: Enhancing LLM Long-Context Fine-tuning with
+ * Contextual Token Sparsity" (USENIX ATC'25; called LeMo in arXiv
+ * 2501.09767).  Each entry point cites the section of that paper's
+ * aipaper.cc summary that defines the operation.
+ *
+ * Conventions shared by every entry point
+ * ----------------------------------------
+ *  - bf16 tensors are passed as `uint16_t*` holding bf16 bit patterns.
+ *  - "DEVICE" pointers are CUDA device (global memory) pointers on the
+ *    current device; "HOST" pointers are ordinary host memory.
+ *  - All work is enqueued on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream).  No entry point synchronises except lemo_get_error.
+ *  - The caller owns and allocates every buffer, including the workspace.
+ *    The library never allocates device memory.
+ *  - Argument errors are detected on the host before anything is enqueued:
+ *    the call returns LEMO_ERR_INVALID_ARG / LEMO_ERR_UNSUPPORTED and
+ *    launches nothing.  A CUDA launch error is returned as LEMO_ERR_CUDA.
+ *  - Errors that only the device can see (cu_seqlens inconsistent with the
+ *    shape, an index out of range, a capacity overflow, a bounded wait that
+ *    ran out) are recorded in a per-device error word and the affected work
+ *    is skipped; lemo_get_error() reports and clears it.
+ *  - Packed variable-length batches: sequence s occupies rows
+ *    cu_seqlens[s] .. cu_seqlens[s+1]-1 of every [total_L, ...] tensor.
+ *    Token blocks of `block` tokens start at each sequence's first row; the
+ *    last block of a sequence may be short.  Block-indexed arrays
+ *    ([total_blocks]) list all blocks of sequence 0, then sequence 1, ...,
+ *    where total_blocks = sum_s ceil(L_s / block).
+ */
+#ifndef LEMO_H
+#define LEMO_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LEMO_API __attribute__((visibility("default")))
+#else
+#define LEMO_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum lemo_status {
+    LEMO_OK = 0,
+    LEMO_ERR_INVALID_ARG = 1,  /* bad pointer, size, stride or cu_seqlens     */
+    LEMO_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. dh = 96)    */
+    LEMO_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed         */
+    LEMO_ERR_CAPACITY = 4,     /* an output buffer was too small (device side) */
+    LEMO_ERR_TIMEOUT = 5       /* a bounded device-side wait ran out           */
+} lemo_status;
+
+/* A cudaStream_t, passed as an opaque pointer. */
+typedef void* lemo_stream;
+
+/* Shape of one layer call on a packed batch. */
+typedef struct lemo_shape {
+    int32_t batch;              /* number of sequences, >= 1                       */
+    const int32_t* cu_seqlens;  /* DEVICE int32 [batch+1]: 0 = cu[0] <= cu[1] <= ...
+                                   <= cu[batch] = total_L (checked on device)       */
+    int32_t total_L;            /* rows of the packed batch, >= 0                  */
+    int32_t max_seqlen;         /* upper bound of every L_s (checked on device),
+                                   0 <= max_seqlen <= 4194304                      */
+    int32_t H;                  /* attention heads, >= 1                           */
+    int32_t dh;                 /* head dimension: 64 or 128                       */
+    int32_t block;              /* token block size b: 64 or 128                   */
+} lemo_shape;
+
+/* Human-readable name of a status code (static string). */
+LEMO_API const char* lemo_status_string(lemo_status st);
+
+/*
+ * Bytes of workspace that lemo_score_blocks / lemo_select need for `shape`
+ * (one buffer serves both; calls on one stream may share it).  The bound
+ * covers the per-sequence plan arrays, the compaction look-back descriptors
+ * and the block-score matrices when the caller passes block_max = NULL:
+ * ceil(max_seqlen/b) * (total_L/b + batch) floats.  Returns 0 for an invalid
+ * shape.  HOST-only computation, no CUDA call.
+ */
+LEMO_API size_t lemo_workspace_size(const lemo_shape* shape);
+
+/*
+ * Number of floats of the optional block_max output of lemo_score_blocks,
+ * sum_s ceil(L_s/b)^2, computed from HOST sequence lengths `lengths_host`
+ * [batch].  Returns 0 on a bad argument.
+ */
+LEMO_API int64_t lemo_block_max_elems(int32_t batch, const int32_t* lengths_host, int32_t block);
+
+/*
+ * Block-wise token informativeness scores (steps a1-a3).
+ *
+ * Defined by the Jenga summary, section 4.2.1: Eq. 1 (the informativeness
+ * of token j sums the raw pre-softmax scores S_ij = Q_i . K_j), Eq. 2 (a
+ * score block's informativeness is the maximum over its entries of the
+ * per-head positive scores summed over heads and divided by N_head) and the
+ * Fig. 6 caption (block scores are aggregated along the column).  Causal:
+ * only pairs i > j of one sequence count (the diagonal is excluded).
+ *
+ *   A_ij     = (1/H) * sum_h max(scale * Q[i,h,:] . K[j,h,:], 0)
+ *   M[n][m]  = max over i in block n, j in block m, j < i, of A_ij   (n >= m;
+ *              0 if the block holds no such pair)
+ *   score[m] = sum_{n = m}^{N_b - 1} M[n][m]                 (per sequence)
+ *
+ * q, k         DEVICE bf16 [total_L, H, dh] row-major (row stride H*dh),
+ *              16-byte aligned.
+ * scale        > 0; 1.0 gives raw Q.K (no 1/sqrt(dh)).
+ * block_max    DEVICE fp32, optional (NULL = keep it in the workspace).  When
+ *              given: for each sequence an [N_b, N_b] row-major matrix at
+ *              offset sum_{s'<s} N_b,s'^2 (see lemo_block_max_elems); only
+ *              entries with n >= m are written.
+ * block_scores DEVICE fp32 [total_blocks]: score[m] of every token block.
+ * ws, ws_bytes DEVICE workspace of at least lemo_workspace_size(shape) bytes,
+ *              256-byte aligned, contents need no initialisation.
+ *
+ * The score matrix S is never written to memory: the kernel multiplies
+ * Q and K tiles of one head at a time on the tensor cores (tcgen05, fp32
+ * accumulation in tensor memory) and folds each head into the running
+ * positive-part sum in registers; block maxima go to M, and a second pass
+ * sums M's columns in a fixed order (deterministic, no float atomics).
+ */
+LEMO_API lemo_status lemo_score_blocks(const lemo_shape* shape, const uint16_t* q, const uint16_t* k,
+                              float scale, float* block_max, float* block_scores,
+                              void* ws, size_t ws_bytes, lemo_stream stream);
+
+/*
+ * Threshold comparison and compaction of kept token ids (steps a4-a5).
+ *
+ * Jenga summary, section 4.2.1, "Layer-specific Threshold": the score of each
+ * token block is compared with the layer's threshold and all tokens of the
+ * block are retained or eliminated together.  Compaction lists the kept
+ * tokens in their original order (the selective load of section 4.2.3 reads
+ * them from their original positions).
+ *
+ *   block_mask[g] = (block_scores[g] >= threshold)       (NaN scores: 0)
+ *   kept_idx      = ascending global row ids of tokens whose block is kept
+ *   cu_kept[s]    = number of kept tokens in sequences 0..s-1; cu_kept[batch] = K
+ *   *kept_total   = K
+ *
+ * block_scores DEVICE fp32 [total_blocks] (e.g. from lemo_score_blocks).
+ * block_mask   DEVICE uint8 [total_blocks].
+ * kept_idx     DEVICE int32 with room for total_L entries (worst case); only
+ *              the first K are written.
+ * cu_kept      DEVICE int32 [batch+1].   kept_total  DEVICE int32 [1].
+ * ws, ws_bytes as for lemo_score_blocks.
+ *
+ * One pass: warp ballots and a block-wide scan count kept tokens per tile of
+ * 2048 tokens, and a decoupled look-back over tile descriptors in the
+ * workspace chains the tiles' offsets.  Tiles take ids from an atomic ticket,
+ * so a tile only ever waits on tiles that are already running; each wait is
+ * bounded in time and reports LEMO_ERR_TIMEOUT through lemo_get_error.
+ * K stays on the device: nothing is copied to the host.
+ */
+LEMO_API lemo_status lemo_select(const lemo_shape* shape, const float* block_scores, float threshold,
+                        uint8_t* block_mask, int32_t* kept_idx, int32_t* cu_kept,
+                        int32_t* kept_total, void* ws, size_t ws_bytes, lemo_stream stream);
+
+/*
+ * Gather of kept rows into a zero-padded dense buffer (step a6).
+ *
+ * Jenga summary, section 4.2.3, "Permutation-free Token Movement" ->
+ * "Selective Load": kept tokens are read straight from their original rows;
+ * the zero padding of the naive path becomes a zero tail.
+ *
+ *   for r < K:            y[r, 0:d] = x[kept_idx[r], 0:d]   (bit copy)
+ *   for K <= r < K_pad:   y[r, 0:d] = 0                     (K_pad = K rounded up to pad_to)
+ *
+ * x          DEVICE bf16, x_rows rows of stride ld_x elements.
+ * d          row width in elements, d % 8 == 0.
+ * kept_idx   DEVICE int32 [>= K], each in [0, x_rows) (checked on device).
+ * kept_total DEVICE int32 [1] holding K (read on the device).
+ * pad_to     >= 1.
+ * y          DEVICE bf16, y_rows_capacity rows of stride ld_y; rows >= K_pad
+ *            are not touched.  If K_pad > y_rows_capacity, only the first
+ *            y_rows_capacity rows are written and LEMO_ERR_CAPACITY is
+ *            recorded.  Size y for round_up(total_L, pad_to) rows to never
+ *            need K on the host.
+ * Pointers 16-byte aligned; ld_x, ld_y >= d and multiples of 8; x and y
+ * must not overlap.
+ */
+LEMO_API lemo_status lemo_gather_pad(const uint16_t* x, int64_t ld_x, int64_t x_rows, int32_t d,
+                            const int32_t* kept_idx, const int32_t* kept_total, int32_t pad_to,
+                            uint16_t* y, int64_t ld_y, int64_t y_rows_capacity,
+                            lemo_stream stream);
+
+/*
+ * Scatter-back fused with the residual add, in place (step a7).
+ *
+ * Jenga summary, section 4.2.3, "In-place Addition": the sublayer output is
+ * added directly into the original input rows, which completes the padding
+ * (eliminated rows are simply not touched) and the residual add in one step.
+ *
+ *   for r < K:  x[kept_idx[r], 0:d] = bf16_rne(float(x[kept_idx[r], :]) + float(y[r, :]))
+ *   every other row of x keeps its bytes; rows of y at or beyond K are not read.
+ *
+ * The fp32 sum of two bf16 values rounded once to bf16 (nearest, ties to
+ * even) equals the exactly rounded sum, so the result is bit-exact.
+ * kept_idx entries must be distinct (lemo_select produces ascending ids) and
+ * in [0, x_rows) (checked on device).  x and y must not overlap.  Alignment
+ * and stride rules as for lemo_gather_pad.
+ */
+LEMO_API lemo_status lemo_scatter_residual(uint16_t* x, int64_t ld_x, int64_t x_rows, int32_t d,
+                                  const uint16_t* y, int64_t ld_y, const int32_t* kept_idx,
+                                  const int32_t* kept_total, lemo_stream stream);
+
+/*
+ * Synchronises `stream`, then reports and clears the device error word of the
+ * current device: LEMO_OK, LEMO_ERR_INVALID_ARG (cu_seqlens or an index
+ * failed a device-side check), LEMO_ERR_CAPACITY, LEMO_ERR_TIMEOUT, or
+ * LEMO_ERR_CUDA if the stream itself reported an error.
+ */
+LEMO_API lemo_status lemo_get_error(lemo_stream stream);
+
+/*
+ * Test hooks (process-wide, not thread-safe; for the library's own tests).
+ * select_skip_publish_tile >= 0 makes that compaction tile withhold its
+ * look-back descriptor so the tiles after it exhaust their bounded wait;
+ * -1 disables it.  spin_limit_ns bounds every device-side wait
+ * (0 restores the default of 2 s).
+ */
+LEMO_API void lemo_set_test_hooks(int32_t select_skip_publish_tile, int64_t spin_limit_ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LEMO_H */

@@ -1,0 +1,73 @@
+"""GPU parity at the full workload sizes, in the launch configuration the
+benchmark times (one Layer per layer, default grids), against oracle values
+stored by tests/golden/make_golden.py (oracle-only script) and against block
+rows the oracle recomputes live.
+
+The stored files carry sha256 digests of the generated inputs; a mismatch
+means the generator drifted and the stored values no longer apply.
+"""
+
+import json
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from contextual_token_sparsity_b200 import lemo, synth
+from gpu_common import BAND, assert_scores_close, check_mask, check_movement, run_layer
+
+pytestmark = pytest.mark.gpu
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def cuda_ready():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import __graft_entry__
+    __graft_entry__.build()
+    torch.cuda.set_device(0)
+    lemo.lemo_set_test_hooks(-1, 0)
+
+
+def _golden(key):
+    path = os.path.join(GOLDEN, f"{key}.json")
+    if not os.path.exists(path):
+        pytest.skip(f"no stored oracle values for {key}")
+    with open(path) as f:
+        return json.load(f)
+
+
+CASES = [("c2", 0), ("c4", 0), ("c3", 0), ("c3", 1), ("c3", 2), ("c5", 0)]
+
+
+@pytest.mark.parametrize("key,layer", CASES, ids=[f"{k}-layer{l}" for k, l in CASES])
+def test_full_config(key, layer):
+    w = synth.WORKLOADS[key]
+    g = _golden(key)["layers"][layer]
+    inp = synth.make_workload(key, layer)
+    assert synth.digest(inp["q"], inp["k"], inp["cu_seqlens"]) == g["digest_qk"]
+    assert synth.digest(inp["x"], inp["y_out"]) == g["digest_x"]
+    s_ref = np.array([float(v) for v in g["scores"]])
+    theta = float(g["theta"])
+    cu = inp["cu_seqlens"]
+
+    res = run_layer(w.lengths, w.H, w.dh, w.block, w.d, inp["q"], inp["k"], inp["x"],
+                    inp["y_out"], theta)
+    assert_scores_close(res["scores"], s_ref)
+    banded = check_mask(res, s_ref, theta)
+    assert int(res["mask"].sum()) == g["kept_blocks"] or banded > 0
+    check_movement(res, cu, w.block, inp["x"], inp["y_out"], 128)
+
+    # live oracle on sampled query-block rows of block_max (first, middle, last)
+    q = oracle.bf16_bits_to_f64(inp["q"]).reshape(-1, w.H, w.dh)
+    k = oracle.bf16_bits_to_f64(inp["k"]).reshape(-1, w.H, w.dh)
+    s = len(w.lengths) - 1 if len(w.lengths) > 1 else 0
+    Qs, Ks = q[cu[s]:cu[s + 1]], k[cu[s]:cu[s + 1]]
+    nb = -(-int(cu[s + 1] - cu[s]) // w.block)
+    for n in sorted({0, nb // 2, nb - 1}):
+        row = oracle.block_max_row(Qs, Ks, n, w.block)
+        assert_scores_close(res["M"][s][n, : n + 1], row, f"block_max row {n}")
