@@ -1,0 +1,600 @@
+"""Throughput of the contextual-token-sparsity hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lemo|reference]
+                    [--workload c3]
+
+One step is one pass of the whole path - block scores, threshold, compaction,
+gather, scatter with residual add - over every layer of the workload (default:
+three Llama-2-7B layers at L = 16384, H = 32, dh = 128, b = 64, d = 4096 with
+keep ratios 30/50/70 %).  The metric is tokens per second per layer: layers x
+tokens / step time.  Inputs are seeded synthetic data already resident in HBM
+when the timed region starts; each step streams ~1 GB of Q/K/residual rows,
+far more than the 126 MB L2, so L2 is not flushed between steps.
+
+Prints ONE JSON line (rank 0).  With --gpus N > 1 (under torchrun) every rank
+runs its own copy of the workload (independent layers, no collective on the
+data path: weak scaling); the step time is the maximum over ranks.
+
+``--impl reference`` times the CPU oracle (float64 numpy, the repository's
+correctness reference) on a bounded sample of the same workload, as the
+reference arm.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "tokens/sec per layer (score+select+gather+scatter) and % of roofline"
+UNIT = "tokens/s"
+PAD_TO = 128
+LAUNCHES_PER_LAYER = 7  # plan+score+colsum, plan+select, gather, scatter
+SCORE_SOURCES = ["score.cuh", "common.cuh", "tile_plan.h"]
+
+
+# ----------------------------------------------------------------------------
+# ranks
+# ----------------------------------------------------------------------------
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world: int, backend: str):
+    import datetime
+
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=300))
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Maximum of a float over all ranks (identity for one rank)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, max_seconds: float) -> float:
+    """Units processed by all ranks divided by the slowest rank's time."""
+    return units_per_rank * world / max_seconds
+
+
+def barrier(world: int, local: int, cuda: bool = True):
+    if world > 1:
+        import torch.distributed as dist
+        if cuda:
+            dist.barrier(device_ids=[local])
+        else:
+            dist.barrier()
+
+
+# ----------------------------------------------------------------------------
+# algorithmic work of the path (per layer)
+# ----------------------------------------------------------------------------
+
+def score_flops(lengths, H, dh) -> float:
+    """2 flops per multiply-add over the causal pairs i > j of every sequence."""
+    return float(sum(H * dh * L * (L - 1) for L in lengths))
+
+
+def move_bytes(K: int, d: int, pad_to: int = PAD_TO):
+    K_pad = -(-K // pad_to) * pad_to
+    gather = 4 * K * d + 2 * (K_pad - K) * d + 4 * K
+    scatter = 6 * K * d + 4 * K
+    return gather, scatter
+
+
+def select_bytes(total_L: int, nblocks: int, K: int, batch: int) -> int:
+    return 4 * nblocks + nblocks + 4 * K + 4 * (batch + 1) * 2 + 4
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def score_source_digest() -> str:
+    h = hashlib.sha256()
+    for name in SCORE_SOURCES:
+        with open(os.path.join(ROOT, "contextual_token_sparsity_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per scorer launch from a committed ncu summary, if it was
+    taken on the current scorer source (else None)."""
+    path = os.path.join(ROOT, "profiles", f"score_tiles_{workload}.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        p = json.load(f)
+    if p.get("source_digest") != score_source_digest():
+        return None
+    return p.get("dram_bytes_per_launch")
+
+
+def thresholds(key: str, layers: int):
+    """Per-layer thresholds stored by the oracle-only golden script."""
+    path = os.path.join(ROOT, "tests", "golden", f"{key}.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        g = json.load(f)
+    return [float(g["layers"][l]["theta"]) for l in range(layers)]
+
+
+# ----------------------------------------------------------------------------
+# clocks
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples of one GPU (every 100 ms)."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index  # nvidia-smi id: a GPU UUID or an index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"lemo_clocks_{os.getpid()}_{index}.csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.fh,
+                stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) == 8:
+                    rows.append(parts)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        if not rows:
+            return None
+
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return float("nan")
+        sm = [num(r[0]) for r in rows]
+        mx = [num(r[1]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower() == "active"})
+        loaded = [s for s in sm if not math.isnan(s)]
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "samples": len(rows),
+                "power_w_max": max(num(r[2]) for r in rows),
+                "reasons": reasons}
+
+
+# ----------------------------------------------------------------------------
+# the GPU arm
+# ----------------------------------------------------------------------------
+
+def run_lemo(args):
+    import torch
+
+    from contextual_token_sparsity_b200 import lemo, synth
+    from contextual_token_sparsity_b200.pipeline import Layer, to_device_bf16
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    init_dist(world, "nccl")
+    dev = torch.device("cuda", local)
+    lemo.load()
+
+    w = synth.WORKLOADS[args.workload]
+    nl = w.layers
+    thetas = thresholds(args.workload, nl)
+    theta_src = "oracle scores (tests/golden)"
+
+    # inputs: per layer Q, K and sublayer output; one residual stream x
+    host = [synth.make_workload(args.workload, l, with_x=True) for l in range(nl)]
+    layers = [Layer(w.lengths, w.H, w.dh, w.block, w.d, pad_to=PAD_TO, device=dev)
+              for _ in range(nl)]
+    q = [to_device_bf16(h["q"], dev) for h in host]
+    k = [to_device_bf16(h["k"], dev) for h in host]
+    y_out = [to_device_bf16(h["y_out"], dev) for h in host]
+    x0 = to_device_bf16(host[0]["x"], dev)
+    x = x0.clone()
+    if thetas is None:  # no stored oracle thresholds: derive from this GPU's scores
+        thetas = []
+        for l in range(nl):
+            s = layers[l].score(q[l], k[l]).cpu().numpy()[: layers[l].total_blocks]
+            srt = np.sort(s.astype(np.float64))[::-1]
+            kk = int(math.floor(w.keep[l] * srt.size + 0.5))
+            thetas.append(float(0.5 * (srt[kk - 1] + srt[kk])))
+        theta_src = "keep ratio on GPU scores"
+    stream = torch.cuda.current_stream(dev)
+
+    comp = ("score", "select", "gather", "scatter")
+
+    def step(evs=None):
+        for l in range(nl):
+            L_ = layers[l]
+            if evs is not None:
+                evs[l][0].record(stream)
+            L_.score(q[l], k[l])
+            if evs is not None:
+                evs[l][1].record(stream)
+            L_.select(thetas[l])
+            if evs is not None:
+                evs[l][2].record(stream)
+            L_.gather(x)
+            if evs is not None:
+                evs[l][3].record(stream)
+            L_.scatter(x, y_out[l])
+            if evs is not None:
+                evs[l][4].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = lemo.lemo_get_error()
+    if st != lemo.LEMO_OK:
+        raise RuntimeError(f"device error during warm-up: {lemo.STATUS.get(st, st)}")
+    kept = [int(L_.kept_total.item()) for L_ in layers]
+
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        gpu_id = str(local)
+    clocks = ClockSampler(gpu_id)
+    clocks.start()
+    time.sleep(0.3)
+    ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(nl)]
+          for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    barrier(world, local)
+    torch.cuda.synchronize()
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(ev[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world, local)
+    elapsed_s = t_start.elapsed_time(t_end) / 1e3
+    clk = clocks.stop()
+    st = lemo.lemo_get_error()
+    if st != lemo.LEMO_OK:
+        raise RuntimeError(f"device error in timed region: {lemo.STATUS.get(st, st)}")
+    max_s = max_over_ranks(elapsed_s, world, dev)
+
+    comp_ms = {c: [] for c in comp}
+    for i in range(args.steps):
+        for l in range(nl):
+            for ci, c in enumerate(comp):
+                comp_ms[c].append(ev[i][l][ci].elapsed_time(ev[i][l][ci + 1]))
+    avg_us = {c: 1e3 * statistics.fmean(v) for c, v in comp_ms.items()}
+
+    tokens_per_step = nl * w.total_L
+    value = whole_job_rate(tokens_per_step, world, max_s / args.steps)
+
+    # roofline of the dominant kernel (the scorer: dense contraction -> tensor)
+    peaks = load_peaks()
+    F = score_flops(w.lengths, w.H, w.dh)
+    score_s = avg_us["score"] / 1e6
+    long_region = elapsed_s > 2.0
+    peak_tf = peaks["bf16_tflops_sustained"] if long_region else peaks["bf16_tflops"]
+    achieved_tf = F / score_s / 1e12
+    traffic = profiled_traffic(args.workload)
+    roofline = {"bound": "tensor", "kernel": "score_tiles_kernel (+plan, column sum)",
+                "achieved": round(achieved_tf, 1), "peak": peak_tf, "unit": "TFLOP/s",
+                "frac": round(achieved_tf / peak_tf, 4), "traffic": traffic,
+                "peak_source": f"{peaks['source']} bf16 "
+                               f"{'sustained' if long_region else 'burst'} cuBLAS GEMM",
+                "algorithmic_flops_per_launch": F}
+    # whole-path roofline: scorer at the tensor peak + movement at HBM bandwidth
+    bw = peaks["hbm_gbs"] * 1e9
+    movement = []
+    t_roof = 0.0
+    for l in range(nl):
+        g_b, s_b = move_bytes(kept[l], w.d)
+        sel_b = select_bytes(w.total_L, layers[l].total_blocks, kept[l], len(w.lengths))
+        t_roof += F / (peak_tf * 1e12) + (g_b + s_b + sel_b) / bw
+        movement.append({"K": kept[l], "gather_bytes": g_b, "scatter_bytes": s_b})
+    gather_gbs = statistics.fmean(
+        move_bytes(kept[l], w.d)[0] for l in range(nl)) / (avg_us["gather"] / 1e6) / 1e9
+    scatter_gbs = statistics.fmean(
+        move_bytes(kept[l], w.d)[1] for l in range(nl)) / (avg_us["scatter"] / 1e6) / 1e9
+    step_s = max_s / args.steps
+
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(step_s * 1e3, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{args.workload}: {w.name}", "layers": nl,
+                   "seq_lens": list(w.lengths), "heads": w.H, "head_dim": w.dh,
+                   "block": w.block, "d": w.d, "keep": list(w.keep), "kept_tokens": kept,
+                   "thresholds": thetas, "threshold_source": theta_src, "pad_to": PAD_TO,
+                   "l2": "not flushed; each step streams "
+                         f"{(nl * (2 * w.total_L * w.H * w.dh * 2) + 3 * w.total_L * w.d * 2) / 1e9:.2f}"
+                         " GB of Q/K/residual rows (> 126 MB L2)",
+                   "parallelism": f"{world} independent replica(s), no collective"},
+        "roofline": roofline,
+        "path_roofline": {"frac": round(t_roof / step_s, 4),
+                          "roofline_ms_per_step": round(t_roof * 1e3, 4),
+                          "model": "scorer flops at the bf16 peak + select/gather/scatter "
+                                   "bytes at the HBM copy bandwidth"},
+        "kernels_us": {c: round(v, 2) for c, v in avg_us.items()},
+        "movement": {"gather_gbs": round(gather_gbs, 1), "scatter_gbs": round(scatter_gbs, 1),
+                     "hbm_peak_gbs": peaks["hbm_gbs"],
+                     "gather_frac": round(gather_gbs / peaks["hbm_gbs"], 4),
+                     "scatter_frac": round(scatter_gbs / peaks["hbm_gbs"], 4)},
+        "gpu_launches": LAUNCHES_PER_LAYER * nl * args.steps,
+        "clocks": clk,
+    }
+
+    # end to end through the C ABI with host buffers: H2D of each layer's
+    # Q/K/sublayer output and of the residual, the path, D2H of the residual
+    # and of the block scores, every step.
+    if not args.no_e2e:
+        out["e2e"] = run_e2e(args, host, layers, thetas, dev, world, local, tokens_per_step)
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(args.workload, budget_s=args.cpu_seconds)
+
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def run_e2e(args, host, layers, thetas, dev, world, local, tokens_per_step):
+    import torch
+    nl = len(layers)
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).pin_memory()  # noqa
+    hq = [pin(h["q"]) for h in host]
+    hk = [pin(h["k"]) for h in host]
+    hy = [pin(h["y_out"]) for h in host]
+    hx = pin(host[0]["x"])
+    hx_out = torch.empty_like(hx).pin_memory()
+    hs_out = [torch.empty(L_.block_scores.numel(), dtype=torch.float32).pin_memory()
+              for L_ in layers]
+    dq = [torch.empty(t.shape, dtype=torch.int16, device=dev) for t in hq]
+    dk = [torch.empty(t.shape, dtype=torch.int16, device=dev) for t in hk]
+    dy = [torch.empty(t.shape, dtype=torch.int16, device=dev) for t in hy]
+    dx = torch.empty(hx.shape, dtype=torch.int16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    h2d = sum(t.numel() * 2 for t in hq + hk + hy) + hx.numel() * 2
+    d2h = hx_out.numel() * 2 + sum(t.numel() * 4 for t in hs_out)
+
+    def step():
+        dx.copy_(hx, non_blocking=True)
+        for l in range(nl):
+            dq[l].copy_(hq[l], non_blocking=True)
+            dk[l].copy_(hk[l], non_blocking=True)
+            dy[l].copy_(hy[l], non_blocking=True)
+            L_ = layers[l]
+            L_.step(dq[l].view(torch.bfloat16), dk[l].view(torch.bfloat16), thetas[l],
+                    dx.view(torch.bfloat16), dy[l].view(torch.bfloat16))
+            hs_out[l].copy_(L_.block_scores, non_blocking=True)
+        hx_out.copy_(dx, non_blocking=True)
+
+    steps = max(3, min(args.steps, args.e2e_steps))
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    barrier(world, local)
+    torch.cuda.synchronize()
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    barrier(world, local)
+    s = max_over_ranks(a.elapsed_time(b) / 1e3, world, dev)
+    return {"value": round(whole_job_rate(tokens_per_step, world, s / steps), 1), "unit": UNIT,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
+            "ms_per_step": round(1e3 * s / steps, 3),
+            "path": "pinned host -> device copies, lemo_* calls, device -> pinned host copies"}
+
+
+# ----------------------------------------------------------------------------
+# the CPU oracle (cpu_baseline leg and reference arm)
+# ----------------------------------------------------------------------------
+
+def blas_threads() -> int:
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        n = [i.get("num_threads", 1) for i in info if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return 1
+
+
+class OracleSample:
+    """The CPU oracle on a bounded sample of one layer, scaled to tokens/s.
+
+    The oracle scores one query-block row at a time; a sample is a set of
+    query-block rows drawn at random until a time budget is spent.  A row's
+    cost is proportional to its number of key blocks (n + 1), so the full
+    layer's scoring time is the sample time times (all block pairs / sampled
+    block pairs).  Selection, compaction, gather and scatter run in full.
+    """
+
+    def __init__(self, key: str, layer: int = 0):
+        import oracle
+        from contextual_token_sparsity_b200 import synth
+        self.oracle = oracle
+        self.key, self.layer = key, layer
+        self.w = w = synth.WORKLOADS[key]
+        self.inp = inp = synth.make_workload(key, layer, with_x=True)
+        cu = inp["cu_seqlens"]
+        s = int(np.argmax(w.lengths))  # sample rows from the longest sequence
+        L = w.lengths[s]
+        self.q = oracle.bf16_bits_to_f64(inp["q"][cu[s]:cu[s + 1]]).reshape(L, w.H, w.dh)
+        self.k = oracle.bf16_bits_to_f64(inp["k"][cu[s]:cu[s + 1]]).reshape(L, w.H, w.dh)
+        self.nb = -(-L // w.block)
+        self.all_pairs = sum((-(-Ls // w.block)) * ((-(-Ls // w.block)) + 1) // 2
+                             for Ls in w.lengths)
+        self.t_rest = None
+
+    def time_rows(self, budget_s: float, seed: int):
+        order = np.random.default_rng(seed).permutation(self.nb)
+        t0 = time.perf_counter()
+        pairs = rows = 0
+        for n in order:
+            self.oracle.block_max_row(self.q, self.k, int(n), self.w.block)
+            pairs += int(n) + 1
+            rows += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
+        t = time.perf_counter() - t0
+        return t * self.all_pairs / pairs, rows, pairs, t
+
+    def time_rest(self):
+        """select + compact + gather + scatter of the layer, in full."""
+        if self.t_rest is None:
+            o, w, inp = self.oracle, self.w, self.inp
+            gpath = os.path.join(ROOT, "tests", "golden", f"{self.key}.json")
+            if os.path.exists(gpath):
+                with open(gpath) as f:
+                    g = json.load(f)["layers"][self.layer]
+                sc = np.array([float(v) for v in g["scores"]])
+                theta = float(g["theta"])
+            else:
+                sc = np.linspace(1.0, 0.0, sum(-(-Ls // w.block) for Ls in w.lengths))
+                theta = 0.5
+            t1 = time.perf_counter()
+            mask = o.keep_mask(sc, theta)
+            idx, _, _ = o.compact(mask, inp["cu_seqlens"], w.block)
+            o.gather_pad(inp["x"], idx, PAD_TO)
+            o.scatter_residual(inp["x"], inp["y_out"], idx)
+            self.t_rest = time.perf_counter() - t1
+        return self.t_rest
+
+    def describe(self, rows, pairs, t_rows):
+        return (f"layer {self.layer} of {self.key}: {rows} of {self.nb} query-block rows "
+                f"({pairs} of {self.all_pairs} block pairs, {t_rows:.1f} s) scored by the "
+                f"oracle and scaled by block pairs; select/compact/gather/scatter timed in "
+                f"full ({self.t_rest:.1f} s); float64 numpy, BLAS on all cores, elementwise "
+                f"work single-threaded")
+
+
+def cpu_baseline(key: str, budget_s: float = 20.0, layer: int = 0):
+    smp = OracleSample(key, layer)
+    t_rest = smp.time_rest()
+    t_score, rows, pairs, t_rows = smp.time_rows(budget_s, seed=0)
+    t_layer = t_score + t_rest
+    return {"value": round(smp.w.total_L / t_layer, 3), "unit": UNIT, "cores": blas_threads(),
+            "kind": "oracle", "sample": smp.describe(rows, pairs, t_rows),
+            "seconds_per_layer_estimate": round(t_layer, 2)}
+
+
+def run_reference(args):
+    world, rank, local = dist_env()
+    if rank != 0:
+        return  # the reference arm runs on rank 0 only
+    smp = OracleSample(args.workload, 0)
+    w = smp.w
+    t_rest = smp.time_rest()
+    per_step = max(0.3, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    vals, desc = [], ""
+    for i in range(args.warmup + args.steps):
+        t_score, rows, pairs, t_rows = smp.time_rows(per_step, seed=i)
+        if i >= args.warmup:
+            vals.append(t_score + t_rest)
+            desc = smp.describe(rows, pairs, t_rows)
+    t_layer = statistics.fmean(vals)
+    value = w.total_L / t_layer
+    out = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(t_layer * w.layers * 1e3, 1), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "impl": "reference",
+        "config": {"workload": f"{args.workload}: {w.name}", "layers": w.layers,
+                   "seq_lens": list(w.lengths), "heads": w.H, "head_dim": w.dh,
+                   "block": w.block, "d": w.d, "keep": list(w.keep),
+                   "parallelism": "CPU oracle, rank 0 only"},
+        "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": blas_threads(),
+                         "kind": "oracle", "sample": f"per step: {desc}"},
+        "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description="contextual token sparsity hot-path benchmark")
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["lemo", "reference"], default="lemo")
+    ap.add_argument("--workload", default="c3", choices=["c1", "c2", "c3", "c4", "c5"])
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world = dist_env()[0]
+    if args.gpus != world and world > 1:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_lemo(args)
+
+
+if __name__ == "__main__":
+    main()
