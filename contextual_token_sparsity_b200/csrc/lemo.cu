@@ -22,7 +22,6 @@ constexpr int64_t kDefaultSpinNs = 2000000000LL;
 
 std::mutex g_mu;
 int g_sms[kMaxDevices];              // 0 = not queried yet
-bool g_score_attr[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 int g_skip_publish_tile = -1;
 int64_t g_spin_ns = kDefaultSpinNs;
@@ -93,18 +92,58 @@ void launch_plan(const lemo_shape* s, char* ws, const lemo::WsLayout& lay, int32
                                           s->block, ws, lay, zero_word);
 }
 
-bool encode_rows(CUtensorMap* tm, const uint16_t* base, int64_t rows, int64_t width,
-                 uint32_t box_rows) {
+// 3-D view of a [rows, H*dh] bf16 matrix as (64 elements, rows, H*dh/64
+// slices of 64), so that one box (64, box_rows, dh/64) fetches one head of
+// box_rows rows as dh/64 consecutive 128-byte-swizzled K-major tiles.
+bool encode_heads(CUtensorMap* tm, const uint16_t* base, int64_t rows, int64_t width, int dh,
+                  uint32_t box_rows) {
     PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
     if (!enc) return false;
-    const cuuint64_t dims[2] = {(cuuint64_t)width, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)(width * 2)};
-    const cuuint32_t box[2] = {(cuuint32_t)lemo::score::KB, box_rows};
-    const cuuint32_t estr[2] = {1, 1};
-    return enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(base), dims,
+    const cuuint64_t dims[3] = {(cuuint64_t)lemo::score::KB, (cuuint64_t)rows,
+                                (cuuint64_t)(width / lemo::score::KB)};
+    const cuuint64_t strides[2] = {(cuuint64_t)(width * 2), (cuuint64_t)(lemo::score::KB * 2)};
+    const cuuint32_t box[3] = {(cuuint32_t)lemo::score::KB, box_rows,
+                               (cuuint32_t)(dh / lemo::score::KB)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(base), dims,
                strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
            CUDA_SUCCESS;
+}
+
+// CTA pairs of the scoring kernel that fit on the device at once (one
+// persistent wave).  Sets the kernel's shared-memory limit on first use.
+int g_score_pairs[kMaxDevices];
+
+int score_pairs(int dev, int sms) {
+    namespace sc = lemo::score;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_score_pairs[dev] == 0) {
+        if (cudaFuncSetAttribute(sc::score_tiles_kernel,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 sc::SMEM_BYTES) != cudaSuccess)
+            return 0;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
+        cfg.blockDim = dim3(sc::THREADS, 1, 1);
+        cfg.dynamicSmemBytes = sc::SMEM_BYTES;
+        cudaLaunchAttribute attr;
+        attr.id = cudaLaunchAttributeClusterDimension;
+        attr.val.clusterDim.x = 2;
+        attr.val.clusterDim.y = 1;
+        attr.val.clusterDim.z = 1;
+        cfg.attrs = &attr;
+        cfg.numAttrs = 1;
+        int clusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&clusters, sc::score_tiles_kernel, &cfg) !=
+                cudaSuccess ||
+            clusters < 1) {
+            cudaGetLastError();
+            clusters = sms / 2;
+        }
+        g_score_pairs[dev] = clusters < sms / 2 ? clusters : sms / 2;
+    }
+    return g_score_pairs[dev];
 }
 
 // Persistent grid of the row-copy kernels: as many CTAs as fit on the SMs
@@ -193,19 +232,11 @@ lemo_status lemo_score_blocks(const lemo_shape* shape, const uint16_t* q, const 
         namespace sc = lemo::score;
         CUtensorMap tm_q, tm_k;
         const int64_t width = (int64_t)shape->H * shape->dh;
-        if (!encode_rows(&tm_q, q, shape->total_L, width, sc::BM) ||
-            !encode_rows(&tm_k, k, shape->total_L, width, sc::BN))
+        if (!encode_heads(&tm_q, q, shape->total_L, width, shape->dh, sc::ROWS) ||
+            !encode_heads(&tm_k, k, shape->total_L, width, shape->dh, sc::ROWS))
             return LEMO_ERR_CUDA;
-        {
-            std::lock_guard<std::mutex> lk(g_mu);
-            if (!g_score_attr[dev]) {
-                if (cudaFuncSetAttribute(sc::score_tiles_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         sc::SMEM_BYTES) != cudaSuccess)
-                    return LEMO_ERR_CUDA;
-                g_score_attr[dev] = true;
-            }
-        }
+        const int pairs = score_pairs(dev, sms);
+        if (pairs <= 0) return LEMO_ERR_CUDA;
         sc::Args a;
         a.cu = shape->cu_seqlens;
         a.batch = shape->batch;
@@ -217,9 +248,14 @@ lemo_status lemo_score_blocks(const lemo_shape* shape, const uint16_t* q, const 
         a.ws = w;
         a.lay = lay;
         a.spin_limit_ns = (uint64_t)g_spin_ns;
-        sc::score_tiles_kernel<<<sms, sc::THREADS, sc::SMEM_BYTES, st>>>(tm_q, tm_k, a);
+        sc::score_tiles_kernel<<<2 * pairs, sc::THREADS, sc::SMEM_BYTES, st>>>(tm_q, tm_k, a);
         if ((e = launch_status()) != LEMO_OK) return e;
-        sc::column_sum_kernel<<<sms, 256, 0, st>>>(mblk, w, lay, shape->batch, block_scores);
+        // one warp per token block; the host knows an upper bound of their number
+        const int64_t nb_bound =
+            ((int64_t)shape->total_L + (int64_t)shape->batch * (shape->block - 1)) / shape->block;
+        const int64_t cs_ctas = (nb_bound + 7) / 8;
+        const int cs_grid = (int)(cs_ctas < (int64_t)sms * 8 ? (cs_ctas > 0 ? cs_ctas : 1) : sms * 8);
+        sc::column_sum_kernel<<<cs_grid, 256, 0, st>>>(mblk, w, lay, shape->batch, block_scores);
         if ((e = launch_status()) != LEMO_OK) return e;
     }
     return LEMO_OK;

@@ -136,31 +136,32 @@ TILE_CHECK = r"""
 #include "tile_plan.h"
 using namespace lemo_plan;
 int main() {
-  const int Ls[] = {1, 2, 63, 64, 65, 127, 128, 129, 255, 256, 257, 300, 1000, 1024, 2047,
-                    3072, 4096, 8192, 16384, 32768};
+  const int Ls[] = {1, 2, 63, 64, 65, 127, 128, 129, 255, 256, 257, 300, 511, 512, 513, 1000,
+                    1024, 2047, 2049, 3072, 4096, 8192, 16384, 32768};
   for (int L : Ls) {
     const int nq = (int)query_tiles(L);
     const long long T = seq_tiles(L);
     long long brute = 0;
-    for (int q = 0; q < nq; ++q) brute += q / 2 + 1;
+    for (int q = 0; q < nq; ++q)
+      for (int k = 0; k * TN <= q * TM + TM - 1; ++k) ++brute;
     if (brute != T) { printf("count L=%d %lld %lld\n", L, T, brute); return 1; }
-    std::vector<int> seen((size_t)nq * (nq / 2 + 1), 0);
+    std::vector<int> seen((size_t)nq * nq, 0);
     int prev_group = -1;
     for (long long t = 0; t < T; ++t) {
       int qi, kj; decode_tile(L, t, &qi, &kj);
-      if (qi < 0 || qi >= nq || kj < 0 || kj > qi / 2) { printf("range L=%d t=%lld\n", L, t); return 1; }
+      if (qi < 0 || qi >= nq || kj < 0 || kj > qi) { printf("range L=%d t=%lld\n", L, t); return 1; }
       int g = qi / GROUP;
       if (g < prev_group) { printf("group order L=%d\n", L); return 1; }
       prev_group = g;
-      if (seen[(size_t)qi * (nq / 2 + 1) + kj]++) { printf("dup L=%d\n", L); return 1; }
+      if (seen[(size_t)qi * nq + kj]++) { printf("dup L=%d\n", L); return 1; }
     }
     for (int b : {64, 128}) {             // every score block n >= m in exactly one tile
       const int nb = (L + b - 1) / b;
       std::vector<int> cov((size_t)nb * nb, 0);
       for (long long t = 0; t < T; ++t) {
         int qi, kj; decode_tile(L, t, &qi, &kj);
-        for (int n = qi * BM / b; n < (qi + 1) * BM / b; ++n)
-          for (int m = kj * BN / b; m < (kj + 1) * BN / b; ++m)
+        for (int n = qi * TM / b; n < (qi + 1) * TM / b; ++n)
+          for (int m = kj * TN / b; m < (kj + 1) * TN / b; ++m)
             if (n < nb && m <= n) cov[(size_t)n * nb + m]++;
       }
       for (int n = 0; n < nb; ++n)
