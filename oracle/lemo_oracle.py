@@ -374,7 +374,7 @@ def predict_scores(q_hat, k_hat, cu_seqlens, block: int, H: int, dh: int):
 def recall(mask_pred, mask_exact) -> float:
     """|kept_pred AND kept_exact| / |kept_exact| (1.0 when nothing is kept).
 
-    The pages report predictor recall ([Jenga] §5, predictor evaluation)
+    The pages report predictor recall ([Jenga] §6.2, Fig. 17(a))
     without a formula; this is the plain reading: the share of exactly-kept
     token blocks that the predicted scores also keep.
     """
