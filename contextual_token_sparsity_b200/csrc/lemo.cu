@@ -296,6 +296,79 @@ lemo_status lemo_select(const lemo_shape* shape, const float* block_scores, floa
     return launch_status();
 }
 
+// ---------------------------------------------------------------------------
+// lemo_select with its scratch in a device array owned by the library (for
+// callers that cannot allocate).  The array is reserved in every GPU's memory
+// when the library is loaded.  Host code must not pass the symbol itself to a
+// kernel - on the host it names a host-side stand-in - so its device address
+// is looked up once per device (with that device current) and cached.
+// ---------------------------------------------------------------------------
+}  // extern "C"
+
+namespace {
+constexpr int32_t kStaticMaxBatch = 4096;
+constexpr int32_t kStaticMaxTokens = 1 << 24;
+constexpr size_t kStaticScratchBytes = 160 * 1024;
+char* g_static_scratch_dev[kMaxDevices];  // device address of the array, per device
+}  // namespace
+
+static __device__ __align__(256) char g_select_scratch[kStaticScratchBytes];
+
+extern "C" {
+
+lemo_status lemo_select_static_ws(const lemo_shape* shape, const float* block_scores,
+                                  float threshold, uint8_t* block_mask, int32_t* kept_idx,
+                                  int32_t* cu_kept, int32_t* kept_total, lemo_stream stream) {
+    lemo_status e = check_shape(shape, false);
+    if (e != LEMO_OK) return e;
+    if (!block_scores || !block_mask || !kept_idx || !cu_kept || !kept_total)
+        return LEMO_ERR_INVALID_ARG;
+    if (!aligned(block_scores, 4) || !aligned(kept_idx, 4) || !aligned(cu_kept, 4) ||
+        !aligned(kept_total, 4))
+        return LEMO_ERR_INVALID_ARG;
+    if (shape->batch > kStaticMaxBatch || shape->total_L > kStaticMaxTokens)
+        return LEMO_ERR_CAPACITY;
+    const lemo::WsLayout lay = layout_of(shape);
+    if (lay.mblk > kStaticScratchBytes) return LEMO_ERR_CAPACITY;  // selection stops before M
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LEMO_ERR_CUDA;
+    char* w = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!g_static_scratch_dev[dev]) {
+            void* p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_select_scratch) != cudaSuccess || !p) {
+                cudaGetLastError();
+                return LEMO_ERR_CUDA;
+            }
+            g_static_scratch_dev[dev] = static_cast<char*>(p);
+        }
+        w = g_static_scratch_dev[dev];
+    }
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    // The plan kernel re-initialises the look-back descriptors, the ticket and
+    // kept_total at the start of every call.
+    launch_plan(shape, w, lay, kept_total, st);
+    if ((e = launch_status()) != LEMO_OK) return e;
+    lemo::SelectArgs a;
+    a.cu = shape->cu_seqlens;
+    a.batch = shape->batch;
+    a.total_L = shape->total_L;
+    a.block = shape->block;
+    a.scores = block_scores;
+    a.theta = threshold;
+    a.mask = block_mask;
+    a.kept_idx = kept_idx;
+    a.cu_kept = cu_kept;
+    a.kept_total = kept_total;
+    a.ws = w;
+    a.lay = lay;
+    a.skip_publish_tile = g_skip_publish_tile;
+    a.spin_limit_ns = (uint64_t)g_spin_ns;
+    lemo::select_kernel<<<(unsigned)lay.n_lookback, lemo::kSelectThreads, 0, st>>>(a);
+    return launch_status();
+}
+
 lemo_status lemo_gather_pad(const uint16_t* x, int64_t ld_x, int64_t x_rows, int32_t d,
                             const int32_t* kept_idx, const int32_t* kept_total, int32_t pad_to,
                             uint16_t* y, int64_t ld_y, int64_t y_rows_capacity,

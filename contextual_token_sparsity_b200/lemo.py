@@ -53,6 +53,8 @@ _SIGS = {
                                          _P, _P, ctypes.c_size_t, _P]),
     "lemo_select": (ctypes.c_int, [ctypes.POINTER(lemo_shape), _P, ctypes.c_float, _P, _P, _P,
                                    _P, _P, ctypes.c_size_t, _P]),
+    "lemo_select_static_ws": (ctypes.c_int, [ctypes.POINTER(lemo_shape), _P, ctypes.c_float, _P,
+                                             _P, _P, _P, _P]),
     "lemo_gather_pad": (ctypes.c_int, [_P, _I64, _I64, _I32, _P, _P, _I32, _P, _I64, _I64, _P]),
     "lemo_scatter_residual": (ctypes.c_int, [_P, _I64, _I64, _I32, _P, _I64, _P, _P, _P]),
     "lemo_get_error": (ctypes.c_int, [_P]),
@@ -129,6 +131,15 @@ def lemo_select(shape, block_scores, threshold, block_mask, kept_idx, cu_kept, k
                               _ptr(block_mask), _ptr(kept_idx), _ptr(cu_kept), _ptr(kept_total),
                               _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "lemo_select")
+
+
+def lemo_select_static_ws(shape, block_scores, threshold, block_mask, kept_idx, cu_kept,
+                          kept_total, stream=None):
+    """lemo_select with the library's own device scratch (no workspace argument)."""
+    _check(load().lemo_select_static_ws(ctypes.byref(shape), _ptr(block_scores), float(threshold),
+                                        _ptr(block_mask), _ptr(kept_idx), _ptr(cu_kept),
+                                        _ptr(kept_total), _stream(stream)),
+           "lemo_select_static_ws")
 
 
 def lemo_gather_pad(x, kept_idx, kept_total, pad_to, y, stream=None, d=None):

@@ -163,6 +163,34 @@ LEMO_API lemo_status lemo_select(const lemo_shape* shape, const float* block_sco
                         int32_t* kept_total, void* ws, size_t ws_bytes, lemo_stream stream);
 
 /*
+ * lemo_select without a caller-provided workspace.  The paper has no
+ * counterpart to this entry point; it is a deployment variant of lemo_select.
+ *
+ * Some callers cannot allocate device memory where they select tokens: code
+ * running under a memory pool that owns the whole device and forbids further
+ * cudaMalloc calls, or a latency-critical loop that must not pay for the
+ * device-wide synchronisation cudaMalloc/cudaFree can imply.  This call
+ * computes exactly what lemo_select computes (same arguments, outputs and
+ * errors) but keeps its scratch - the per-call plan of the batch and the
+ * look-back descriptors - in a 160 KB array that the library reserves in the
+ * memory of every GPU it is loaded on (held until the process exits).  It
+ * calls no allocating function.
+ *
+ * Limits: batch <= 4096 and total_L <= 16777216; a larger shape returns
+ * LEMO_ERR_CAPACITY and enqueues nothing.
+ * The first call on a device looks up the array's device address with that
+ * device current; make that first call before any stream capture.
+ * Every call on a device uses the same array and re-initialises what must
+ * start at zero at its beginning, so calls that can overlap on the GPU (for
+ * example on two streams with no ordering between them) race and corrupt each
+ * other's results: order them on one stream.
+ */
+LEMO_API lemo_status lemo_select_static_ws(const lemo_shape* shape, const float* block_scores,
+                                           float threshold, uint8_t* block_mask,
+                                           int32_t* kept_idx, int32_t* cu_kept,
+                                           int32_t* kept_total, lemo_stream stream);
+
+/*
  * Gather of kept rows into a zero-padded dense buffer (step a6).
  *
  * Jenga summary, section 4.2.3, "Permutation-free Token Movement" ->
