@@ -130,16 +130,25 @@ def score_source_digest() -> str:
 
 
 def profiled_traffic(workload: str):
-    """DRAM bytes per scorer launch from a committed ncu summary, if it was
-    taken on the current scorer source (else None)."""
-    path = os.path.join(ROOT, "profiles", f"score_tiles_{workload}.json")
-    if not os.path.exists(path):
+    """DRAM bytes per scorer launch from the committed ncu summary
+    (profiles/score_tiles_*.md), if it was taken on the current scorer source
+    (else None)."""
+    path = os.path.join(ROOT, "profiles", "score_tiles_c2.md")
+    if workload != "c3" or not os.path.exists(path):
         return None
+    rec = {}
     with open(path) as f:
-        p = json.load(f)
-    if p.get("source_digest") != score_source_digest():
+        for line in f:
+            line = line.strip()
+            if " = " in line:
+                k, v = line.split(" = ", 1)
+                rec[k.strip()] = v.strip()
+    if rec.get("source_digest") != score_source_digest():
         return None
-    return p.get("dram_bytes_per_launch")
+    try:
+        return int(rec["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
 
 
 def thresholds(key: str, layers: int):

@@ -1,0 +1,64 @@
+"""Multi-rank host logic of bench.py on CPU (gloo, world size 2).
+
+With N ranks every rank runs its own copy of the workload (independent layers,
+no data-path collective).  The only cross-rank step is the timing reduction:
+the step time is the maximum over ranks and the throughput counts every
+rank's tokens.  These tests run that logic in two gloo processes.
+"""
+
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    import datetime
+
+    import torch.distributed as dist
+
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        w, r, l = bench.dist_env()
+        assert (w, r, l) == (world, rank, rank)
+        elapsed = 1.0 + rank  # rank 1 is the slow one
+        bench.barrier(world, l, cuda=False)
+        m = bench.max_over_ranks(elapsed, world, None)
+        rate = bench.whole_job_rate(3 * 16384, world, m)
+        out.put((rank, m, rate))
+        bench.barrier(world, l, cuda=False)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_take_max_time_and_count_all_tokens():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    out = ctx.Queue()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, out)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+    assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+    res = sorted(out.get(timeout=10) for _ in range(world))
+    for rank, m, rate in res:
+        assert m == pytest.approx(2.0)
+        assert rate == pytest.approx(2 * 3 * 16384 / 2.0)
+
+
+def test_single_rank_is_identity():
+    import bench
+    assert bench.max_over_ranks(3.5, 1) == 3.5
+    assert bench.whole_job_rate(100, 1, 2.0) == 50.0
