@@ -11,6 +11,7 @@
 #include "lemo.h"
 #include "common.cuh"
 #include "move.cuh"
+#include "predict.cuh"
 #include "score.cuh"
 #include "select.cuh"
 
@@ -172,6 +173,48 @@ lemo_status check_move(const void* x, int64_t ld_x, int64_t x_rows, int32_t d, c
     if (ld_x < d || ld_y < d || ld_x % 8 != 0 || ld_y % 8 != 0) return LEMO_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(y, 16) || !aligned(kept_idx, 4) || !aligned(kept_total, 4))
         return LEMO_ERR_INVALID_ARG;
+    return LEMO_OK;
+}
+
+// Workspace of lemo_predict_scores: the plan/score layout (its block-score
+// region holds the block products P) followed by the predictor buffers.
+struct PredictLayout {
+    lemo::WsLayout base;
+    size_t xbar, hq, hk, part, qh, kh, total;
+    int64_t tb;      // upper bound of the number of token blocks
+    int splits;      // split-K factor of the first predictor GEMM
+};
+
+PredictLayout predict_layout(const lemo_shape* s, int d, int rank) {
+    PredictLayout p;
+    p.base = layout_of(s);
+    p.tb = ((int64_t)s->total_L + (int64_t)s->batch * (s->block - 1)) / s->block;
+    if (p.tb < 1) p.tb = 1;
+    const int64_t hd = (int64_t)s->H * s->dh;
+    const int64_t tiles = ((rank + 63) / 64) * ((p.tb + 63) / 64);
+    int64_t splits = (296 + tiles - 1) / tiles;  // about two CTAs per SM
+    const int64_t max_splits = (d + 255) / 256;   // at least 256 of K per split
+    if (splits > max_splits) splits = max_splits;
+    if (splits < 1) splits = 1;
+    p.splits = (int)splits;
+    size_t off = p.base.total;
+    p.xbar = off; off = lemo::align_up(off + 4 * (size_t)p.tb * d, 256);
+    p.hq = off;   off = lemo::align_up(off + 4 * (size_t)p.tb * rank, 256);
+    p.hk = off;   off = lemo::align_up(off + 4 * (size_t)p.tb * rank, 256);
+    p.part = off; off = lemo::align_up(off + 4 * (size_t)p.splits * p.tb * rank, 256);
+    p.qh = off;   off = lemo::align_up(off + 4 * (size_t)p.tb * hd, 256);
+    p.kh = off;   off = lemo::align_up(off + 4 * (size_t)p.tb * hd, 256);
+    p.total = off;
+    return p;
+}
+
+lemo_status check_predict(const lemo_shape* s, int d, int rank) {
+    lemo_status e = check_shape(s, false);
+    if (e != LEMO_OK) return e;
+    if (s->H < 1 || s->dh < 1 || d < 1 || rank < 1) return LEMO_ERR_INVALID_ARG;
+    if (d % 8 != 0) return LEMO_ERR_UNSUPPORTED;
+    if (s->dh > 1024 || (int64_t)s->H * s->dh > (1 << 20) || d > (1 << 20) || rank > (1 << 16))
+        return LEMO_ERR_UNSUPPORTED;
     return LEMO_OK;
 }
 
@@ -417,6 +460,76 @@ lemo_status lemo_scatter_residual(uint16_t* x, int64_t ld_x, int64_t x_rows, int
     lemo::scatter_residual_kernel<<<move_grid(dev, sms, 1, lemo::scatter_residual_kernel),
                                     lemo::kMoveThreads, 0,
                                     reinterpret_cast<cudaStream_t>(stream)>>>(a);
+    return launch_status();
+}
+
+size_t lemo_predict_workspace_size(const lemo_shape* shape, int32_t d, int32_t rank) {
+    if (check_predict(shape, d, rank) != LEMO_OK) return 0;
+    return predict_layout(shape, d, rank).total;
+}
+
+lemo_status lemo_predict_scores(const lemo_shape* shape, int32_t d, const uint16_t* x,
+                                int64_t ld_x, const uint16_t* w1q, const uint16_t* w2q,
+                                const uint16_t* w1k, const uint16_t* w2k, int32_t rank,
+                                float* block_scores, void* ws, size_t ws_bytes,
+                                lemo_stream stream) {
+    namespace pr = lemo::predict;
+    lemo_status e = check_predict(shape, d, rank);
+    if (e != LEMO_OK) return e;
+    if (!x || !w1q || !w2q || !w1k || !w2k || !block_scores || !ws) return LEMO_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || ld_x < d || ld_x % 8 != 0 || !aligned(w1q, 2) || !aligned(w2q, 2) ||
+        !aligned(w1k, 2) || !aligned(w2k, 2) || !aligned(block_scores, 4) || !aligned(ws, 256))
+        return LEMO_ERR_INVALID_ARG;
+    const PredictLayout p = predict_layout(shape, d, rank);
+    if (ws_bytes < p.total) return LEMO_ERR_INVALID_ARG;
+    int dev = 0;
+    const int sms = device_sms(&dev);
+    if (sms <= 0) return LEMO_ERR_CUDA;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    char* w = static_cast<char*>(ws);
+    const lemo::WsLayout& lay = p.base;
+    const lemo::PlanHeader* hdr = reinterpret_cast<const lemo::PlanHeader*>(w + lay.hdr);
+    float* xbar = reinterpret_cast<float*>(w + p.xbar);
+    float* part = reinterpret_cast<float*>(w + p.part);
+    float* P = reinterpret_cast<float*>(w + lay.mblk);
+    const int hd = shape->H * shape->dh;
+
+    launch_plan(shape, w, lay, nullptr, st);
+    if ((e = launch_status()) != LEMO_OK) return e;
+    if (shape->total_L == 0) return LEMO_OK;
+    const unsigned ytiles = (unsigned)((p.tb + pr::GT - 1) / pr::GT);
+    pr::pool_kernel<<<dim3((unsigned)p.tb, (unsigned)((d + pr::kPoolCols - 1) / pr::kPoolCols)),
+                      pr::kPoolThreads, 0, st>>>(x, ld_x, d, shape->cu_seqlens, shape->batch,
+                                                 shape->block, w, lay, xbar);
+    if ((e = launch_status()) != LEMO_OK) return e;
+    const int kchunk = ((d + p.splits - 1) / p.splits + pr::GK - 1) / pr::GK * pr::GK;
+    for (int side = 0; side < 2; ++side) {
+        const uint16_t* w1 = side == 0 ? w1q : w1k;
+        const uint16_t* w2 = side == 0 ? w2q : w2k;
+        float* hid = reinterpret_cast<float*>(w + (side == 0 ? p.hq : p.hk));
+        float* out = reinterpret_cast<float*>(w + (side == 0 ? p.qh : p.kh));
+        pr::gemm_kernel<<<dim3((unsigned)((rank + pr::GT - 1) / pr::GT), ytiles, (unsigned)p.splits),
+                          256, 0, st>>>(xbar, d, w1, rank, part, hdr, rank, d, kchunk);
+        pr::reduce_kernel<<<sms * 4, 256, 0, st>>>(part, p.splits, hdr, rank, true, hid);
+        pr::gemm_kernel<<<dim3((unsigned)((hd + pr::GT - 1) / pr::GT), ytiles, 1), 256, 0, st>>>(
+            hid, rank, w2, hd, out, hdr, hd, rank, rank);
+        if ((e = launch_status()) != LEMO_OK) return e;
+    }
+    const unsigned ptiles = (unsigned)((p.tb + pr::PT - 1) / pr::PT);
+    const size_t psmem = 2 * sizeof(float) * pr::PT * (shape->dh + 1);
+    if (psmem > 48 * 1024) {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (cudaFuncSetAttribute(pr::products_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)psmem) != cudaSuccess)
+            return LEMO_ERR_CUDA;
+    }
+    pr::products_kernel<<<dim3(ptiles, ptiles), pr::PT * pr::PT, psmem, st>>>(
+        reinterpret_cast<float*>(w + p.qh), reinterpret_cast<float*>(w + p.kh), shape->H,
+        shape->dh, shape->batch, w, lay, 1.f / (float)shape->H, P);
+    if ((e = launch_status()) != LEMO_OK) return e;
+    const int64_t cs_ctas = (p.tb + 7) / 8;
+    const int cs_grid = (int)(cs_ctas < (int64_t)sms * 8 ? cs_ctas : sms * 8);
+    lemo::score::column_sum_kernel<<<cs_grid, 256, 0, st>>>(P, w, lay, shape->batch, block_scores);
     return launch_status();
 }
 

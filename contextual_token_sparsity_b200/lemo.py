@@ -57,6 +57,9 @@ _SIGS = {
                                              _P, _P, _P, _P]),
     "lemo_gather_pad": (ctypes.c_int, [_P, _I64, _I64, _I32, _P, _P, _I32, _P, _I64, _I64, _P]),
     "lemo_scatter_residual": (ctypes.c_int, [_P, _I64, _I64, _I32, _P, _I64, _P, _P, _P]),
+    "lemo_predict_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(lemo_shape), _I32, _I32]),
+    "lemo_predict_scores": (ctypes.c_int, [ctypes.POINTER(lemo_shape), _I32, _P, _I64, _P, _P, _P,
+                                           _P, _I32, _P, _P, ctypes.c_size_t, _P]),
     "lemo_get_error": (ctypes.c_int, [_P]),
     "lemo_set_test_hooks": (None, [_I32, _I64]),
 }
@@ -157,6 +160,20 @@ def lemo_scatter_residual(x, y, kept_idx, kept_total, stream=None, d=None):
                                         y.stride(0), _ptr(kept_idx), _ptr(kept_total),
                                         _stream(stream)),
            "lemo_scatter_residual")
+
+
+def lemo_predict_workspace_size(shape: lemo_shape, d: int, rank: int) -> int:
+    return int(load().lemo_predict_workspace_size(ctypes.byref(shape), int(d), int(rank)))
+
+
+def lemo_predict_scores(shape, x, w1q, w2q, w1k, w2k, block_scores, ws, stream=None, d=None):
+    """x [rows, ld_x] bf16; w1 [d, rank], w2 [rank, H*dh] bf16 row-major tensors."""
+    d = x.shape[1] if d is None else d
+    _check(load().lemo_predict_scores(ctypes.byref(shape), int(d), _ptr(x), x.stride(0),
+                                      _ptr(w1q), _ptr(w2q), _ptr(w1k), _ptr(w2k),
+                                      int(w1q.shape[1]), _ptr(block_scores), _ptr(ws),
+                                      ws.numel() * ws.element_size(), _stream(stream)),
+           "lemo_predict_scores")
 
 
 def lemo_get_error(stream=None) -> int:

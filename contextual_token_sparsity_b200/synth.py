@@ -27,6 +27,7 @@ __all__ = [
     "rng_for",
     "salient_rows",
     "qk_direct",
+    "projected_x",
     "qk_projected",
     "normal_bf16",
     "predictor_weights",
@@ -97,6 +98,16 @@ def qk_direct(lengths, H: int, dh: int, salient_fracs, seed: int):
             cu, sal)
 
 
+def projected_x(L: int, d: int, salient_frac: float, seed: int):
+    """Embeddings X ~ N(0, 1) [L, d] with round(frac * L) salient rows scaled
+    by 4, as bf16 bits; returns (x_bits, salient ids)."""
+    rx = rng_for(seed, 4)
+    x = rx.standard_normal((L, d), dtype=np.float32)
+    sal = salient_rows(rx, L, salient_frac)
+    x[sal] *= 4.0
+    return to_bf16_bits(x), sal
+
+
 def qk_projected(L: int, d: int, H: int, dh: int, salient_frac: float, seed: int,
                  chunk: int = 4096):
     """Embeddings X ~ N(0, 1) [L, d] with a salient subset scaled by 4, and
@@ -106,11 +117,8 @@ def qk_projected(L: int, d: int, H: int, dh: int, salient_frac: float, seed: int
     in float64 from those bf16 values (row chunks of ``chunk``) and rounded.
     Returns (x_bits [L, d], q_bits [L, H*dh], k_bits [L, H*dh], salient ids).
     """
-    rx, rw = rng_for(seed, 4), rng_for(seed, 5)
-    x = rx.standard_normal((L, d), dtype=np.float32)
-    sal = salient_rows(rx, L, salient_frac)
-    x[sal] *= 4.0
-    x_bits = to_bf16_bits(x)
+    x_bits, sal = projected_x(L, d, salient_frac, seed)
+    rw = rng_for(seed, 5)
     std = 1.0 / np.sqrt(d)
     wq = bf16_bits_to_f32(to_bf16_bits(rw.standard_normal((d, H * dh)) * std)).astype(np.float64)
     wk = bf16_bits_to_f32(to_bf16_bits(rw.standard_normal((d, H * dh)) * std)).astype(np.float64)

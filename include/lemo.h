@@ -239,6 +239,46 @@ LEMO_API lemo_status lemo_scatter_residual(uint16_t* x, int64_t ld_x, int64_t x_
                                   const int32_t* kept_total, lemo_stream stream);
 
 /*
+ * Workspace bytes of lemo_predict_scores for `shape`, residual width d and
+ * predictor rank (the plan arrays, block means, hidden activations, split-K
+ * partial sums, predicted Q/K block embeddings and the block-product
+ * matrices).  Returns 0 for invalid arguments.  HOST-only computation.
+ */
+LEMO_API size_t lemo_predict_workspace_size(const lemo_shape* shape, int32_t d, int32_t rank);
+
+/*
+ * Predicted token-block scores from low-rank ReLU predictors (step a8).
+ *
+ * Jenga summary, section 4.2.2, "Neural-network-based Predictor" and Eq. 3:
+ * each layer has a query predictor and a key predictor that read one
+ * representative embedding per token block; the product of their outputs
+ * approximates the block-pair informativeness, which is aggregated along the
+ * column like the exact scores.
+ *
+ *   xbar_g   = mean of the rows of token block g of x
+ *   Qhat     = relu(xbar W1q) W2q,   Khat = relu(xbar W1k) W2k      ([blocks, H*dh])
+ *   P[n][m]  = (1/H) sum_h max(Qhat_n^h . Khat_m^h, 0)   for n >= m in one sequence
+ *   score[m] = sum_{n = m}^{N_b - 1} P[n][m]
+ *
+ * x            DEVICE bf16 [total_L rows, stride ld_x], 16-byte aligned,
+ *              d % 8 == 0, ld_x >= d, ld_x % 8 == 0.
+ * w1q, w1k     DEVICE bf16 [d, rank] row-major.
+ * w2q, w2k     DEVICE bf16 [rank, H*dh] row-major.  Pruned predictor neurons
+ *              (zero columns of W1 / rows of W2) may simply be left out by
+ *              passing the compacted matrices and the smaller rank.
+ * block_scores DEVICE fp32 [total_blocks].
+ * ws, ws_bytes DEVICE workspace of lemo_predict_workspace_size bytes,
+ *              256-byte aligned.
+ * Computed in fp32 on the CUDA cores; split-K sums are reduced in a fixed
+ * order, so the result is deterministic.
+ */
+LEMO_API lemo_status lemo_predict_scores(const lemo_shape* shape, int32_t d, const uint16_t* x,
+                                         int64_t ld_x, const uint16_t* w1q, const uint16_t* w2q,
+                                         const uint16_t* w1k, const uint16_t* w2k, int32_t rank,
+                                         float* block_scores, void* ws, size_t ws_bytes,
+                                         lemo_stream stream);
+
+/*
  * Synchronises `stream`, then reports and clears the device error word of the
  * current device: LEMO_OK, LEMO_ERR_INVALID_ARG (cu_seqlens or an index
  * failed a device-side check), LEMO_ERR_CAPACITY, LEMO_ERR_TIMEOUT, or
