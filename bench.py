@@ -341,6 +341,7 @@ def run_lemo(args):
     roofline = {"bound": "tensor", "kernel": "score_tiles_kernel (+plan, column sum)",
                 "achieved": round(achieved_tf, 1), "peak": peak_tf, "unit": "TFLOP/s",
                 "frac": round(achieved_tf / peak_tf, 4), "traffic": traffic,
+                "frac_of_sustained_peak": round(achieved_tf / peaks["bf16_tflops_sustained"], 4),
                 "peak_source": f"{peaks['source']} bf16 "
                                f"{'sustained' if long_region else 'burst'} cuBLAS GEMM",
                 "algorithmic_flops_per_launch": F}

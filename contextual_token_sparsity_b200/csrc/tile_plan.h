@@ -30,7 +30,7 @@ namespace lemo_plan {
 
 constexpr int TM = 256;  // query rows of a tile (two CTAs x 128)
 constexpr int TN = 256;  // key columns of a tile
-constexpr int GROUP = 8;
+constexpr int GROUP = 16;
 
 LEMO_HD int64_t query_tiles(int64_t L) { return (L + TM - 1) / TM; }
 
