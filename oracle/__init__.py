@@ -32,4 +32,7 @@ from .lemo_oracle import (  # noqa: F401
     predictor_embeddings,
     predict_scores,
     recall,
+    recompute_input,
+    mlp_token_scores,
+    mlp_block_scores,
 )

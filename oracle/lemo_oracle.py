@@ -46,6 +46,13 @@ design notes of the repository):
 9. Predictor: representative embedding = block mean of X; Eq. 3 is read per
    head with the same positive part / mean over heads as Eq. 2 and block-level
    causality n >= m (diagonal block included).
+10. Backward input recomputation: x_in is recovered as bf16(x_out - y) on the
+    kept rows (one rounding), which is not an exact inverse of the rounded
+    forward addition.
+11. MLP-block elimination: a token's informativeness is the sum of the
+    positive parts of its MLP intermediate activation (the ReLU output, or
+    SiLU(gate) * up); a token block's score is the maximum over its tokens,
+    the block rule of Eq. 2.
 
 Each function below is pinned by tests under ``tests/`` against hand-worked
 values, closed forms, brute force on tiny inputs, library reductions or
@@ -73,6 +80,9 @@ __all__ = [
     "predictor_embeddings",
     "predict_scores",
     "recall",
+    "recompute_input",
+    "mlp_token_scores",
+    "mlp_block_scores",
 ]
 
 _BF16_MAX = (2.0 - 2.0 ** -7) * 2.0 ** 127
@@ -382,3 +392,54 @@ def recall(mask_pred, mask_exact) -> float:
     e = np.asarray(mask_exact).astype(bool)
     ne = int(e.sum())
     return 1.0 if ne == 0 else float((p & e).sum()) / ne
+
+
+# ---------------------------------------------------------------------------
+# Extensions: backward input recomputation and MLP-block elimination
+# ---------------------------------------------------------------------------
+
+def recompute_input(x_out_bits, y_bits, kept_idx) -> np.ndarray:
+    """Recover the layer input from its output by subtraction.
+
+    [Jenga] §4.2.3 "In-place Addition": during backpropagation the original
+    inputs are recomputed by subtracting the sublayer output from the output
+    embeddings.  For r < K, row kept_idx[r] becomes bf16(x_out - y[r]) (exact
+    difference rounded once, ties to even); every other row keeps its bytes.
+    """
+    x_in = np.array(x_out_bits, dtype=np.uint16, copy=True)
+    d = x_in.shape[1]
+    for r in range(len(kept_idx)):
+        t = int(kept_idx[r])
+        diff = bf16_bits_to_f64(x_in[t]) - bf16_bits_to_f64(np.asarray(y_bits[r])[:d])
+        x_in[t] = f64_to_bf16_bits(diff)
+    return x_in
+
+
+def mlp_token_scores(act_bits=None, gate_bits=None, up_bits=None) -> np.ndarray:
+    """Per-token informativeness from MLP intermediate activations.
+
+    [Jenga] §4.2.1 "Extend to MLP Block": the activations used are the ReLU
+    outputs (ReLU MLPs) or SiLU(gate) * up (SiLU MLPs).  Reading taken: the
+    token's score is the sum of the positive parts of that vector.  Pass
+    either ``act_bits`` (bf16 [L, d_ff], used as is) or ``gate_bits`` and
+    ``up_bits`` (bf16 [L, d_ff]; SiLU(g) = g / (1 + exp(-g)) in float64).
+    """
+    if act_bits is not None:
+        a = bf16_bits_to_f64(act_bits)
+    else:
+        g = bf16_bits_to_f64(gate_bits)
+        u = bf16_bits_to_f64(up_bits)
+        a = g / (1.0 + np.exp(-g)) * u
+    return np.maximum(a, 0.0).sum(axis=1)
+
+
+def mlp_block_scores(token_scores, cu_seqlens, block: int) -> np.ndarray:
+    """Token-block score of the MLP path: the maximum over the block's tokens
+    (Eq. 2's block rule), blocks of all sequences concatenated in order."""
+    ts = np.asarray(token_scores, dtype=np.float64)
+    cu = [int(c) for c in np.asarray(cu_seqlens)]
+    out = []
+    for s in range(len(cu) - 1):
+        for t0 in range(cu[s], cu[s + 1], block):
+            out.append(ts[t0:min(t0 + block, cu[s + 1])].max())
+    return np.asarray(out, dtype=np.float64)

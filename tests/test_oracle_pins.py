@@ -422,3 +422,61 @@ def test_predict_scores_brute():
 def test_recall():
     assert oracle.recall([1, 0, 1, 1], [1, 1, 0, 1]) == pytest.approx(2 / 3)
     assert oracle.recall([0, 0], [0, 0]) == 1.0
+
+
+# --------------------------------------------- backward recompute, MLP scores
+
+def test_recompute_input_inverts_exact_additions():
+    """Small integers: x_out = x_in + y is exact, so subtraction recovers x_in."""
+    rng = np.random.default_rng(40)
+    x_in = bits(rng.integers(-50, 50, size=(200, 16)))
+    idx = np.arange(0, 200, 3, dtype=np.int32)
+    y = bits(rng.integers(-50, 50, size=(len(idx), 16)))
+    x_out = oracle.scatter_residual(x_in, y, idx)
+    assert np.array_equal(oracle.recompute_input(x_out, y, idx), x_in)
+
+
+def test_recompute_input_error_bound_and_untouched_rows():
+    """In general the recovered row is within one bf16 ulp of x_out of the
+    original (one rounding in each direction), and other rows keep their bytes."""
+    rng = np.random.default_rng(41)
+    x_in = synth.to_bf16_bits(rng.standard_normal((300, 32)))
+    idx = np.arange(1, 300, 2, dtype=np.int32)
+    y = synth.to_bf16_bits(rng.standard_normal((len(idx), 32)) * 10 ** rng.uniform(-2, 2, (len(idx), 1)))
+    x_out = oracle.scatter_residual(x_in, y, idx)
+    rec = oracle.recompute_input(x_out, y, idx)
+    keep = np.ones(300, bool)
+    keep[idx] = False
+    assert np.array_equal(rec[keep], x_out[keep])
+    xo = oracle.bf16_bits_to_f64(x_out[idx])
+    ulp = np.ldexp(1.0, np.frexp(np.abs(xo) + 1e-300)[1] - 8)
+    err = np.abs(oracle.bf16_bits_to_f64(rec[idx]) - oracle.bf16_bits_to_f64(x_in[idx]))
+    assert (err <= ulp + 1e-300).all()
+    # and the definition: one rounding of the exact difference, via float32
+    f32 = synth.bf16_bits_to_f32(x_out[idx]) - synth.bf16_bits_to_f32(y)
+    assert np.array_equal(rec[idx], synth.to_bf16_bits(f32))
+
+
+def test_mlp_scores_brute_force():
+    rng = np.random.default_rng(42)
+    a = bits(rng.integers(-4, 5, size=(10, 6)))
+    af = synth.bf16_bits_to_f32(a).astype(np.float64)
+    want = [sum(max(v, 0.0) for v in row) for row in af]
+    np.testing.assert_array_equal(oracle.mlp_token_scores(act_bits=a), want)
+    cu = np.array([0, 7, 10])
+    blocks = oracle.mlp_block_scores(want, cu, 4)
+    np.testing.assert_array_equal(blocks, [max(want[0:4]), max(want[4:7]), max(want[7:10])])
+
+
+def test_mlp_silu_gate_matches_relu_path_and_closed_form():
+    rng = np.random.default_rng(43)
+    g = synth.to_bf16_bits(rng.standard_normal((5, 8)) * 3)
+    u = synth.to_bf16_bits(rng.standard_normal((5, 8)))
+    gf = synth.bf16_bits_to_f32(g).astype(np.float64)
+    uf = synth.bf16_bits_to_f32(u).astype(np.float64)
+    silu = gf * (0.5 * (1.0 + np.tanh(0.5 * gf)))  # logistic via tanh: an independent route
+    want = np.maximum(silu * uf, 0.0).sum(axis=1)
+    np.testing.assert_allclose(oracle.mlp_token_scores(gate_bits=g, up_bits=u), want, rtol=1e-13)
+    # gate = 0: SiLU(0) = 0, every score is 0
+    z = np.zeros_like(g)
+    assert (oracle.mlp_token_scores(gate_bits=z, up_bits=u) == 0).all()
