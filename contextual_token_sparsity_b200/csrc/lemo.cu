@@ -10,6 +10,7 @@
 
 #include "lemo.h"
 #include "common.cuh"
+#include "mlp.cuh"
 #include "move.cuh"
 #include "predict.cuh"
 #include "score.cuh"
@@ -88,9 +89,9 @@ lemo_status check_ws(const lemo_shape* s, const void* ws, size_t ws_bytes) {
 }
 
 void launch_plan(const lemo_shape* s, char* ws, const lemo::WsLayout& lay, int32_t* zero_word,
-                 cudaStream_t st) {
+                 cudaStream_t st, float* zero_blocks = nullptr) {
     lemo::plan_kernel<<<1, 1024, 0, st>>>(s->cu_seqlens, s->batch, s->total_L, s->max_seqlen,
-                                          s->block, ws, lay, zero_word);
+                                          s->block, ws, lay, zero_word, zero_blocks);
 }
 
 // 3-D view of a [rows, H*dh] bf16 matrix as (64 elements, rows, H*dh/64
@@ -149,7 +150,7 @@ int score_pairs(int dev, int sms) {
 
 // Persistent grid of the row-copy kernels: as many CTAs as fit on the SMs
 // at once (one full wave), so no CTA waits for a second wave.
-int g_move_ctas[kMaxDevices][2];
+int g_move_ctas[kMaxDevices][3];
 
 template <typename Kernel>
 int move_grid(int dev, int sms, int which, Kernel kernel) {
@@ -460,6 +461,74 @@ lemo_status lemo_scatter_residual(uint16_t* x, int64_t ld_x, int64_t x_rows, int
     lemo::scatter_residual_kernel<<<move_grid(dev, sms, 1, lemo::scatter_residual_kernel),
                                     lemo::kMoveThreads, 0,
                                     reinterpret_cast<cudaStream_t>(stream)>>>(a);
+    return launch_status();
+}
+
+lemo_status lemo_recompute_input(uint16_t* x, int64_t ld_x, int64_t x_rows, int32_t d,
+                                 const uint16_t* y, int64_t ld_y, const int32_t* kept_idx,
+                                 const int32_t* kept_total, lemo_stream stream) {
+    lemo_status e = check_move(x, ld_x, x_rows, d, y, ld_y, kept_idx, kept_total);
+    if (e != LEMO_OK) return e;
+    int dev = 0;
+    const int sms = device_sms(&dev);
+    if (sms <= 0) return LEMO_ERR_CUDA;
+    lemo::MoveArgs a;
+    a.src = reinterpret_cast<const uint4*>(y);
+    a.dst = reinterpret_cast<uint4*>(x);
+    a.ld_src = ld_y / 8;
+    a.ld_dst = ld_x / 8;
+    a.x_rows = x_rows;
+    a.dvec = d / 8;
+    a.kept_idx = kept_idx;
+    a.kept_total = kept_total;
+    a.pad_to = 1;
+    a.cap = 0;
+    lemo::recompute_input_kernel<<<move_grid(dev, sms, 2, lemo::recompute_input_kernel),
+                                   lemo::kMoveThreads, 0,
+                                   reinterpret_cast<cudaStream_t>(stream)>>>(a);
+    return launch_status();
+}
+
+lemo_status lemo_mlp_block_scores(const lemo_shape* shape, int32_t d_ff, const uint16_t* act,
+                                  const uint16_t* gate, const uint16_t* up, int64_t ld,
+                                  float* token_scores, float* block_scores, void* ws,
+                                  size_t ws_bytes, lemo_stream stream) {
+    lemo_status e = check_shape(shape, false);
+    if (e != LEMO_OK) return e;
+    const bool relu_mode = act != nullptr;
+    if (relu_mode ? (gate || up) : (!gate || !up)) return LEMO_ERR_INVALID_ARG;
+    if (!block_scores || d_ff < 1 || ld < d_ff) return LEMO_ERR_INVALID_ARG;
+    if (d_ff % 8 != 0 || ld % 8 != 0) return LEMO_ERR_UNSUPPORTED;
+    if ((act && !aligned(act, 16)) || (gate && !aligned(gate, 16)) || (up && !aligned(up, 16)) ||
+        !aligned(block_scores, 4) || (token_scores && !aligned(token_scores, 4)))
+        return LEMO_ERR_INVALID_ARG;
+    if ((e = check_ws(shape, ws, ws_bytes)) != LEMO_OK) return e;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const lemo::WsLayout lay = layout_of(shape);
+    char* w = static_cast<char*>(ws);
+    launch_plan(shape, w, lay, nullptr, st, block_scores);  // also clears block_scores
+    if ((e = launch_status()) != LEMO_OK) return e;
+    if (shape->total_L == 0) return LEMO_OK;
+    lemo::mlp::Args a;
+    a.act = act;
+    a.gate = gate;
+    a.up = up;
+    a.ld = ld;
+    a.dvec = d_ff / 8;
+    a.cu = shape->cu_seqlens;
+    a.batch = shape->batch;
+    a.block = shape->block;
+    a.ws = w;
+    a.lay = lay;
+    a.token_scores = token_scores;
+    a.block_scores = block_scores;
+    int dev = 0;
+    const int sms = device_sms(&dev);
+    if (sms <= 0) return LEMO_ERR_CUDA;
+    const int64_t ctas_needed =
+        ((int64_t)shape->total_L + lemo::mlp::kThreads / 32 - 1) / (lemo::mlp::kThreads / 32);
+    const int64_t grid = ctas_needed < (int64_t)sms * 4 ? ctas_needed : (int64_t)sms * 4;
+    lemo::mlp::block_scores_kernel<<<(unsigned)grid, lemo::mlp::kThreads, 0, st>>>(a);
     return launch_status();
 }
 

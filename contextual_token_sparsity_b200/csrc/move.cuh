@@ -128,4 +128,51 @@ __global__ void __launch_bounds__(kMoveThreads) scatter_residual_kernel(MoveArgs
     }
 }
 
+// Backward-pass input recomputation (Jenga summary, section 4.2.3: the
+// original inputs are recovered by subtracting the sublayer output):
+// x[kept_idx[r]] = bf16(x[kept_idx[r]] - y[r]) for r < K, in place, one
+// rounding of the exact difference.
+__device__ __forceinline__ uint32_t sub_bf16x2_rn(uint32_t a, uint32_t b) {
+    const float alo = __uint_as_float(a << 16), ahi = __uint_as_float(a & 0xffff0000u);
+    const float blo = __uint_as_float(b << 16), bhi = __uint_as_float(b & 0xffff0000u);
+    const __nv_bfloat162 r = __floats2bfloat162_rn(alo - blo, ahi - bhi);
+    return *reinterpret_cast<const uint32_t*>(&r);
+}
+
+__global__ void __launch_bounds__(kMoveThreads) recompute_input_kernel(MoveArgs a) {
+    int64_t K = *a.kept_total;
+    if (K < 0) K = 0;
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = ((int64_t)blockIdx.x * kMoveThreads + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * kMoveThreads) >> 5;
+    constexpr int U = kMoveUnroll / 2;
+    for (int64_t r = warp; r < K; r += nwarps) {
+        const int64_t t = a.kept_idx[r];
+        if (t < 0 || t >= a.x_rows) {
+            if (lane == 0) raise_error(LEMO_ERR_INVALID_ARG);
+            continue;
+        }
+        uint4* xr = a.dst + t * a.ld_dst;
+        const uint4* yr = a.src + r * a.ld_src;
+        for (int c0 = 0; c0 < a.dvec; c0 += 32 * U) {
+            uint4 xv[U], yv[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int c = c0 + u * 32 + lane;
+                if (c < a.dvec) {
+                    xv[u] = xr[c];
+                    yv[u] = ld_stream(yr + c);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int c = c0 + u * 32 + lane;
+                if (c < a.dvec)
+                    xr[c] = make_uint4(sub_bf16x2_rn(xv[u].x, yv[u].x), sub_bf16x2_rn(xv[u].y, yv[u].y),
+                                       sub_bf16x2_rn(xv[u].z, yv[u].z), sub_bf16x2_rn(xv[u].w, yv[u].w));
+            }
+        }
+    }
+}
+
 }  // namespace lemo

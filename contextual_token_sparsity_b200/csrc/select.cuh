@@ -42,12 +42,14 @@ __device__ __forceinline__ T block_scan_incl(T v, T* warp_sums, T* total) {
 // Plan: per-sequence prefix arrays of a packed batch, device-side checks of
 // cu_seqlens, and a reset of the compaction look-back state.  One CTA.
 // `zero_word` (optional) is set to 0 first, so that a compaction that gives
-// up leaves K = 0 behind rather than a stale count.
+// up leaves K = 0 behind rather than a stale count.  `zero_blocks` (optional)
+// gets its first total_blocks entries cleared (the host only knows an upper
+// bound of that count).
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ cu, int batch,
                                                     int total_L, int max_seqlen, int block,
                                                     char* __restrict__ ws, WsLayout lay,
-                                                    int32_t* zero_word) {
+                                                    int32_t* zero_word, float* zero_blocks) {
     PlanHeader* hdr = reinterpret_cast<PlanHeader*>(ws + lay.hdr);
     int64_t* tile_prefix = reinterpret_cast<int64_t*>(ws + lay.tile_prefix);
     int32_t* blk_prefix = reinterpret_cast<int32_t*>(ws + lay.blk_prefix);
@@ -96,6 +98,8 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
         carry_b += tot_b;
     }
     __syncthreads();
+    if (zero_blocks && !bad)
+        for (int i = tid; i < carry_b; i += blockDim.x) zero_blocks[i] = 0.f;
     if (tid == 0) {
         tile_prefix[batch] = carry_t;
         m_prefix[batch] = carry_m;

@@ -57,6 +57,9 @@ _SIGS = {
                                              _P, _P, _P, _P]),
     "lemo_gather_pad": (ctypes.c_int, [_P, _I64, _I64, _I32, _P, _P, _I32, _P, _I64, _I64, _P]),
     "lemo_scatter_residual": (ctypes.c_int, [_P, _I64, _I64, _I32, _P, _I64, _P, _P, _P]),
+    "lemo_recompute_input": (ctypes.c_int, [_P, _I64, _I64, _I32, _P, _I64, _P, _P, _P]),
+    "lemo_mlp_block_scores": (ctypes.c_int, [ctypes.POINTER(lemo_shape), _I32, _P, _P, _P, _I64,
+                                             _P, _P, _P, ctypes.c_size_t, _P]),
     "lemo_predict_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(lemo_shape), _I32, _I32]),
     "lemo_predict_scores": (ctypes.c_int, [ctypes.POINTER(lemo_shape), _I32, _P, _I64, _P, _P, _P,
                                            _P, _I32, _P, _P, ctypes.c_size_t, _P]),
@@ -160,6 +163,26 @@ def lemo_scatter_residual(x, y, kept_idx, kept_total, stream=None, d=None):
                                         y.stride(0), _ptr(kept_idx), _ptr(kept_total),
                                         _stream(stream)),
            "lemo_scatter_residual")
+
+
+def lemo_recompute_input(x, y, kept_idx, kept_total, stream=None, d=None):
+    """x [rows, ld_x] (in place), y [>= K, ld_y] bf16 2-D tensors."""
+    d = x.shape[1] if d is None else d
+    _check(load().lemo_recompute_input(_ptr(x), x.stride(0), x.shape[0], int(d), _ptr(y),
+                                       y.stride(0), _ptr(kept_idx), _ptr(kept_total),
+                                       _stream(stream)),
+           "lemo_recompute_input")
+
+
+def lemo_mlp_block_scores(shape, block_scores, ws, act=None, gate=None, up=None,
+                          token_scores=None, stream=None):
+    """act, or gate and up: bf16 [total_L, ld] tensors (d_ff = their width)."""
+    ref = act if act is not None else gate
+    _check(load().lemo_mlp_block_scores(ctypes.byref(shape), int(ref.shape[1]), _ptr(act),
+                                        _ptr(gate), _ptr(up), ref.stride(0), _ptr(token_scores),
+                                        _ptr(block_scores), _ptr(ws),
+                                        ws.numel() * ws.element_size(), _stream(stream)),
+           "lemo_mlp_block_scores")
 
 
 def lemo_predict_workspace_size(shape: lemo_shape, d: int, rank: int) -> int:

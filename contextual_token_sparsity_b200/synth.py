@@ -31,6 +31,7 @@ __all__ = [
     "qk_projected",
     "normal_bf16",
     "predictor_weights",
+    "mlp_activations",
     "Workload",
     "WORKLOADS",
     "make_workload",
@@ -149,6 +150,24 @@ def predictor_weights(d: int, rank: int, out: int, zero_frac: float, seed: int, 
     w2[dead, :] = 0.0
     live = np.setdiff1d(np.arange(rank), dead)
     return to_bf16_bits(w1), to_bf16_bits(w2), live
+
+
+def mlp_activations(L: int, d_ff: int, salient_frac: float, seed: int, gated: bool = True):
+    """MLP intermediate activations at a layer's shape: gate, up ~ N(0, 1)
+    [L, d_ff] (SiLU-gated MLP) or ReLU outputs relu(N(0, 1)) (ReLU MLP), with
+    round(frac * L) salient token rows scaled by 4.  Returns bf16 bits:
+    (gate, up) or (act,)."""
+    r = rng_for(seed, 12)
+    sal = salient_rows(r, L, salient_frac)
+    if gated:
+        g = r.standard_normal((L, d_ff), dtype=np.float32)
+        u = r.standard_normal((L, d_ff), dtype=np.float32)
+        g[sal] *= 4.0
+        u[sal] *= 4.0
+        return to_bf16_bits(g), to_bf16_bits(u)
+    a = np.maximum(r.standard_normal((L, d_ff), dtype=np.float32), 0.0)
+    a[sal] *= 4.0
+    return (to_bf16_bits(a),)
 
 
 @dataclasses.dataclass

@@ -239,6 +239,57 @@ LEMO_API lemo_status lemo_scatter_residual(uint16_t* x, int64_t ld_x, int64_t x_
                                   const int32_t* kept_total, lemo_stream stream);
 
 /*
+ * Backward-pass recomputation of the layer input (extension of step a7).
+ *
+ * Jenga summary, section 4.2.3, "In-place Addition": during backpropagation
+ * the original inputs are recomputed by subtracting the sublayer output from
+ * the output embeddings instead of being stored.
+ *
+ *   for r < K:  x[kept_idx[r], 0:d] = bf16_rne(float(x[kept_idx[r], :]) - float(y[r, :]))
+ *   every other row of x keeps its bytes.
+ *
+ * One rounding of the exact difference, so the result is bit-exact; it is
+ * not an exact inverse of the rounded forward addition (the recovered row is
+ * within one bf16 ulp of x_out of the original).  The other passes of the
+ * backward token movement reuse the forward kernels: lemo_gather_pad on the
+ * output gradient gives the sublayer's output gradient at the kept rows, and
+ * lemo_scatter_residual adds the sublayer's input gradient back into the
+ * residual gradient.  Arguments, alignment and errors as
+ * lemo_scatter_residual.
+ */
+LEMO_API lemo_status lemo_recompute_input(uint16_t* x, int64_t ld_x, int64_t x_rows, int32_t d,
+                                          const uint16_t* y, int64_t ld_y,
+                                          const int32_t* kept_idx, const int32_t* kept_total,
+                                          lemo_stream stream);
+
+/*
+ * Token-block scores of the MLP block (extension of steps a1-a3).
+ *
+ * Jenga summary, section 4.2.1, "Extend to MLP Block": token elimination is
+ * extended to the MLP using its intermediate activations - the ReLU outputs of
+ * ReLU MLPs, or SiLU(gate) * up of SiLU-gated MLPs.  The page gives no
+ * aggregation; the one used here is the plainest that matches Eq. 2's block
+ * rule:
+ *
+ *   token_score[t] = sum_c max(a[t, c], 0)
+ *   block_scores[g] = max over the tokens t of block g of token_score[t]
+ *
+ * Pass either `act` (a = act, e.g. ReLU outputs) with gate = up = NULL, or
+ * `gate` and `up` with act = NULL (a = SiLU(gate) * up, SiLU(g) = g / (1 +
+ * e^-g), evaluated in fp32 as g (1 + tanh(g/2)) / 2 with the hardware tanh).  All are DEVICE bf16 [total_L rows, stride ld], 16-byte
+ * aligned, d_ff % 8 == 0, ld >= d_ff and ld % 8 == 0.  token_scores
+ * (optional, DEVICE fp32 [total_L]) and block_scores (DEVICE fp32
+ * [total_blocks]) are outputs; the block scores feed lemo_select unchanged.
+ * ws as for lemo_select.  Deterministic (fixed summation order per token;
+ * the block maximum does not depend on order).
+ */
+LEMO_API lemo_status lemo_mlp_block_scores(const lemo_shape* shape, int32_t d_ff,
+                                           const uint16_t* act, const uint16_t* gate,
+                                           const uint16_t* up, int64_t ld, float* token_scores,
+                                           float* block_scores, void* ws, size_t ws_bytes,
+                                           lemo_stream stream);
+
+/*
  * Workspace bytes of lemo_predict_scores for `shape`, residual width d and
  * predictor rank (the plan arrays, block means, hidden activations, split-K
  * partial sums, predicted Q/K block embeddings and the block-product
