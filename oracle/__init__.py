@@ -9,7 +9,8 @@ the definitions of
 * "Jenga: Enhancing LLM Long-Context Fine-tuning with Contextual Token
   Sparsity" (aipaper.cc summary of the USENIX ATC'25 paper), §4.2.1 Eq. 1,
   Eq. 2, Fig. 6 and the layer-specific-threshold paragraph; §4.2.2 Eq. 3;
-  §4.2.3 "Permutation-free Token Movement" (selective load, in-place addition);
+  §4.2.3 "Permutation-free Token Movement" (selective load, in-place addition)
+  and "Segment-based Peak Cutting";
 * "LeMo" (pith.science reading of arXiv 2501.09767), "What carries the
   argument".
 
@@ -35,4 +36,7 @@ from .lemo_oracle import (  # noqa: F401
     recompute_input,
     mlp_token_scores,
     mlp_block_scores,
+    lm_head_loss,
+    lm_head_loss_f64,
+    lm_head_rows,
 )

@@ -53,6 +53,10 @@ design notes of the repository):
     positive parts of its MLP intermediate activation (the ReLU output, or
     SiLU(gate) * up); a token block's score is the maximum over its tokens,
     the block rule of Eq. 2.
+12. Segment-based peak cutting: the loss is the mean next-token cross
+    entropy of the lm-head logits over the tokens whose target is not the
+    ignore index (0 when there is none); segmenting the tokens changes only
+    the order of work, so the oracle is the unsegmented definition.
 
 Each function below is pinned by tests under ``tests/`` against hand-worked
 values, closed forms, brute force on tiny inputs, library reductions or
@@ -83,6 +87,9 @@ __all__ = [
     "recompute_input",
     "mlp_token_scores",
     "mlp_block_scores",
+    "lm_head_loss",
+    "lm_head_loss_f64",
+    "lm_head_rows",
 ]
 
 _BF16_MAX = (2.0 - 2.0 ** -7) * 2.0 ** 127
@@ -443,3 +450,83 @@ def mlp_block_scores(token_scores, cu_seqlens, block: int) -> np.ndarray:
         for t0 in range(cu[s], cu[s + 1], block):
             out.append(ts[t0:min(t0 + block, cu[s + 1])].max())
     return np.asarray(out, dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------
+# Extension: segment-based peak cutting of the lm-head loss (§4.2.3)
+# ---------------------------------------------------------------------------
+
+def lm_head_loss(h_bits, w_bits, targets, ignore_index: int = -100):
+    """Mean cross entropy of the lm-head logits and its gradients, float64.
+
+    [Jenga] §4.2.3 "Segment-based Peak Cutting": each token's logits over the
+    vocabulary feed a next-token loss; the pages split the tokens into
+    segments and finish each segment's gradient before the next one, which
+    changes the peak memory but not the result.  This is the plain
+    definition the segmented computation must reproduce:
+
+        z        = h W^T                        (logits, [T, V])
+        lse_t    = log sum_v exp(z_tv)
+        loss     = (1/n) sum_{t valid} (lse_t - z_t,y_t),  n = #valid tokens
+        dz_t     = (softmax(z_t) - onehot(y_t)) / n   (0 for ignored tokens)
+        dh       = dz W,   dW = dz^T h
+
+    ``h_bits`` bf16 [T, d], ``w_bits`` bf16 [V, d] (the lm-head weight),
+    ``targets`` int [T]; a target equal to ``ignore_index`` is ignored.  With
+    no valid token the loss and both gradients are 0.
+    Returns (loss, dh [T, d], dW [V, d], lse [T]) in float64.
+    """
+    return lm_head_loss_f64(bf16_bits_to_f64(h_bits), bf16_bits_to_f64(w_bits), targets,
+                            ignore_index)
+
+
+def lm_head_loss_f64(h, w, targets, ignore_index: int = -100):
+    """``lm_head_loss`` on float64 arrays h [T, d], w [V, d] (no bf16 decode)."""
+    h = np.asarray(h, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    y = np.asarray(targets, dtype=np.int64)
+    T, V = h.shape[0], w.shape[0]
+    valid = y != ignore_index
+    if np.any((y[valid] < 0) | (y[valid] >= V)):
+        raise ValueError("target outside [0, V)")
+    z = h @ w.T
+    zmax = z.max(axis=1, keepdims=True)
+    lse = (zmax + np.log(np.exp(z - zmax).sum(axis=1, keepdims=True)))[:, 0]
+    n = int(valid.sum())
+    if n == 0:
+        return 0.0, np.zeros_like(h), np.zeros_like(w), lse
+    rows = np.nonzero(valid)[0]
+    loss = float((lse[rows] - z[rows, y[rows]]).sum() / n)
+    dz = np.exp(z - lse[:, None])
+    dz[rows, y[rows]] -= 1.0
+    dz[~valid] = 0.0
+    dz /= n
+    return loss, dz @ w, dz.T @ h, lse
+
+
+def lm_head_rows(h_bits, w_bits, targets, rows, n_valid: int, ignore_index: int = -100):
+    """Per-token terms of ``lm_head_loss`` for the listed token rows only.
+
+    For each t in ``rows``: (lse_t - z_t,y_t) (0 if ignored) and the row dh_t
+    = dz_t W, with dz_t scaled by 1/``n_valid`` (the valid-token count of the
+    whole batch).  The same definition as ``lm_head_loss``, evaluated one row
+    at a time so that sampled rows of a large workload stay cheap.
+    Returns (per-row loss terms [len(rows)], dh rows [len(rows), d]).
+    """
+    w = bf16_bits_to_f64(w_bits)
+    out_l, out_dh = [], []
+    for t in rows:
+        ht = bf16_bits_to_f64(np.asarray(h_bits)[int(t)])
+        z = w @ ht
+        m = z.max()
+        lse = m + math.log(np.exp(z - m).sum())
+        yt = int(targets[int(t)])
+        if yt == ignore_index or n_valid == 0:
+            out_l.append(0.0)
+            out_dh.append(np.zeros(w.shape[1]))
+            continue
+        p = np.exp(z - lse)
+        p[yt] -= 1.0
+        out_l.append(lse - z[yt])
+        out_dh.append((p / n_valid) @ w)
+    return np.asarray(out_l), np.asarray(out_dh).reshape(len(out_l), w.shape[1])
