@@ -13,7 +13,7 @@
 namespace lemo {
 
 constexpr int kMoveThreads = 256;
-constexpr int kMoveUnroll = 8;  // 16-byte vectors per lane in flight
+constexpr int kMoveUnroll = 16;  // 16-byte vectors per lane in flight
 
 struct MoveArgs {
     const uint4* src;  // gather: x ; scatter: y
