@@ -2,10 +2,13 @@
 // tensor-map encoding and launches.  The kernels live in the included .cuh
 // files; everything is one translation unit so that the device error word is
 // a single symbol per device.
+#include <cublas_v2.h>  // types only: cuBLAS itself is opened with dlopen on first use
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
+#include <dlfcn.h>
 
+#include <climits>
 #include <mutex>
 
 #include "lemo.h"
@@ -14,6 +17,7 @@
 #include "move.cuh"
 #include "predict.cuh"
 #include "score.cuh"
+#include "segloss.cuh"
 #include "select.cuh"
 
 namespace {
@@ -217,6 +221,72 @@ lemo_status check_predict(const lemo_shape* s, int d, int rank) {
     if (s->dh > 1024 || (int64_t)s->H * s->dh > (1 << 20) || d > (1 << 20) || rank > (1 << 16))
         return LEMO_ERR_UNSUPPORTED;
     return LEMO_OK;
+}
+
+// ---------------------------------------------------------------------------
+// cuBLAS for the plain GEMMs of the segmented loss, opened on first use so
+// that the rest of the library does not depend on it.
+// ---------------------------------------------------------------------------
+struct Blas {
+    using Create = cublasStatus_t (*)(cublasHandle_t*);
+    using SetStream = cublasStatus_t (*)(cublasHandle_t, cudaStream_t);
+    using SetWorkspace = cublasStatus_t (*)(cublasHandle_t, void*, size_t);
+    using GemmEx = cublasStatus_t (*)(cublasHandle_t, cublasOperation_t, cublasOperation_t, int, int,
+                                      int, const void*, const void*, cudaDataType, int, const void*,
+                                      cudaDataType, int, const void*, void*, cudaDataType, int,
+                                      cublasComputeType_t, cublasGemmAlgo_t);
+    bool tried = false;
+    Create create = nullptr;
+    SetStream set_stream = nullptr;
+    SetWorkspace set_workspace = nullptr;
+    GemmEx gemm = nullptr;
+    cublasHandle_t handle[kMaxDevices] = {};
+};
+Blas g_blas;
+constexpr size_t kBlasWorkspace = 32u << 20;
+
+// Handle of device `dev` (created on first use), or nullptr if cuBLAS is
+// unavailable.  Caller holds g_mu.
+cublasHandle_t blas_handle(int dev) {
+    Blas& b = g_blas;
+    if (!b.tried) {
+        b.tried = true;
+        void* lib = dlopen("libcublas.so.12", RTLD_NOW | RTLD_GLOBAL);
+        if (lib) {
+            b.create = reinterpret_cast<Blas::Create>(dlsym(lib, "cublasCreate_v2"));
+            b.set_stream = reinterpret_cast<Blas::SetStream>(dlsym(lib, "cublasSetStream_v2"));
+            b.set_workspace = reinterpret_cast<Blas::SetWorkspace>(dlsym(lib, "cublasSetWorkspace_v2"));
+            b.gemm = reinterpret_cast<Blas::GemmEx>(dlsym(lib, "cublasGemmEx"));
+        }
+    }
+    if (!b.create || !b.set_stream || !b.set_workspace || !b.gemm) return nullptr;
+    if (!b.handle[dev] && b.create(&b.handle[dev]) != CUBLAS_STATUS_SUCCESS) b.handle[dev] = nullptr;
+    return b.handle[dev];
+}
+
+// Workspace of lemo_segment_loss.
+struct SegLayout {
+    size_t n_valid, token_loss, blas, z, g, total;
+    int64_t ld;    // row stride of the segment's logits and gradient
+    int64_t rows;  // rows of one segment buffer
+};
+
+SegLayout seg_layout(int64_t T, int V, int seg_rows) {
+    SegLayout l;
+    l.ld = ((int64_t)V + 7) / 8 * 8;
+    l.rows = T < seg_rows ? (T > 0 ? T : 1) : seg_rows;
+    size_t off = 0;
+    l.n_valid = off; off = lemo::align_up(off + 4, 256);
+    l.token_loss = off; off = lemo::align_up(off + 4 * (size_t)(T > 0 ? T : 1), 256);
+    l.blas = off; off = lemo::align_up(off + kBlasWorkspace, 256);
+    l.z = off; off = lemo::align_up(off + 4 * (size_t)l.rows * l.ld, 256);
+    l.g = off; off = lemo::align_up(off + 2 * (size_t)l.rows * l.ld, 256);
+    l.total = off;
+    return l;
+}
+
+bool seg_args_ok(int64_t T, int V, int seg_rows) {
+    return T >= 0 && T <= INT_MAX && V >= 1 && seg_rows >= 1 && (int64_t)V + 7 <= INT_MAX;
 }
 
 }  // namespace
@@ -599,6 +669,89 @@ lemo_status lemo_predict_scores(const lemo_shape* shape, int32_t d, const uint16
     const int64_t cs_ctas = (p.tb + 7) / 8;
     const int cs_grid = (int)(cs_ctas < (int64_t)sms * 8 ? cs_ctas : sms * 8);
     lemo::score::column_sum_kernel<<<cs_grid, 256, 0, st>>>(P, w, lay, shape->batch, block_scores);
+    return launch_status();
+}
+
+size_t lemo_segment_loss_workspace_size(int64_t T, int32_t V, int32_t seg_rows) {
+    if (!seg_args_ok(T, V, seg_rows)) return 0;
+    return seg_layout(T, V, seg_rows).total;
+}
+
+lemo_status lemo_segment_loss(const uint16_t* h, int64_t ld_h, int64_t T, int32_t d,
+                              const uint16_t* w, int64_t ld_w, int32_t V, const int32_t* targets,
+                              int32_t ignore_index, int32_t seg_rows, float* loss,
+                              float* token_loss, uint16_t* dh, int64_t ld_dh, float* dw,
+                              int64_t ld_dw, void* ws, size_t ws_bytes, lemo_stream stream) {
+    namespace sl = lemo::segloss;
+    if (!seg_args_ok(T, V, seg_rows) || d < 1) return LEMO_ERR_INVALID_ARG;
+    if (!loss || !ws || (T > 0 && (!h || !w || !targets))) return LEMO_ERR_INVALID_ARG;
+    if (d % 8 != 0) return LEMO_ERR_UNSUPPORTED;
+    auto stride_ok = [d](int64_t ld) { return ld >= d && ld % 8 == 0 && ld <= INT_MAX; };
+    if (!stride_ok(ld_h) || !stride_ok(ld_w) || (dh && !stride_ok(ld_dh)) || (dw && !stride_ok(ld_dw)))
+        return LEMO_ERR_INVALID_ARG;
+    if (!aligned(h, 16) || !aligned(w, 16) || !aligned(targets, 4) || !aligned(loss, 4) ||
+        (token_loss && !aligned(token_loss, 4)) || (dh && !aligned(dh, 16)) ||
+        (dw && !aligned(dw, 16)) || !aligned(ws, 256))
+        return LEMO_ERR_INVALID_ARG;
+    const SegLayout l = seg_layout(T, V, seg_rows);
+    if (ws_bytes < l.total) return LEMO_ERR_INVALID_ARG;
+    int dev = 0;
+    if (device_sms(&dev) <= 0) return LEMO_ERR_CUDA;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    char* wsp = static_cast<char*>(ws);
+    int32_t* n_valid = reinterpret_cast<int32_t*>(wsp + l.n_valid);
+    float* tl = token_loss ? token_loss : reinterpret_cast<float*>(wsp + l.token_loss);
+    float* z = reinterpret_cast<float*>(wsp + l.z);
+    uint16_t* g = reinterpret_cast<uint16_t*>(wsp + l.g);
+
+    // The handle's stream and workspace are per call: hold the lock until
+    // every GEMM of this call is enqueued.
+    std::lock_guard<std::mutex> lk(g_mu);
+    cublasHandle_t hb = nullptr;
+    if (T > 0) {
+        hb = blas_handle(dev);
+        if (!hb) return LEMO_ERR_UNSUPPORTED;
+        if (g_blas.set_stream(hb, st) != CUBLAS_STATUS_SUCCESS ||
+            g_blas.set_workspace(hb, wsp + l.blas, kBlasWorkspace) != CUBLAS_STATUS_SUCCESS)
+            return LEMO_ERR_CUDA;
+    }
+    sl::count_kernel<<<1, sl::kCountThreads, 0, st>>>(targets, T, V, ignore_index, n_valid);
+    lemo_status e = launch_status();
+    if (e != LEMO_OK) return e;
+    const float one = 1.f, zero = 0.f;
+    for (int64_t s0 = 0; s0 < T; s0 += seg_rows) {
+        const int S = (int)(T - s0 < seg_rows ? T - s0 : seg_rows);
+        const uint16_t* hs = h + s0 * ld_h;
+        // z^T [V, S] = W [V, d] . h_seg^T   (column-major view of row-major z [S, ld])
+        if (g_blas.gemm(hb, CUBLAS_OP_T, CUBLAS_OP_N, V, S, d, &one, w, CUDA_R_16BF, (int)ld_w, hs,
+                        CUDA_R_16BF, (int)ld_h, &zero, z, CUDA_R_32F, (int)l.ld, CUBLAS_COMPUTE_32F,
+                        CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS)
+            return LEMO_ERR_CUDA;
+        sl::RowArgs a;
+        a.z = z;
+        a.ldz = l.ld;
+        a.g = g;
+        a.ldg = l.ld;
+        a.y = targets + s0;
+        a.token_loss = tl + s0;
+        a.n_valid = n_valid;
+        a.V = V;
+        a.ignore = ignore_index;
+        sl::row_kernel<<<S, sl::kRowThreads, 0, st>>>(a);
+        if ((e = launch_status()) != LEMO_OK) return e;
+        // dh_seg^T [d, S] = W^T [d, V] . dz^T [V, S]
+        if (dh && g_blas.gemm(hb, CUBLAS_OP_N, CUBLAS_OP_N, d, S, V, &one, w, CUDA_R_16BF, (int)ld_w,
+                              g, CUDA_R_16BF, (int)l.ld, &zero, dh + s0 * ld_dh, CUDA_R_16BF,
+                              (int)ld_dh, CUBLAS_COMPUTE_32F,
+                              CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS)
+            return LEMO_ERR_CUDA;
+        // dW^T [d, V] += h_seg^T [d, S] . dz [S, V]
+        if (dw && g_blas.gemm(hb, CUBLAS_OP_N, CUBLAS_OP_T, d, V, S, &one, hs, CUDA_R_16BF, (int)ld_h,
+                              g, CUDA_R_16BF, (int)l.ld, &one, dw, CUDA_R_32F, (int)ld_dw,
+                              CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS)
+            return LEMO_ERR_CUDA;
+    }
+    sl::loss_kernel<<<1, sl::kCountThreads, 0, st>>>(tl, T, n_valid, loss);
     return launch_status();
 }
 

@@ -63,6 +63,9 @@ _SIGS = {
     "lemo_predict_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(lemo_shape), _I32, _I32]),
     "lemo_predict_scores": (ctypes.c_int, [ctypes.POINTER(lemo_shape), _I32, _P, _I64, _P, _P, _P,
                                            _P, _I32, _P, _P, ctypes.c_size_t, _P]),
+    "lemo_segment_loss_workspace_size": (ctypes.c_size_t, [_I64, _I32, _I32]),
+    "lemo_segment_loss": (ctypes.c_int, [_P, _I64, _I64, _I32, _P, _I64, _I32, _P, _I32, _I32, _P,
+                                         _P, _P, _I64, _P, _I64, _P, ctypes.c_size_t, _P]),
     "lemo_get_error": (ctypes.c_int, [_P]),
     "lemo_set_test_hooks": (None, [_I32, _I64]),
 }
@@ -197,6 +200,22 @@ def lemo_predict_scores(shape, x, w1q, w2q, w1k, w2k, block_scores, ws, stream=N
                                       int(w1q.shape[1]), _ptr(block_scores), _ptr(ws),
                                       ws.numel() * ws.element_size(), _stream(stream)),
            "lemo_predict_scores")
+
+
+def lemo_segment_loss_workspace_size(T: int, V: int, seg_rows: int) -> int:
+    return int(load().lemo_segment_loss_workspace_size(int(T), int(V), int(seg_rows)))
+
+
+def lemo_segment_loss(h, w, targets, seg_rows, loss, ws, token_loss=None, dh=None, dw=None,
+                      ignore_index=-100, stream=None):
+    """h [T, ld_h] and w [V, ld_w] bf16 2-D tensors, targets int32 [T]; dh
+    bf16 [T, ld_dh] and dw fp32 [V, ld_dw] optional (dw is accumulated)."""
+    _check(load().lemo_segment_loss(
+        _ptr(h), h.stride(0), h.shape[0], int(h.shape[1]), _ptr(w), w.stride(0), int(w.shape[0]),
+        _ptr(targets), int(ignore_index), int(seg_rows), _ptr(loss), _ptr(token_loss), _ptr(dh),
+        dh.stride(0) if dh is not None else 0, _ptr(dw), dw.stride(0) if dw is not None else 0,
+        _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+        "lemo_segment_loss")
 
 
 def lemo_get_error(stream=None) -> int:

@@ -170,6 +170,30 @@ def mlp_activations(L: int, d_ff: int, salient_frac: float, seed: int, gated: bo
     return (to_bf16_bits(a),)
 
 
+def lm_head_inputs(T: int, d: int, V: int, seed: int, logit_std: float = 2.0,
+                   ignore_frac: float = 0.0, ignore_index: int = -100):
+    """Inputs of the lm-head loss: final hidden states h ~ N(0, 1) [T, d],
+    lm-head weight W ~ N(0, logit_std^2 / d) [V, d] (logits of standard
+    deviation about logit_std), uniform next-token targets in [0, V) with a
+    seeded fraction set to ``ignore_index``.  Returns (h bits, W bits, int32
+    targets)."""
+    r = rng_for(seed, 13)
+    h = to_bf16_bits(r.standard_normal((T, d), dtype=np.float32))
+    w = r.standard_normal((V, d), dtype=np.float32)
+    w *= np.float32(logit_std / np.sqrt(d))
+    y = r.integers(0, V, size=T).astype(np.int32)
+    if ignore_frac > 0:
+        y[r.random(T) < ignore_frac] = ignore_index
+    return h, to_bf16_bits(w), y
+
+
+# Segmented lm-head loss at the Llama-2-7B head (d = 4096, V = 32000) over
+# the 16384 tokens of one long sequence, 16 segments of 1024 tokens.
+LM_HEAD_WORKLOADS = {
+    "lmhead-7b": dict(T=16384, d=4096, V=32000, seg_rows=1024, seed=0),
+}
+
+
 @dataclasses.dataclass
 class Workload:
     """One configuration of the path: shapes, seeds and keep ratios."""

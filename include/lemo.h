@@ -330,6 +330,65 @@ LEMO_API lemo_status lemo_predict_scores(const lemo_shape* shape, int32_t d, con
                                          lemo_stream stream);
 
 /*
+ * Workspace bytes of lemo_segment_loss for T tokens, vocabulary V and
+ * segments of seg_rows tokens: the valid-token count, the per-token loss
+ * terms, 32 MiB for the library GEMMs, and ONE segment's fp32 logits plus
+ * their bf16 gradient (2 x min(seg_rows, T) x round_up(V, 8) elements).
+ * That last part is the activation peak that segmenting divides by T /
+ * seg_rows.  Returns 0 for invalid arguments.  HOST-only computation.
+ */
+LEMO_API size_t lemo_segment_loss_workspace_size(int64_t T, int32_t V, int32_t seg_rows);
+
+/*
+ * Segment-based peak cutting of the lm-head loss (extension).
+ *
+ * Jenga summary, section 4.2.3, "Segment-based Peak Cutting": the final loss
+ * over a large vocabulary is computed segment by segment, each segment's
+ * logits are dropped as soon as its gradient is done, so the activation
+ * peak falls to 1/N for N segments.  The result is that of the unsegmented
+ * definition:
+ *
+ *   z = h W^T,  lse_t = log sum_v exp(z_tv)
+ *   loss = (1/n) sum_{t valid} (lse_t - z_t,y_t),   n = #{t : y_t != ignore_index}
+ *   dz_t = (softmax(z_t) - onehot(y_t)) / n   (0 for ignored tokens)
+ *   dh = dz W,   dW += dz^T h
+ *
+ * With n = 0 the loss is 0 and the gradients are zero.
+ *
+ * h            DEVICE bf16 [T, d], row stride ld_h (the final hidden states).
+ * w            DEVICE bf16 [V, d], row stride ld_w (the lm-head weight).
+ * targets      DEVICE int32 [T]: the next-token ids, or ignore_index.
+ *              A target outside [0, V) that is not ignore_index is reported
+ *              as LEMO_ERR_INVALID_ARG by lemo_get_error (that token adds
+ *              nothing).
+ * seg_rows     tokens per segment (>= 1); the last segment may be shorter.
+ * loss         DEVICE fp32 scalar (output).
+ * token_loss   optional DEVICE fp32 [T]: lse_t - z_t,y_t (0 if ignored).
+ * dh           optional DEVICE bf16 [T, d], row stride ld_dh (written).
+ * dw           optional DEVICE fp32 [V, d], row stride ld_dw: ACCUMULATED
+ *              (dW += ...), so zero it for a fresh gradient.  Pass NULL when
+ *              the lm head is frozen (LoRA fine-tuning).
+ * ws, ws_bytes DEVICE workspace of lemo_segment_loss_workspace_size bytes,
+ *              256-byte aligned.
+ * Constraints: d % 8 == 0; every stride a multiple of 8 elements and every
+ * matrix 16-byte aligned; d, V, seg_rows and strides below 2^31.  With T = 0,
+ * h, w and targets may be NULL (the loss is 0).
+ *
+ * The three GEMMs of a segment run in cuBLAS (bf16 inputs, fp32
+ * accumulation, cuBLAS loaded on first use; LEMO_ERR_UNSUPPORTED if it is not
+ * found); the softmax / loss / gradient of each logit row is this library's
+ * kernel.  The first call on a device creates a cuBLAS handle; the GEMMs use
+ * the caller's workspace.  The loss is the fixed-order sum of the per-token
+ * terms (deterministic).  Logits are fp32, dz and dh are rounded to bf16.
+ */
+LEMO_API lemo_status lemo_segment_loss(const uint16_t* h, int64_t ld_h, int64_t T, int32_t d,
+                                       const uint16_t* w, int64_t ld_w, int32_t V,
+                                       const int32_t* targets, int32_t ignore_index,
+                                       int32_t seg_rows, float* loss, float* token_loss,
+                                       uint16_t* dh, int64_t ld_dh, float* dw, int64_t ld_dw,
+                                       void* ws, size_t ws_bytes, lemo_stream stream);
+
+/*
  * Synchronises `stream`, then reports and clears the device error word of the
  * current device: LEMO_OK, LEMO_ERR_INVALID_ARG (cu_seqlens or an index
  * failed a device-side check), LEMO_ERR_CAPACITY, LEMO_ERR_TIMEOUT, or

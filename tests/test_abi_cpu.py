@@ -130,6 +130,47 @@ def test_host_validation_returns_before_cuda(lib):
                                      None) == lemo.LEMO_ERR_INVALID_ARG
 
 
+def test_segment_loss_workspace_and_validation(lib):
+    def align(v):
+        return (v + 255) // 256 * 256
+    for T, V, S in [(16384, 32000, 1024), (300, 1000, 64), (5, 13, 64), (0, 7, 3)]:
+        ld = -(-V // 8) * 8
+        rows = min(S, max(T, 1)) if T < S else S
+        want = align(4)
+        want = align(want + 4 * max(T, 1))
+        want = align(want + (32 << 20))
+        want = align(want + 4 * rows * ld)
+        want = align(want + 2 * rows * ld)
+        assert lemo.lemo_segment_loss_workspace_size(T, V, S) == want, (T, V, S)
+    # the peak part scales with the segment rows, not with T
+    a = lemo.lemo_segment_loss_workspace_size(16384, 32000, 1024)
+    b = lemo.lemo_segment_loss_workspace_size(16384, 32000, 16384)
+    assert (b - a) == align(4 * 16384 * 32000) + align(2 * 16384 * 32000) - \
+        align(4 * 1024 * 32000) - align(2 * 1024 * 32000)
+    assert lemo.lemo_segment_loss_workspace_size(-1, 10, 4) == 0
+    assert lemo.lemo_segment_loss_workspace_size(10, 0, 4) == 0
+    assert lemo.lemo_segment_loss_workspace_size(10, 10, 0) == 0
+    buf, big = 0x10000, 1 << 40
+    f = lib.lemo_segment_loss
+    ok = [buf, 64, 10, 64, buf, 64, 100, buf, -100, 4, buf, None, buf, 64, buf, 64, buf, big, None]
+    def call(**kw):
+        args = list(ok)
+        names = ["h", "ld_h", "T", "d", "w", "ld_w", "V", "y", "ign", "seg", "loss", "tl", "dh",
+                 "ld_dh", "dw", "ld_dw", "ws", "ws_bytes", "st"]
+        for k, v in kw.items():
+            args[names.index(k)] = v
+        return f(*args)
+    assert call(d=12, ld_h=16, ld_w=16, ld_dh=16, ld_dw=16) == lemo.LEMO_ERR_UNSUPPORTED
+    assert call(ld_h=60) == lemo.LEMO_ERR_INVALID_ARG        # stride < d
+    assert call(ld_w=68) == lemo.LEMO_ERR_INVALID_ARG        # stride not a multiple of 8
+    assert call(h=buf + 8) == lemo.LEMO_ERR_INVALID_ARG      # misaligned h
+    assert call(seg=0) == lemo.LEMO_ERR_INVALID_ARG
+    assert call(loss=None) == lemo.LEMO_ERR_INVALID_ARG
+    assert call(ws_bytes=1024) == lemo.LEMO_ERR_INVALID_ARG  # workspace too small
+    assert call(ws=buf + 16) == lemo.LEMO_ERR_INVALID_ARG    # workspace not 256-aligned
+    assert call(dw=buf, ld_dw=32) == lemo.LEMO_ERR_INVALID_ARG
+
+
 TILE_CHECK = r"""
 #include <cstdio>
 #include <vector>
