@@ -39,4 +39,6 @@ from .lemo_oracle import (  # noqa: F401
     lm_head_loss,
     lm_head_loss_f64,
     lm_head_rows,
+    attention_kept,
+    attention_residual_exact,
 )

@@ -57,6 +57,12 @@ design notes of the repository):
     entropy of the lm-head logits over the tokens whose target is not the
     ignore index (0 when there is none); segmenting the tokens changes only
     the order of work, so the oracle is the unsegmented definition.
+13. Permutation-free attention: the kept tokens of a sequence attend to the
+    kept tokens of the same sequence at or before their own position (causal,
+    self included), softmax(scale Q K^T) V per head with scale 1/sqrt(dh) by
+    default; the attention output (heads concatenated, width H*dh) is added
+    in place into the residual rows of the kept tokens, whose width must be
+    H*dh.  An output projection, where a model has one, is the caller's.
 
 Each function below is pinned by tests under ``tests/`` against hand-worked
 values, closed forms, brute force on tiny inputs, library reductions or
@@ -90,6 +96,8 @@ __all__ = [
     "lm_head_loss",
     "lm_head_loss_f64",
     "lm_head_rows",
+    "attention_kept",
+    "attention_residual_exact",
 ]
 
 _BF16_MAX = (2.0 - 2.0 ** -7) * 2.0 ** 127
@@ -530,3 +538,62 @@ def lm_head_rows(h_bits, w_bits, targets, rows, n_valid: int, ignore_index: int 
         out_l.append(lse - z[yt])
         out_dh.append((p / n_valid) @ w)
     return np.asarray(out_l), np.asarray(out_dh).reshape(len(out_l), w.shape[1])
+
+
+# ---------------------------------------------------------------------------
+# Extension: permutation-free attention over the kept tokens (§4.2.3)
+# ---------------------------------------------------------------------------
+
+def attention_kept(q_bits, k_bits, v_bits, kept_idx, cu_kept, H: int, dh: int,
+                   scale: float | None = None) -> np.ndarray:
+    """Causal multi-head attention among the kept tokens, float64.
+
+    [Jenga] §4.2.3 "Permutation-free Token Movement": the attention reads the
+    kept tokens directly from their original rows (selective load) instead
+    of a re-permuted copy.  Kept rows r of sequence s are
+    kept_idx[cu_kept[s] : cu_kept[s+1]] (ascending positions); query r
+    attends to the kept keys r' of the same sequence with position
+    kept_idx[r'] <= kept_idx[r]:
+
+        O_r^h = sum_{r'} softmax_r'(scale * Q_r^h . K_r'^h) V_r'^h
+
+    ``q_bits``, ``k_bits``, ``v_bits``: bf16 [total_L, H*dh] in original token
+    order; scale defaults to 1/sqrt(dh).  Returns float64 [K, H*dh], row r
+    the output of kept token r.
+    """
+    if scale is None:
+        scale = 1.0 / math.sqrt(dh)
+    idx = np.asarray(kept_idx, dtype=np.int64)
+    cu = [int(c) for c in np.asarray(cu_kept)]
+    K = len(idx)
+    out = np.zeros((K, H * dh), dtype=np.float64)
+    for s in range(len(cu) - 1):
+        rows = idx[cu[s]:cu[s + 1]]
+        if len(rows) == 0:
+            continue
+        q = bf16_bits_to_f64(np.asarray(q_bits)[rows]).reshape(-1, H, dh)
+        k = bf16_bits_to_f64(np.asarray(k_bits)[rows]).reshape(-1, H, dh)
+        v = bf16_bits_to_f64(np.asarray(v_bits)[rows]).reshape(-1, H, dh)
+        n = len(rows)
+        allowed = rows[None, :] <= rows[:, None]  # key position <= query position
+        for h in range(H):
+            logits = scale * (q[:, h, :] @ k[:, h, :].T)
+            logits = np.where(allowed, logits, -np.inf)
+            m = logits.max(axis=1, keepdims=True)
+            p = np.exp(logits - m)
+            p /= p.sum(axis=1, keepdims=True)
+            out[cu[s]:cu[s] + n, h * dh:(h + 1) * dh] = p @ v[:, h, :]
+    return out
+
+
+def attention_residual_exact(x_bits, o, kept_idx) -> np.ndarray:
+    """The in-place addition of the attention output before rounding.
+
+    [Jenga] §4.2.3 "In-place Addition": row kept_idx[r] of x receives
+    x + O_r; every other row keeps its value.  Returns float64 [rows, d] (the
+    exact sums; the stored result is their bf16 rounding).
+    """
+    x = bf16_bits_to_f64(x_bits).copy()
+    idx = np.asarray(kept_idx, dtype=np.int64)
+    x[idx] += np.asarray(o, dtype=np.float64)
+    return x
