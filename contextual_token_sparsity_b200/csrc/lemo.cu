@@ -12,6 +12,7 @@
 #include <mutex>
 
 #include "lemo.h"
+#include "attn.cuh"
 #include "common.cuh"
 #include "mlp.cuh"
 #include "move.cuh"
@@ -116,6 +117,23 @@ bool encode_heads(CUtensorMap* tm, const uint16_t* base, int64_t rows, int64_t w
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
            CUDA_SUCCESS;
 }
+
+// 2-D view of a [rows, width] bf16 matrix with row stride ld (elements);
+// one box is 64 columns x 64 rows with 128-byte swizzle.
+bool encode_rows(CUtensorMap* tm, const uint16_t* base, int64_t rows, int64_t width, int64_t ld) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)width, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
+    const cuuint32_t box[2] = {(cuuint32_t)lemo::attn::KB, (cuuint32_t)lemo::attn::CHUNK};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(base), dims,
+               strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+bool g_attn_smem_set[kMaxDevices];
 
 // CTA pairs of the scoring kernel that fit on the device at once (one
 // persistent wave).  Sets the kernel's shared-memory limit on first use.
@@ -669,6 +687,77 @@ lemo_status lemo_predict_scores(const lemo_shape* shape, int32_t d, const uint16
     const int64_t cs_ctas = (p.tb + 7) / 8;
     const int cs_grid = (int)(cs_ctas < (int64_t)sms * 8 ? cs_ctas : sms * 8);
     lemo::score::column_sum_kernel<<<cs_grid, 256, 0, st>>>(P, w, lay, shape->batch, block_scores);
+    return launch_status();
+}
+
+size_t lemo_attention_workspace_size(int32_t batch) {
+    if (batch < 1) return 0;
+    return lemo::attn::ws_bytes(batch);
+}
+
+lemo_status lemo_attention_kept(const lemo_shape* shape, const uint16_t* q, const uint16_t* k,
+                                const uint16_t* v, int64_t ld_qkv, const int32_t* kept_idx,
+                                const int32_t* cu_kept, const int32_t* kept_total, float scale,
+                                uint16_t* x, int64_t ld_x, uint16_t* o, int64_t ld_o, void* ws,
+                                size_t ws_bytes, lemo_stream stream) {
+    namespace at = lemo::attn;
+    lemo_status e = check_shape(shape, true);
+    if (e != LEMO_OK) return e;
+    if (!q || !k || !v || !kept_idx || !cu_kept || !kept_total || !ws) return LEMO_ERR_INVALID_ARG;
+    if ((x == nullptr) == (o == nullptr)) return LEMO_ERR_INVALID_ARG;  // exactly one output
+    if (!(scale > 0.f) || !(scale < 3.0e38f)) return LEMO_ERR_INVALID_ARG;
+    const int64_t hd = (int64_t)shape->H * shape->dh;
+    if (ld_qkv < hd || ld_qkv % 8 != 0 || (x && (ld_x < hd || ld_x % 8 != 0)) ||
+        (o && (ld_o < hd || ld_o % 8 != 0)))
+        return LEMO_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || (x && !aligned(x, 16)) ||
+        (o && !aligned(o, 16)) || !aligned(kept_idx, 4) || !aligned(cu_kept, 4) ||
+        !aligned(kept_total, 4) || !aligned(ws, 256))
+        return LEMO_ERR_INVALID_ARG;
+    if (ws_bytes < at::ws_bytes(shape->batch)) return LEMO_ERR_INVALID_ARG;
+    const int64_t items = ((int64_t)shape->total_L + (int64_t)shape->batch * (at::BM - 1)) / at::BM;
+    if (items * shape->H >= (int64_t)1 << 31) return LEMO_ERR_UNSUPPORTED;
+    int dev = 0;
+    if (device_sms(&dev) <= 0) return LEMO_ERR_CUDA;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    char* w = static_cast<char*>(ws);
+    at::plan_kernel<<<1, 1024, 0, st>>>(cu_kept, kept_total, shape->cu_seqlens, shape->batch, w);
+    if ((e = launch_status()) != LEMO_OK) return e;
+    if (shape->total_L == 0 || items == 0) return LEMO_OK;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!g_attn_smem_set[dev]) {
+            if (cudaFuncSetAttribute(at::attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     at::SMEM_BYTES) != cudaSuccess)
+                return LEMO_ERR_CUDA;
+            g_attn_smem_set[dev] = true;
+        }
+    }
+    CUtensorMap tq, tk, tv;
+    if (!encode_rows(&tq, q, shape->total_L, hd, ld_qkv) ||
+        !encode_rows(&tk, k, shape->total_L, hd, ld_qkv) ||
+        !encode_rows(&tv, v, shape->total_L, hd, ld_qkv))
+        return LEMO_ERR_CUDA;
+    at::Args a;
+    a.kept_idx = kept_idx;
+    a.cu_kept = cu_kept;
+    a.cu_seqlens = shape->cu_seqlens;
+    a.batch = shape->batch;
+    a.H = shape->H;
+    a.dh = shape->dh;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.x = x;
+    a.ld_x = ld_x;
+    a.x_rows = shape->total_L;
+    a.o = o;
+    a.ld_o = ld_o;
+    a.ws = w;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        a.spin_limit_ns = (uint64_t)g_spin_ns;
+    }
+    at::attn_kernel<<<(unsigned)(items * shape->H), at::THREADS, at::SMEM_BYTES, st>>>(tq, tk, tv,
+                                                                                      a);
     return launch_status();
 }
 

@@ -63,6 +63,10 @@ _SIGS = {
     "lemo_predict_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(lemo_shape), _I32, _I32]),
     "lemo_predict_scores": (ctypes.c_int, [ctypes.POINTER(lemo_shape), _I32, _P, _I64, _P, _P, _P,
                                            _P, _I32, _P, _P, ctypes.c_size_t, _P]),
+    "lemo_attention_workspace_size": (ctypes.c_size_t, [_I32]),
+    "lemo_attention_kept": (ctypes.c_int, [ctypes.POINTER(lemo_shape), _P, _P, _P, _I64, _P, _P,
+                                           _P, ctypes.c_float, _P, _I64, _P, _I64, _P,
+                                           ctypes.c_size_t, _P]),
     "lemo_segment_loss_workspace_size": (ctypes.c_size_t, [_I64, _I32, _I32]),
     "lemo_segment_loss": (ctypes.c_int, [_P, _I64, _I64, _I32, _P, _I64, _I32, _P, _I32, _I32, _P,
                                          _P, _P, _I64, _P, _I64, _P, ctypes.c_size_t, _P]),
@@ -200,6 +204,25 @@ def lemo_predict_scores(shape, x, w1q, w2q, w1k, w2k, block_scores, ws, stream=N
                                       int(w1q.shape[1]), _ptr(block_scores), _ptr(ws),
                                       ws.numel() * ws.element_size(), _stream(stream)),
            "lemo_predict_scores")
+
+
+def lemo_attention_workspace_size(batch: int) -> int:
+    return int(load().lemo_attention_workspace_size(int(batch)))
+
+
+def lemo_attention_kept(shape, q, k, v, kept_idx, cu_kept, kept_total, ws, x=None, o=None,
+                        scale=None, stream=None):
+    """q, k, v bf16 [total_L, ld] 2-D tensors (same stride); exactly one of x
+    (residual, updated in place) or o (compact output) bf16 2-D tensors."""
+    import math
+    if scale is None:
+        scale = 1.0 / math.sqrt(shape.dh)
+    _check(load().lemo_attention_kept(
+        ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), q.stride(0), _ptr(kept_idx),
+        _ptr(cu_kept), _ptr(kept_total), float(scale), _ptr(x),
+        x.stride(0) if x is not None else 0, _ptr(o), o.stride(0) if o is not None else 0,
+        _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+        "lemo_attention_kept")
 
 
 def lemo_segment_loss_workspace_size(T: int, V: int, seg_rows: int) -> int:

@@ -330,6 +330,57 @@ LEMO_API lemo_status lemo_predict_scores(const lemo_shape* shape, int32_t d, con
                                          lemo_stream stream);
 
 /*
+ * Workspace bytes of lemo_attention_kept for `batch` sequences (the query
+ * tiles of each sequence and their prefix).  Returns 0 if batch < 1.
+ */
+LEMO_API size_t lemo_attention_workspace_size(int32_t batch);
+
+/*
+ * Permutation-free attention over the kept tokens (extension; replaces the
+ * gather -> attention -> scatter of steps a6-a7 by one kernel).
+ *
+ * Jenga summary, section 4.2.3, "Permutation-free Token Movement": instead
+ * of eliminating, re-permuting, padding and adding back, the attention
+ * kernel loads the kept tokens from their original rows (selective load) and
+ * adds its output in place into the original input (in-place addition).
+ * For every sequence s, kept rows r in [cu_kept[s], cu_kept[s+1]) at
+ * positions kept_idx[r] (ascending) and every head h:
+ *
+ *   O_r^h = sum_{r' <= r, same sequence} softmax_r'(scale * Q_r^h . K_r'^h) V_r'^h
+ *   x[kept_idx[r], h*dh:(h+1)*dh] = bf16(x + O_r^h)   (x != NULL: in place)
+ *   o[r, h*dh:(h+1)*dh]           = bf16(O_r^h)       (o != NULL: compact)
+ *
+ * Exactly one of x, o is given.  Rows of x of eliminated tokens are not
+ * touched; an output projection, where the model has one, is the caller's
+ * (then use o, the projection GEMM and lemo_scatter_residual).
+ *
+ * shape        batch, cu_seqlens (DEVICE), total_L, H, dh (64 or 128),
+ *              block (64 or 128) as for lemo_score_blocks.
+ * q, k, v      DEVICE bf16 [total_L, H*dh], row stride ld_qkv (elements,
+ *              multiple of 8), 16-byte aligned; original token order.
+ * kept_idx, cu_kept, kept_total   DEVICE int32, as written by lemo_select:
+ *              the kept rows must come as whole blocks of a multiple of 64
+ *              tokens (a sequence's last block may be short), i.e. every 64
+ *              consecutive kept rows counted from a sequence's first kept row
+ *              are consecutive positions of that sequence.  A violation is
+ *              reported as LEMO_ERR_INVALID_ARG by lemo_get_error.
+ * scale        softmax scale (> 0), usually 1/sqrt(dh).
+ * x, ld_x      DEVICE bf16 residual [total_L, >= H*dh], 16-byte aligned,
+ *              must not overlap q, k or v.
+ * o, ld_o      DEVICE bf16 [kept_total, >= H*dh], 16-byte aligned.
+ * ws, ws_bytes DEVICE workspace of lemo_attention_workspace_size(batch)
+ *              bytes, 256-byte aligned.
+ * tcgen05 tensor-core kernel: fp32 scores and accumulation, probabilities
+ * rounded to bf16 for the P V product, the output rounded once to bf16.
+ */
+LEMO_API lemo_status lemo_attention_kept(const lemo_shape* shape, const uint16_t* q,
+                                         const uint16_t* k, const uint16_t* v, int64_t ld_qkv,
+                                         const int32_t* kept_idx, const int32_t* cu_kept,
+                                         const int32_t* kept_total, float scale, uint16_t* x,
+                                         int64_t ld_x, uint16_t* o, int64_t ld_o, void* ws,
+                                         size_t ws_bytes, lemo_stream stream);
+
+/*
  * Workspace bytes of lemo_segment_loss for T tokens, vocabulary V and
  * segments of seg_rows tokens: the valid-token count, the per-token loss
  * terms, 32 MiB for the library GEMMs, and ONE segment's fp32 logits plus

@@ -41,4 +41,5 @@ from .lemo_oracle import (  # noqa: F401
     lm_head_rows,
     attention_kept,
     attention_residual_exact,
+    attention_kept_rows,
 )

@@ -98,6 +98,7 @@ __all__ = [
     "lm_head_rows",
     "attention_kept",
     "attention_residual_exact",
+    "attention_kept_rows",
 ]
 
 _BF16_MAX = (2.0 - 2.0 ** -7) * 2.0 ** 127
@@ -597,3 +598,26 @@ def attention_residual_exact(x_bits, o, kept_idx) -> np.ndarray:
     idx = np.asarray(kept_idx, dtype=np.int64)
     x[idx] += np.asarray(o, dtype=np.float64)
     return x
+
+
+def attention_kept_rows(q_bits, k_bits, v_bits, kept_idx, cu_kept, H: int, dh: int, rows,
+                        scale: float | None = None) -> np.ndarray:
+    """``attention_kept`` evaluated for the listed compact rows only (the same
+    definition, one query row at a time, for sampled rows of large inputs).
+    Returns float64 [len(rows), H*dh]."""
+    if scale is None:
+        scale = 1.0 / math.sqrt(dh)
+    idx = np.asarray(kept_idx, dtype=np.int64)
+    cu = np.asarray(cu_kept, dtype=np.int64)
+    out = np.zeros((len(rows), H * dh), dtype=np.float64)
+    for n, r in enumerate(rows):
+        s = int(np.searchsorted(cu, r, side="right")) - 1
+        keys = idx[cu[s]:r + 1]  # kept keys of the sequence up to row r (ascending)
+        q = bf16_bits_to_f64(np.asarray(q_bits)[idx[r]]).reshape(H, dh)
+        k = bf16_bits_to_f64(np.asarray(k_bits)[keys]).reshape(-1, H, dh)
+        v = bf16_bits_to_f64(np.asarray(v_bits)[keys]).reshape(-1, H, dh)
+        for h in range(H):
+            logits = scale * (k[:, h, :] @ q[h])
+            p = np.exp(logits - logits.max())
+            out[n, h * dh:(h + 1) * dh] = (p / p.sum()) @ v[:, h, :]
+    return out

@@ -123,3 +123,13 @@ def test_residual_touches_only_kept_rows():
     others = [i for i in range(10) if i not in idx]
     assert np.array_equal(ex[others], xf[others])
     np.testing.assert_array_equal(ex[idx], xf[idx] + o)
+
+
+def test_rows_helper_equals_full_definition():
+    lengths, H, dh, b = [90, 50], 2, 4, 8
+    q, k, v = _qkv(sum(lengths), H, dh, 8)
+    idx, cu_kept = _kept(lengths, b, 9)
+    full = oracle.attention_kept(q, k, v, idx, cu_kept, H, dh)
+    rows = [0, 1, int(cu_kept[1]) - 1, int(cu_kept[1]), len(idx) - 1]
+    got = oracle.attention_kept_rows(q, k, v, idx, cu_kept, H, dh, rows)
+    np.testing.assert_allclose(got, full[rows], rtol=1e-12, atol=1e-15)
