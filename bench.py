@@ -547,6 +547,419 @@ def run_segloss(args):
 
 
 # ----------------------------------------------------------------------------
+# extensions: attention over kept tokens, predicted path, MLP-block scores
+# ----------------------------------------------------------------------------
+
+ATTN_METRIC = "tokens/sec per layer of permutation-free attention over kept tokens"
+PREDICT_METRIC = "tokens/sec per layer (predicted score+select+gather+scatter)"
+MLP_METRIC = "tokens/sec per layer (MLP-block score+select+gather+scatter)"
+
+
+def _setup_device(world, local):
+    import torch
+    torch.cuda.set_device(local)
+    init_dist(world, "nccl")
+    dev = torch.device("cuda", local)
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        gpu_id = str(local)
+    return dev, gpu_id
+
+
+def _timed(step, steps, world, local, dev, gpu_id, n_marks=0):
+    """Run `steps` calls of step(evs) between two events on the current
+    stream (barrier + synchronize on both sides); step records its own
+    per-part events into evs (a list of n_marks events per step).  Returns
+    (elapsed seconds, clocks, per-step event lists)."""
+    import torch
+    stream = torch.cuda.current_stream(dev)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_marks)] for _ in range(steps)]
+    clocks = ClockSampler(gpu_id)
+    clocks.start()
+    time.sleep(0.3)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    barrier(world, local)
+    torch.cuda.synchronize()
+    a.record(stream)
+    for i in range(steps):
+        step(ev[i])
+    b.record(stream)
+    torch.cuda.synchronize()
+    barrier(world, local)
+    elapsed = a.elapsed_time(b) / 1e3
+    return elapsed, clocks.stop(), ev
+
+
+def _mean_us(ev, i0, i1):
+    return 1e3 * statistics.fmean(e[i0].elapsed_time(e[i1]) for e in ev)
+
+
+def _e2e(steps, world, local, dev, tokens, inputs, outputs, call):
+    """The same work through the C ABI with host buffers: every step copies
+    each (pinned host -> device) input pair in, runs call(), and copies each
+    (device -> pinned host) output pair out."""
+    import torch
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        for h, d in inputs:
+            d.copy_(h, non_blocking=True)
+        call()
+        for d, h in outputs:
+            h.copy_(d, non_blocking=True)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    barrier(world, local)
+    torch.cuda.synchronize()
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    barrier(world, local)
+    s = max_over_ranks(a.elapsed_time(b) / 1e3, world, dev) / steps
+    nb = lambda t: t.numel() * t.element_size()  # noqa: E731
+    return {"value": round(whole_job_rate(tokens, world, s), 1), "unit": UNIT,
+            "h2d_bytes_per_step": int(sum(nb(h) for h, _ in inputs)),
+            "d2h_bytes_per_step": int(sum(nb(h) for _, h in outputs)), "steps": steps,
+            "ms_per_step": round(1e3 * s, 3),
+            "path": "pinned host -> device copies, lemo_* calls, device -> pinned host copies"}
+
+
+def torch_empty_pinned(shape, dtype):
+    import torch
+    return torch.empty(shape, dtype=dtype).pin_memory()
+
+
+def _finish(out, world, local, rank):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def _header(metric, args, world, step_s, value):
+    return {"metric": metric, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_s * 1e3, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic"}
+
+
+def attention_flops(kept_per_seq, H, dh) -> float:
+    """Causal attention among K_s kept tokens: K_s (K_s + 1) / 2 query-key
+    pairs per head, 2 dh flops for the score and 2 dh for P V."""
+    return float(sum(2 * H * dh * K * (K + 1) for K in kept_per_seq))
+
+
+def run_attention(args):
+    """Attention over the kept tokens of the three c3 layers (keep 30/50/70 %),
+    added in place into the residual stream.  The keep masks come from the
+    path itself (score + select at set-up, with the stored thresholds)."""
+    import torch
+
+    from contextual_token_sparsity_b200 import lemo, synth
+    from contextual_token_sparsity_b200.pipeline import Layer, to_device_bf16
+
+    world, rank, local = dist_env()
+    dev, gpu_id = _setup_device(world, local)
+    lemo.load()
+    key = "c3"
+    w = synth.WORKLOADS[key]
+    nl = w.layers
+    thetas = thresholds(key, nl)
+    if thetas is None:
+        raise RuntimeError("stored thresholds tests/golden/c3.json are missing")
+    hd = w.H * w.dh
+    host = []
+    for l in range(nl):
+        inp = synth.make_workload(key, l, with_x=(l == 0))
+        inp["v"] = synth.normal_bf16(w.total_L, hd, int(w.seeds[l]), 22)
+        host.append(inp)
+    hx = host[0]["x"][:, :hd]
+    layers = [Layer(w.lengths, w.H, w.dh, w.block, hd, pad_to=PAD_TO, device=dev)
+              for _ in range(nl)]
+    q = [to_device_bf16(h["q"], dev) for h in host]
+    k = [to_device_bf16(h["k"], dev) for h in host]
+    v = [to_device_bf16(h["v"], dev) for h in host]
+    x = to_device_bf16(np.ascontiguousarray(hx), dev)
+    for l in range(nl):
+        layers[l].score(q[l], k[l])
+        layers[l].select(thetas[l])
+    ws = [torch.empty(lemo.lemo_attention_workspace_size(len(w.lengths)), dtype=torch.uint8,
+                      device=dev) for _ in range(nl)]
+    torch.cuda.synchronize()
+    cu_k = [L_.cu_kept.cpu().numpy() for L_ in layers]
+    kept_seq = [np.diff(c).tolist() for c in cu_k]
+    kept = [int(c[-1]) for c in cu_k]
+
+    def call(xx, qq=q, kk=k, vv=v, evs=None):
+        for l in range(nl):
+            if evs is not None:
+                evs[l].record()
+            L_ = layers[l]
+            lemo.lemo_attention_kept(L_.shape, qq[l], kk[l], vv[l], L_.kept_idx, L_.cu_kept,
+                                     L_.kept_total, ws[l], x=xx)
+        if evs is not None:
+            evs[nl].record()
+
+    for _ in range(args.warmup):
+        call(x)
+    torch.cuda.synchronize()
+    st = lemo.lemo_get_error()
+    if st != lemo.LEMO_OK:
+        raise RuntimeError(f"device error during warm-up: {lemo.STATUS.get(st, st)}")
+    elapsed, clk, ev = _timed(lambda e: call(x, evs=e), args.steps, world, local, dev, gpu_id,
+                              nl + 1)
+    st = lemo.lemo_get_error()
+    if st != lemo.LEMO_OK:
+        raise RuntimeError(f"device error in timed region: {lemo.STATUS.get(st, st)}")
+    step_s = max_over_ranks(elapsed, world, dev) / args.steps
+    per_layer_us = [_mean_us(ev, l, l + 1) for l in range(nl)]
+    peaks = load_peaks()
+    peak_tf = peaks["bf16_tflops_sustained"] if elapsed > 2.0 else peaks["bf16_tflops"]
+    flops = [attention_flops(kept_seq[l], w.H, w.dh) for l in range(nl)]
+    ach = [flops[l] / (per_layer_us[l] * 1e-6) / 1e12 for l in range(nl)]
+    tot_f = sum(flops)
+    tot_ach = tot_f / (sum(per_layer_us) * 1e-6) / 1e12
+    out = _header(ATTN_METRIC, args, world, step_s, whole_job_rate(nl * w.total_L, world, step_s))
+    out["config"] = {"workload": f"attn-c3: attention over the kept tokens of the {key} layers "
+                                 f"(L={w.total_L}, H={w.H}, dh={w.dh}, b={w.block}, keep "
+                                 f"30/50/70%), output added into the residual in place",
+                     "layers": nl, "kept_tokens": kept, "softmax_scale": "1/sqrt(dh)",
+                     "l2": "not flushed; each step reads 3 x 3 x 134 MB of Q/K/V rows "
+                           "(> 126 MB L2)",
+                     "parallelism": f"{world} independent replica(s), no collective"}
+    out["roofline"] = {"bound": "tensor", "kernel": "attn_kernel (+plan)",
+                       "achieved": round(tot_ach, 1), "peak": peak_tf, "unit": "TFLOP/s",
+                       "frac": round(tot_ach / peak_tf, 4), "traffic": None,
+                       "peak_source": f"{peaks['source']} bf16 "
+                                      f"{'sustained' if elapsed > 2.0 else 'burst'} cuBLAS GEMM",
+                       "algorithmic_flops_per_step": tot_f,
+                       "per_layer": [{"K": kept[l], "us": round(per_layer_us[l], 2),
+                                      "tflops": round(ach[l], 1)} for l in range(nl)]}
+    out["gpu_launches"] = 2 * nl * args.steps
+    out["clocks"] = clk
+    if not args.no_e2e:
+        pin = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).pin_memory()  # noqa
+        hq, hk, hv = ([pin(h[n]) for h in host] for n in ("q", "k", "v"))
+        hxp = pin(hx)
+        hx_out = torch_empty_pinned(hxp.shape, hxp.dtype)
+        dq = [torch.empty(t.shape, dtype=torch.int16, device=dev) for t in hq]
+        dk = [torch.empty(t.shape, dtype=torch.int16, device=dev) for t in hk]
+        dv = [torch.empty(t.shape, dtype=torch.int16, device=dev) for t in hv]
+        dx = torch.empty(hxp.shape, dtype=torch.int16, device=dev)
+        bf = lambda ts: [t.view(torch.bfloat16) for t in ts]  # noqa: E731
+        out["e2e"] = _e2e(max(3, min(args.steps, args.e2e_steps)), world, local, dev,
+                          nl * w.total_L,
+                          list(zip(hq, dq)) + list(zip(hk, dk)) + list(zip(hv, dv)) + [(hxp, dx)],
+                          [(dx, hx_out)],
+                          lambda: call(dx.view(torch.bfloat16), bf(dq), bf(dk), bf(dv)))
+    _finish(out, world, local, rank)
+
+
+def run_predict(args):
+    """The predicted path at the Llama-2-13B layer (c5): block means of X,
+    the two rank-256 ReLU predictors (pruned neurons left out: rank 154),
+    block products and column sums, then select / gather / scatter with the
+    stored predicted-score threshold."""
+    import torch
+
+    from contextual_token_sparsity_b200 import lemo, synth
+    from contextual_token_sparsity_b200.pipeline import Layer, to_device_bf16
+
+    world, rank, local = dist_env()
+    dev, gpu_id = _setup_device(world, local)
+    lemo.load()
+    key = "c5"
+    w = synth.WORKLOADS[key]
+    seed = int(w.seeds[0])
+    path = os.path.join(ROOT, "tests", "golden", f"{key}.json")
+    if not os.path.exists(path):
+        raise RuntimeError("stored thresholds tests/golden/c5.json are missing")
+    with open(path) as f:
+        theta = float(json.load(f)["layers"][0]["pred_theta"])
+    L, d, hd = w.total_L, w.d, w.H * w.dh
+    xb, _ = synth.projected_x(L, d, float(w.salient), seed)
+    w1q, w2q, liveq = synth.predictor_weights(d, w.predictor_rank, hd, 0.4, seed, 10)
+    w1k, w2k, livek = synth.predictor_weights(d, w.predictor_rank, hd, 0.4, seed, 11)
+    w1q, w2q = np.ascontiguousarray(w1q[:, liveq]), np.ascontiguousarray(w2q[liveq])
+    w1k, w2k = np.ascontiguousarray(w1k[:, livek]), np.ascontiguousarray(w2k[livek])
+    y_out = synth.normal_bf16(L, d, seed, 8)
+    layer = Layer(w.lengths, w.H, w.dh, w.block, d, pad_to=PAD_TO, device=dev)
+    x = to_device_bf16(xb, dev)
+    dw = [to_device_bf16(a, dev) for a in (w1q, w2q, w1k, w2k)]
+    yd = to_device_bf16(y_out, dev)
+    rank_eff = int(w1q.shape[1])
+    pws = torch.empty(lemo.lemo_predict_workspace_size(layer.shape, d, rank_eff),
+                      dtype=torch.uint8, device=dev)
+
+    def call(xx, yy, evs=None):
+        if evs is not None:
+            evs[0].record()
+        lemo.lemo_predict_scores(layer.shape, xx, *dw, layer.block_scores, pws)
+        if evs is not None:
+            evs[1].record()
+        layer.select(theta)
+        if evs is not None:
+            evs[2].record()
+        layer.gather(xx)
+        if evs is not None:
+            evs[3].record()
+        layer.scatter(xx, yy)
+        if evs is not None:
+            evs[4].record()
+
+    for _ in range(args.warmup):
+        call(x, yd)
+    torch.cuda.synchronize()
+    st = lemo.lemo_get_error()
+    if st != lemo.LEMO_OK:
+        raise RuntimeError(f"device error during warm-up: {lemo.STATUS.get(st, st)}")
+    K = int(layer.kept_total.item())
+    elapsed, clk, ev = _timed(lambda e: call(x, yd, e), args.steps, world, local, dev, gpu_id, 5)
+    st = lemo.lemo_get_error()
+    if st != lemo.LEMO_OK:
+        raise RuntimeError(f"device error in timed region: {lemo.STATUS.get(st, st)}")
+    step_s = max_over_ranks(elapsed, world, dev) / args.steps
+    us = {n: _mean_us(ev, i, i + 1) for i, n in enumerate(("predict", "select", "gather",
+                                                              "scatter"))}
+    peaks = load_peaks()
+    pool_bytes = 2 * L * d  # X read once for the block means
+    g_b, s_b = move_bytes(K, d)
+    tb = -(-L // w.block)
+    pred_flops = 2 * 2 * tb * (d * rank_eff + rank_eff * hd) + tb * (tb + 1) * hd
+    bw = peaks["hbm_gbs"]
+    out = _header(PREDICT_METRIC, args, world, step_s, whole_job_rate(L, world, step_s))
+    out["config"] = {"workload": f"predict-c5: {w.name}", "seq_lens": list(w.lengths),
+                     "heads": w.H, "head_dim": w.dh, "block": w.block, "d": d,
+                     "predictor_rank": w.predictor_rank, "live_neurons": [len(liveq), len(livek)],
+                     "keep": 0.5, "kept_tokens": K, "threshold_source":
+                     "oracle predicted scores (tests/golden)",
+                     "l2": "not flushed; each step reads the 335 MB X twice (> 126 MB L2)",
+                     "parallelism": f"{world} independent replica(s), no collective"}
+    pred_gbs = pool_bytes / (us["predict"] * 1e-6) / 1e9
+    out["roofline"] = {"bound": "hbm", "kernel": "lemo_predict_scores (pool + predictor GEMMs "
+                       "+ block products + column sum)", "achieved": round(pred_gbs, 1),
+                       "peak": bw, "unit": "GB/s", "frac": round(pred_gbs / bw, 4),
+                       "traffic": None, "algorithmic_bytes_per_call": pool_bytes,
+                       "predictor_flops_per_call": pred_flops}
+    out["kernels_us"] = {n: round(v, 2) for n, v in us.items()}
+    out["movement"] = {"gather_gbs": round(g_b / (us["gather"] * 1e-6) / 1e9, 1),
+                       "scatter_gbs": round(s_b / (us["scatter"] * 1e-6) / 1e9, 1),
+                       "hbm_peak_gbs": bw}
+    # predict: plan, pool, 2 x (gemm, reduce, gemm), products, column sum;
+    # select: plan, select; gather; scatter
+    out["gpu_launches"] = 14 * args.steps
+    out["clocks"] = clk
+    if not args.no_e2e:
+        pin = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).pin_memory()  # noqa
+        hxp, hyp = pin(xb), pin(y_out)
+        hx_out = torch_empty_pinned(hxp.shape, hxp.dtype)
+        hs = torch_empty_pinned(layer.block_scores.shape, torch.float32)
+        dx = torch.empty(hxp.shape, dtype=torch.int16, device=dev)
+        dy = torch.empty(hyp.shape, dtype=torch.int16, device=dev)
+        out["e2e"] = _e2e(max(3, min(args.steps, args.e2e_steps)), world, local, dev, L,
+                          [(hxp, dx), (hyp, dy)], [(dx, hx_out), (layer.block_scores, hs)],
+                          lambda: call(dx.view(torch.bfloat16), dy.view(torch.bfloat16)))
+    _finish(out, world, local, rank)
+
+
+def run_mlp(args):
+    """MLP-block elimination at the Llama-2-7B layer (L = 16384, SiLU-gated
+    d_ff = 11008, b = 64): token scores from SiLU(gate) * up, block maxima,
+    keep mask at 50 %, gather / scatter of d = 4096 rows."""
+    import torch
+
+    from contextual_token_sparsity_b200 import lemo, synth
+    from contextual_token_sparsity_b200.pipeline import Layer, to_device_bf16
+
+    world, rank, local = dist_env()
+    dev, gpu_id = _setup_device(world, local)
+    lemo.load()
+    L, d_ff, d, b, seed = 16384, 11008, 4096, 64, 0
+    gate, up = synth.mlp_activations(L, d_ff, 0.1, seed=seed, gated=True)
+    xb = synth.normal_bf16(L, d, seed, 7)
+    y_out = synth.normal_bf16(L, d, seed, 8)
+    layer = Layer([L], 1, 64, b, d, pad_to=PAD_TO, device=dev)
+    g_d, u_d = to_device_bf16(gate, dev), to_device_bf16(up, dev)
+    x, yd = to_device_bf16(xb, dev), to_device_bf16(y_out, dev)
+    lemo.lemo_mlp_block_scores(layer.shape, layer.block_scores, layer.ws, gate=g_d, up=u_d)
+    s = np.sort(layer.block_scores[: layer.total_blocks].cpu().numpy().astype(np.float64))[::-1]
+    kk = int(math.floor(0.5 * s.size + 0.5))
+    theta = float(0.5 * (s[kk - 1] + s[kk]))
+
+    def call(gg, uu, xx, yy, evs=None):
+        if evs is not None:
+            evs[0].record()
+        lemo.lemo_mlp_block_scores(layer.shape, layer.block_scores, layer.ws, gate=gg, up=uu)
+        if evs is not None:
+            evs[1].record()
+        layer.select(theta)
+        if evs is not None:
+            evs[2].record()
+        layer.gather(xx)
+        if evs is not None:
+            evs[3].record()
+        layer.scatter(xx, yy)
+        if evs is not None:
+            evs[4].record()
+
+    for _ in range(args.warmup):
+        call(g_d, u_d, x, yd)
+    torch.cuda.synchronize()
+    st = lemo.lemo_get_error()
+    if st != lemo.LEMO_OK:
+        raise RuntimeError(f"device error during warm-up: {lemo.STATUS.get(st, st)}")
+    K = int(layer.kept_total.item())
+    elapsed, clk, ev = _timed(lambda e: call(g_d, u_d, x, yd, e), args.steps, world, local, dev,
+                              gpu_id, 5)
+    st = lemo.lemo_get_error()
+    if st != lemo.LEMO_OK:
+        raise RuntimeError(f"device error in timed region: {lemo.STATUS.get(st, st)}")
+    step_s = max_over_ranks(elapsed, world, dev) / args.steps
+    us = {n: _mean_us(ev, i, i + 1) for i, n in enumerate(("mlp_score", "select", "gather",
+                                                              "scatter"))}
+    peaks = load_peaks()
+    bw = peaks["hbm_gbs"]
+    score_bytes = 4 * L * d_ff  # gate and up read once
+    gbs = score_bytes / (us["mlp_score"] * 1e-6) / 1e9
+    g_b, s_b = move_bytes(K, d)
+    out = _header(MLP_METRIC, args, world, step_s, whole_job_rate(L, world, step_s))
+    out["config"] = {"workload": f"mlp-7b: L={L}, SiLU-gated d_ff={d_ff}, b={b}, d={d}, "
+                                 "keep 50%", "kept_tokens": K,
+                     "threshold_source": "keep ratio on the kernel's own block scores",
+                     "l2": "not flushed; each step reads 721 MB of activations (> 126 MB L2)",
+                     "parallelism": f"{world} independent replica(s), no collective"}
+    out["roofline"] = {"bound": "hbm", "kernel": "mlp::block_scores_kernel (+plan, column "
+                       "max)", "achieved": round(gbs, 1), "peak": bw, "unit": "GB/s",
+                       "frac": round(gbs / bw, 4), "traffic": None,
+                       "algorithmic_bytes_per_call": score_bytes}
+    out["kernels_us"] = {n: round(v, 2) for n, v in us.items()}
+    out["movement"] = {"gather_gbs": round(g_b / (us["gather"] * 1e-6) / 1e9, 1),
+                       "scatter_gbs": round(s_b / (us["scatter"] * 1e-6) / 1e9, 1),
+                       "hbm_peak_gbs": bw}
+    out["gpu_launches"] = 6 * args.steps  # plan + scores, plan + select, gather, scatter
+    out["clocks"] = clk
+    if not args.no_e2e:
+        pin = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).pin_memory()  # noqa
+        hg, hu, hxp, hyp = pin(gate), pin(up), pin(xb), pin(y_out)
+        hx_out = torch_empty_pinned(hxp.shape, hxp.dtype)
+        dd = [torch.empty(t.shape, dtype=torch.int16, device=dev) for t in (hg, hu, hxp, hyp)]
+        out["e2e"] = _e2e(max(3, min(args.steps, args.e2e_steps)), world, local, dev, L,
+                          list(zip((hg, hu, hxp, hyp), dd)), [(dd[2], hx_out)],
+                          lambda: call(*[t.view(torch.bfloat16) for t in dd]))
+    _finish(out, world, local, rank)
+
+
+# ----------------------------------------------------------------------------
 # the CPU oracle (cpu_baseline leg and reference arm)
 # ----------------------------------------------------------------------------
 
@@ -680,7 +1093,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["lemo", "reference"], default="lemo")
     ap.add_argument("--workload", default="c3",
-                    choices=["c1", "c2", "c3", "c4", "c5", "lmhead-7b"])
+                    choices=["c1", "c2", "c3", "c4", "c5", "lmhead-7b", "attn-c3",
+                             "predict-c5", "mlp-7b"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -691,12 +1105,14 @@ def main(argv=None):
     world = dist_env()[0]
     if args.gpus != world and world > 1:
         ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}")
-    if args.workload.startswith("lmhead"):
+    extensions = {"lmhead-7b": run_segloss, "attn-c3": run_attention,
+                  "predict-c5": run_predict, "mlp-7b": run_mlp}
+    if args.workload in extensions:
         if args.impl == "reference":
             print(json.dumps({"impl": "reference", "unavailable": "the oracle arm covers the "
                               "per-layer path workloads only"}), flush=True)
         else:
-            run_segloss(args)
+            extensions[args.workload](args)
     elif args.impl == "reference":
         run_reference(args)
     else:
