@@ -139,6 +139,7 @@ struct Args {
 __global__ void __launch_bounds__(1024)
     plan_kernel(const int32_t* __restrict__ cu_kept, const int32_t* __restrict__ kept_total,
                 const int32_t* __restrict__ cu_seqlens, int batch, char* __restrict__ ws) {
+    pdl_entry();
     __shared__ int sum32[32];
     __shared__ int bad;
     WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
@@ -300,6 +301,7 @@ __device__ __forceinline__ void load_tile(const CUtensorMap* tm, uint8_t* dst, i
 __global__ void __launch_bounds__(THREADS, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const Args a) {
+    pdl_entry();
     const WsHeader* hdr = reinterpret_cast<const WsHeader*>(a.ws);
     const int32_t* prefix = reinterpret_cast<const int32_t*>(a.ws + kWsPrefix);
     if (!hdr->valid) return;

@@ -20,6 +20,17 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     return t;
 }
 
+// Programmatic dependent launch.  The host launches every kernel of the
+// library with programmatic stream serialization, so a kernel's CTAs may be
+// scheduled before the previous kernel in the stream has finished.  Each
+// kernel therefore calls pdl_entry() before anything else: it waits until
+// the previous kernel has completed and its memory writes are visible, then
+// lets the next kernel be scheduled.  For a plain launch both are no-ops.
+__device__ __forceinline__ void pdl_entry() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 template <typename T>
 __host__ __device__ __forceinline__ T ceil_div(T a, T b) { return (a + b - 1) / b; }
 

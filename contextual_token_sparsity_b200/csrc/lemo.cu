@@ -10,6 +10,7 @@
 
 #include <climits>
 #include <mutex>
+#include <utility>
 
 #include "lemo.h"
 #include "attn.cuh"
@@ -62,8 +63,34 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return g_encode;
 }
 
+// Every kernel of the library starts with griddepcontrol.wait (pdl_wait),
+// so each one may be launched with programmatic stream serialization: its
+// CTAs can be scheduled while the previous kernel in the stream drains, and
+// they touch no memory before that kernel has completed.  Launch errors are
+// kept for the next launch_status().
+thread_local cudaError_t t_launch_error = cudaSuccess;
+
+template <typename... P, typename... A>
+void launch(void (*kernel)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+            A&&... args) {
+    cudaLaunchConfig_t c = {};
+    c.gridDim = grid;
+    c.blockDim = block;
+    c.dynamicSmemBytes = smem;
+    c.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    c.attrs = at;
+    c.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&c, kernel, std::forward<A>(args)...);
+    if (e != cudaSuccess && t_launch_error == cudaSuccess) t_launch_error = e;
+}
+
 lemo_status launch_status() {
-    return cudaGetLastError() == cudaSuccess ? LEMO_OK : LEMO_ERR_CUDA;
+    const cudaError_t launch_e = t_launch_error;
+    t_launch_error = cudaSuccess;
+    return (cudaGetLastError() == cudaSuccess && launch_e == cudaSuccess) ? LEMO_OK : LEMO_ERR_CUDA;
 }
 
 // Shape checks common to scoring and selection.
@@ -95,8 +122,8 @@ lemo_status check_ws(const lemo_shape* s, const void* ws, size_t ws_bytes) {
 
 void launch_plan(const lemo_shape* s, char* ws, const lemo::WsLayout& lay, int32_t* zero_word,
                  cudaStream_t st, float* zero_blocks = nullptr) {
-    lemo::plan_kernel<<<1, 1024, 0, st>>>(s->cu_seqlens, s->batch, s->total_L, s->max_seqlen,
-                                          s->block, ws, lay, zero_word, zero_blocks);
+    launch(lemo::plan_kernel, 1, 1024, 0, st, s->cu_seqlens, s->batch, s->total_L, s->max_seqlen,
+           s->block, ws, lay, zero_word, zero_blocks);
 }
 
 // 3-D view of a [rows, H*dh] bf16 matrix as (64 elements, rows, H*dh/64
@@ -203,30 +230,52 @@ lemo_status check_move(const void* x, int64_t ld_x, int64_t x_rows, int32_t d, c
 // region holds the block products P) followed by the predictor buffers.
 struct PredictLayout {
     lemo::WsLayout base;
-    size_t xbar, hq, hk, part, qh, kh, total;
+    size_t xbar, part, hid, qh, kh, ppart, total;
     int64_t tb;      // upper bound of the number of token blocks
     int splits;      // split-K factor of the first predictor GEMM
+    int k_chunk;     // K range of one split
+    int hpg;         // heads per group of the block products
+    int groups;      // head groups (partial planes when > 1)
+    int64_t ptiles;  // lower-triangular 64 x 64 tiles of block pairs
 };
 
+// The launch shapes depend only on the shape (not on the device), so the
+// workspace size query and the call agree.  The first GEMM is split along K
+// until about four CTAs per SM of a B200 (148 SMs) are busy, with at least
+// four K stages each: its loop is latency-bound, so shorter loops on more
+// SMs finish sooner.  The block products aim at two CTAs per SM.
 PredictLayout predict_layout(const lemo_shape* s, int d, int rank) {
+    namespace pr = lemo::predict;
+    constexpr int64_t kGemmCtas = 592, kTargetCtas = 296;
     PredictLayout p;
     p.base = layout_of(s);
     p.tb = ((int64_t)s->total_L + (int64_t)s->batch * (s->block - 1)) / s->block;
     if (p.tb < 1) p.tb = 1;
     const int64_t hd = (int64_t)s->H * s->dh;
-    const int64_t tiles = ((rank + 63) / 64) * ((p.tb + 63) / 64);
-    int64_t splits = (296 + tiles - 1) / tiles;  // about two CTAs per SM
-    const int64_t max_splits = (d + 255) / 256;   // at least 256 of K per split
+    const int64_t mt = (p.tb + pr::TM - 1) / pr::TM;
+    const int64_t tiles = 2 * ((rank + pr::TN - 1) / pr::TN) * mt;
+    const int64_t kst = (d + pr::TK - 1) / pr::TK;        // K stages of the first GEMM
+    int64_t splits = (kGemmCtas + tiles - 1) / tiles;
+    const int64_t max_splits = (kst + 3) / 4;              // at least 4 stages per split
     if (splits > max_splits) splits = max_splits;
     if (splits < 1) splits = 1;
-    p.splits = (int)splits;
+    p.k_chunk = (int)((kst + splits - 1) / splits * pr::TK);
+    p.splits = (int)((d + p.k_chunk - 1) / p.k_chunk);
+    p.ptiles = mt * (mt + 1) / 2;
+    int64_t groups = (kTargetCtas + p.ptiles - 1) / p.ptiles;
+    if (groups > s->H) groups = s->H;
+    while (groups > 1 && groups * p.tb * p.tb * 4 > ((int64_t)64 << 20)) --groups;
+    if (groups < 1) groups = 1;
+    p.hpg = (int)((s->H + groups - 1) / groups);
+    p.groups = (s->H + p.hpg - 1) / p.hpg;
     size_t off = p.base.total;
-    p.xbar = off; off = lemo::align_up(off + 4 * (size_t)p.tb * d, 256);
-    p.hq = off;   off = lemo::align_up(off + 4 * (size_t)p.tb * rank, 256);
-    p.hk = off;   off = lemo::align_up(off + 4 * (size_t)p.tb * rank, 256);
-    p.part = off; off = lemo::align_up(off + 4 * (size_t)p.splits * p.tb * rank, 256);
-    p.qh = off;   off = lemo::align_up(off + 4 * (size_t)p.tb * hd, 256);
-    p.kh = off;   off = lemo::align_up(off + 4 * (size_t)p.tb * hd, 256);
+    p.xbar = off;  off = lemo::align_up(off + 4 * (size_t)p.tb * d, 256);
+    p.part = off;  off = lemo::align_up(off + 4 * (size_t)2 * p.splits * p.tb * rank, 256);
+    p.hid = off;   off = lemo::align_up(off + 4 * (size_t)2 * p.tb * rank, 256);
+    p.qh = off;    off = lemo::align_up(off + 4 * (size_t)p.tb * hd, 256);
+    p.kh = off;    off = lemo::align_up(off + 4 * (size_t)p.tb * hd, 256);
+    p.ppart = off;
+    if (p.groups > 1) off = lemo::align_up(off + 4 * (size_t)p.groups * p.tb * p.tb, 256);
     p.total = off;
     return p;
 }
@@ -380,14 +429,15 @@ lemo_status lemo_score_blocks(const lemo_shape* shape, const uint16_t* q, const 
         a.ws = w;
         a.lay = lay;
         a.spin_limit_ns = (uint64_t)g_spin_ns;
-        sc::score_tiles_kernel<<<2 * pairs, sc::THREADS, sc::SMEM_BYTES, st>>>(tm_q, tm_k, a);
+        launch(sc::score_tiles_kernel, 2 * pairs, sc::THREADS, sc::SMEM_BYTES, st, tm_q, tm_k, a);
         if ((e = launch_status()) != LEMO_OK) return e;
         // one warp per token block; the host knows an upper bound of their number
         const int64_t nb_bound =
             ((int64_t)shape->total_L + (int64_t)shape->batch * (shape->block - 1)) / shape->block;
         const int64_t cs_ctas = (nb_bound + 7) / 8;
         const int cs_grid = (int)(cs_ctas < (int64_t)sms * 8 ? (cs_ctas > 0 ? cs_ctas : 1) : sms * 8);
-        sc::column_sum_kernel<<<cs_grid, 256, 0, st>>>(mblk, w, lay, shape->batch, block_scores);
+        launch(sc::column_sum_kernel, cs_grid, 256, 0, st, mblk, w, lay, shape->batch,
+               block_scores);
         if ((e = launch_status()) != LEMO_OK) return e;
     }
     return LEMO_OK;
@@ -424,7 +474,7 @@ lemo_status lemo_select(const lemo_shape* shape, const float* block_scores, floa
     a.lay = lay;
     a.skip_publish_tile = g_skip_publish_tile;
     a.spin_limit_ns = (uint64_t)g_spin_ns;
-    lemo::select_kernel<<<(unsigned)lay.n_lookback, lemo::kSelectThreads, 0, st>>>(a);
+    launch(lemo::select_kernel, (unsigned)lay.n_lookback, lemo::kSelectThreads, 0, st, a);
     return launch_status();
 }
 
@@ -522,8 +572,8 @@ lemo_status lemo_gather_pad(const uint16_t* x, int64_t ld_x, int64_t x_rows, int
     a.kept_total = kept_total;
     a.pad_to = pad_to;
     a.cap = y_rows_capacity;
-    lemo::gather_pad_kernel<<<move_grid(dev, sms, 0, lemo::gather_pad_kernel), lemo::kMoveThreads, 0,
-                              reinterpret_cast<cudaStream_t>(stream)>>>(a);
+    launch(lemo::gather_pad_kernel, move_grid(dev, sms, 0, lemo::gather_pad_kernel),
+           lemo::kMoveThreads, 0, reinterpret_cast<cudaStream_t>(stream), a);
     return launch_status();
 }
 
@@ -546,9 +596,8 @@ lemo_status lemo_scatter_residual(uint16_t* x, int64_t ld_x, int64_t x_rows, int
     a.kept_total = kept_total;
     a.pad_to = 1;
     a.cap = 0;
-    lemo::scatter_residual_kernel<<<move_grid(dev, sms, 1, lemo::scatter_residual_kernel),
-                                    lemo::kMoveThreads, 0,
-                                    reinterpret_cast<cudaStream_t>(stream)>>>(a);
+    launch(lemo::scatter_residual_kernel, move_grid(dev, sms, 1, lemo::scatter_residual_kernel),
+           lemo::kMoveThreads, 0, reinterpret_cast<cudaStream_t>(stream), a);
     return launch_status();
 }
 
@@ -571,9 +620,8 @@ lemo_status lemo_recompute_input(uint16_t* x, int64_t ld_x, int64_t x_rows, int3
     a.kept_total = kept_total;
     a.pad_to = 1;
     a.cap = 0;
-    lemo::recompute_input_kernel<<<move_grid(dev, sms, 2, lemo::recompute_input_kernel),
-                                   lemo::kMoveThreads, 0,
-                                   reinterpret_cast<cudaStream_t>(stream)>>>(a);
+    launch(lemo::recompute_input_kernel, move_grid(dev, sms, 2, lemo::recompute_input_kernel),
+           lemo::kMoveThreads, 0, reinterpret_cast<cudaStream_t>(stream), a);
     return launch_status();
 }
 
@@ -616,7 +664,7 @@ lemo_status lemo_mlp_block_scores(const lemo_shape* shape, int32_t d_ff, const u
     const int64_t ctas_needed =
         ((int64_t)shape->total_L + lemo::mlp::kThreads / 32 - 1) / (lemo::mlp::kThreads / 32);
     const int64_t grid = ctas_needed < (int64_t)sms * 4 ? ctas_needed : (int64_t)sms * 4;
-    lemo::mlp::block_scores_kernel<<<(unsigned)grid, lemo::mlp::kThreads, 0, st>>>(a);
+    launch(lemo::mlp::block_scores_kernel, (unsigned)grid, lemo::mlp::kThreads, 0, st, a);
     return launch_status();
 }
 
@@ -648,45 +696,82 @@ lemo_status lemo_predict_scores(const lemo_shape* shape, int32_t d, const uint16
     const lemo::PlanHeader* hdr = reinterpret_cast<const lemo::PlanHeader*>(w + lay.hdr);
     float* xbar = reinterpret_cast<float*>(w + p.xbar);
     float* part = reinterpret_cast<float*>(w + p.part);
+    float* hid = reinterpret_cast<float*>(w + p.hid);
     float* P = reinterpret_cast<float*>(w + lay.mblk);
     const int hd = shape->H * shape->dh;
 
     launch_plan(shape, w, lay, nullptr, st);
     if ((e = launch_status()) != LEMO_OK) return e;
     if (shape->total_L == 0) return LEMO_OK;
-    const unsigned ytiles = (unsigned)((p.tb + pr::GT - 1) / pr::GT);
-    pr::pool_kernel<<<dim3((unsigned)p.tb, (unsigned)((d + pr::kPoolCols - 1) / pr::kPoolCols)),
-                      pr::kPoolThreads, 0, st>>>(x, ld_x, d, shape->cu_seqlens, shape->batch,
-                                                 shape->block, w, lay, xbar);
+    launch(pr::pool_kernel,
+           dim3((unsigned)p.tb, (unsigned)((d + pr::kPoolCols - 1) / pr::kPoolCols)),
+           pr::kPoolThreads, 0, st, x, ld_x, d, shape->cu_seqlens, shape->batch, shape->block, w,
+           lay, xbar);
     if ((e = launch_status()) != LEMO_OK) return e;
-    const int kchunk = ((d + p.splits - 1) / p.splits + pr::GK - 1) / pr::GK * pr::GK;
-    for (int side = 0; side < 2; ++side) {
-        const uint16_t* w1 = side == 0 ? w1q : w1k;
-        const uint16_t* w2 = side == 0 ? w2q : w2k;
-        float* hid = reinterpret_cast<float*>(w + (side == 0 ? p.hq : p.hk));
-        float* out = reinterpret_cast<float*>(w + (side == 0 ? p.qh : p.kh));
-        pr::gemm_kernel<<<dim3((unsigned)((rank + pr::GT - 1) / pr::GT), ytiles, (unsigned)p.splits),
-                          256, 0, st>>>(xbar, d, w1, rank, part, hdr, rank, d, kchunk);
-        pr::reduce_kernel<<<sms * 4, 256, 0, st>>>(part, p.splits, hdr, rank, true, hid);
-        pr::gemm_kernel<<<dim3((unsigned)((hd + pr::GT - 1) / pr::GT), ytiles, 1), 256, 0, st>>>(
-            hid, rank, w2, hd, out, hdr, hd, rank, rank);
-        if ((e = launch_status()) != LEMO_OK) return e;
-    }
-    const unsigned ptiles = (unsigned)((p.tb + pr::PT - 1) / pr::PT);
-    const size_t psmem = 2 * sizeof(float) * pr::PT * (shape->dh + 1);
-    if (psmem > 48 * 1024) {
-        std::lock_guard<std::mutex> lk(g_mu);
-        if (cudaFuncSetAttribute(pr::products_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)psmem) != cudaSuccess)
-            return LEMO_ERR_CUDA;
-    }
-    pr::products_kernel<<<dim3(ptiles, ptiles), pr::PT * pr::PT, psmem, st>>>(
-        reinterpret_cast<float*>(w + p.qh), reinterpret_cast<float*>(w + p.kh), shape->H,
-        shape->dh, shape->batch, w, lay, 1.f / (float)shape->H, P);
+    const unsigned mtiles = (unsigned)((p.tb + pr::TM - 1) / pr::TM);
+    // hidden layers of both predictors: split-K partials, then relu of their sum
+    pr::GemmArgs g1;
+    g1.a[0] = g1.a[1] = xbar;
+    g1.lda = d;
+    g1.w[0] = w1q;
+    g1.w[1] = w1k;
+    g1.ldw = rank;
+    g1.c[0] = part;
+    g1.c[1] = part + (int64_t)p.splits * p.tb * rank;
+    g1.ldc = rank;
+    g1.c_split = p.tb * rank;
+    g1.hdr = hdr;
+    g1.N = rank;
+    g1.K = d;
+    g1.k_chunk = p.k_chunk;
+    g1.splits = p.splits;
+    launch(pr::gemm_kernel, dim3((unsigned)((rank + pr::TN - 1) / pr::TN), mtiles, 2u * p.splits),
+           pr::kMmaThreads, 0, st, g1);
+    launch(pr::reduce_kernel, dim3((unsigned)sms, 2u), 256, 0, st, part,
+           (int64_t)p.splits * p.tb * rank, p.tb * rank, p.splits, hdr, rank, hid, p.tb * rank);
+    // block embeddings of both predictors
+    pr::GemmArgs g2;
+    g2.a[0] = hid;
+    g2.a[1] = hid + p.tb * rank;
+    g2.lda = rank;
+    g2.w[0] = w2q;
+    g2.w[1] = w2k;
+    g2.ldw = hd;
+    g2.c[0] = reinterpret_cast<float*>(w + p.qh);
+    g2.c[1] = reinterpret_cast<float*>(w + p.kh);
+    g2.ldc = hd;
+    g2.c_split = 0;
+    g2.hdr = hdr;
+    g2.N = hd;
+    g2.K = rank;
+    g2.k_chunk = (rank + pr::TK - 1) / pr::TK * pr::TK;
+    g2.splits = 1;
+    launch(pr::gemm_kernel, dim3((unsigned)((hd + pr::TN - 1) / pr::TN), mtiles, 2u),
+           pr::kMmaThreads, 0, st, g2);
+    if ((e = launch_status()) != LEMO_OK) return e;
+    // block products, mean over heads of the positive parts
+    pr::ProductsArgs pa;
+    pa.qh = g2.c[0];
+    pa.kh = g2.c[1];
+    pa.H = shape->H;
+    pa.dh = shape->dh;
+    pa.hpg = p.hpg;
+    pa.groups = p.groups;
+    pa.batch = shape->batch;
+    pa.tb_cap = p.tb;
+    pa.inv_h = 1.f / (float)shape->H;
+    pa.part = reinterpret_cast<float*>(w + p.ppart);
+    pa.P = P;
+    launch(pr::products_kernel, dim3((unsigned)p.ptiles, (unsigned)p.groups), pr::kMmaThreads, 0,
+           st, pa, w, lay);
     if ((e = launch_status()) != LEMO_OK) return e;
     const int64_t cs_ctas = (p.tb + 7) / 8;
     const int cs_grid = (int)(cs_ctas < (int64_t)sms * 8 ? cs_ctas : sms * 8);
-    lemo::score::column_sum_kernel<<<cs_grid, 256, 0, st>>>(P, w, lay, shape->batch, block_scores);
+    if (p.groups > 1)
+        launch(pr::plane_column_sum_kernel, cs_grid, 256, 0, st, pa, w, lay, block_scores);
+    else
+        launch(lemo::score::column_sum_kernel, cs_grid, 256, 0, st, P, w, lay, shape->batch,
+               block_scores);
     return launch_status();
 }
 
@@ -721,7 +806,8 @@ lemo_status lemo_attention_kept(const lemo_shape* shape, const uint16_t* q, cons
     if (device_sms(&dev) <= 0) return LEMO_ERR_CUDA;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     char* w = static_cast<char*>(ws);
-    at::plan_kernel<<<1, 1024, 0, st>>>(cu_kept, kept_total, shape->cu_seqlens, shape->batch, w);
+    launch(at::plan_kernel, 1, 1024, 0, st, cu_kept, kept_total, shape->cu_seqlens, shape->batch,
+           w);
     if ((e = launch_status()) != LEMO_OK) return e;
     if (shape->total_L == 0 || items == 0) return LEMO_OK;
     {
@@ -756,8 +842,8 @@ lemo_status lemo_attention_kept(const lemo_shape* shape, const uint16_t* q, cons
         std::lock_guard<std::mutex> lk(g_mu);
         a.spin_limit_ns = (uint64_t)g_spin_ns;
     }
-    at::attn_kernel<<<(unsigned)(items * shape->H), at::THREADS, at::SMEM_BYTES, st>>>(tq, tk, tv,
-                                                                                      a);
+    launch(at::attn_kernel, (unsigned)(items * shape->H), at::THREADS, at::SMEM_BYTES, st, tq, tk,
+           tv, a);
     return launch_status();
 }
 
@@ -804,7 +890,7 @@ lemo_status lemo_segment_loss(const uint16_t* h, int64_t ld_h, int64_t T, int32_
             g_blas.set_workspace(hb, wsp + l.blas, kBlasWorkspace) != CUBLAS_STATUS_SUCCESS)
             return LEMO_ERR_CUDA;
     }
-    sl::count_kernel<<<1, sl::kCountThreads, 0, st>>>(targets, T, V, ignore_index, n_valid);
+    launch(sl::count_kernel, 1, sl::kCountThreads, 0, st, targets, T, V, ignore_index, n_valid);
     lemo_status e = launch_status();
     if (e != LEMO_OK) return e;
     const float one = 1.f, zero = 0.f;
@@ -826,7 +912,7 @@ lemo_status lemo_segment_loss(const uint16_t* h, int64_t ld_h, int64_t T, int32_
         a.n_valid = n_valid;
         a.V = V;
         a.ignore = ignore_index;
-        sl::row_kernel<<<S, sl::kRowThreads, 0, st>>>(a);
+        launch(sl::row_kernel, S, sl::kRowThreads, 0, st, a);
         if ((e = launch_status()) != LEMO_OK) return e;
         // dh_seg^T [d, S] = W^T [d, V] . dz^T [V, S]
         if (dh && g_blas.gemm(hb, CUBLAS_OP_N, CUBLAS_OP_N, d, S, V, &one, w, CUDA_R_16BF, (int)ld_w,
@@ -840,7 +926,7 @@ lemo_status lemo_segment_loss(const uint16_t* h, int64_t ld_h, int64_t T, int32_
                               CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS)
             return LEMO_ERR_CUDA;
     }
-    sl::loss_kernel<<<1, sl::kCountThreads, 0, st>>>(tl, T, n_valid, loss);
+    launch(sl::loss_kernel, 1, sl::kCountThreads, 0, st, tl, T, n_valid, loss);
     return launch_status();
 }
 

@@ -69,6 +69,7 @@ struct Args {
 // combine with an integer atomicMax on the float bit patterns (order does
 // not change a maximum: deterministic).  block_scores must be zeroed first.
 __global__ void __launch_bounds__(kThreads) block_scores_kernel(const Args a) {
+    pdl_entry();
     const PlanHeader* hdr = reinterpret_cast<const PlanHeader*>(a.ws + a.lay.hdr);
     if (!hdr->valid) return;
     const int32_t* blk_prefix = reinterpret_cast<const int32_t*>(a.ws + a.lay.blk_prefix);

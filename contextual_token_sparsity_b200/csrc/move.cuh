@@ -38,6 +38,7 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
 
 // y[r] = x[kept_idx[r]] for r < K; y[r] = 0 for K <= r < round_up(K, pad_to).
 __global__ void __launch_bounds__(kMoveThreads) gather_pad_kernel(MoveArgs a) {
+    pdl_entry();
     int64_t K = *a.kept_total;
     if (K < 0) K = 0;
     int64_t K_pad = (K + a.pad_to - 1) / a.pad_to * a.pad_to;
@@ -95,6 +96,7 @@ __device__ __forceinline__ uint4 add_bf16x8(uint4 x, uint4 y) {
 
 // x[kept_idx[r]] = bf16(x[kept_idx[r]] + y[r]) for r < K, in place.
 __global__ void __launch_bounds__(kMoveThreads) scatter_residual_kernel(MoveArgs a) {
+    pdl_entry();
     int64_t K = *a.kept_total;
     if (K < 0) K = 0;
     const int lane = threadIdx.x & 31;
@@ -140,6 +142,7 @@ __device__ __forceinline__ uint32_t sub_bf16x2_rn(uint32_t a, uint32_t b) {
 }
 
 __global__ void __launch_bounds__(kMoveThreads) recompute_input_kernel(MoveArgs a) {
+    pdl_entry();
     int64_t K = *a.kept_total;
     if (K < 0) K = 0;
     const int lane = threadIdx.x & 31;

@@ -295,6 +295,7 @@ __device__ __forceinline__ TileCoord tile_coord(const Args& a, const int64_t* ti
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     score_tiles_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k, const Args a) {
+    pdl_entry();
     const PlanHeader* hdr = reinterpret_cast<const PlanHeader*>(a.ws + a.lay.hdr);
     const int64_t* tile_prefix = reinterpret_cast<const int64_t*>(a.ws + a.lay.tile_prefix);
     const int64_t* m_prefix = reinterpret_cast<const int64_t*>(a.ws + a.lay.m_prefix);
@@ -524,6 +525,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 __global__ void __launch_bounds__(256) column_sum_kernel(const float* __restrict__ mblk,
                                                          const char* __restrict__ ws, WsLayout lay,
                                                          int batch, float* __restrict__ scores) {
+    pdl_entry();
     const PlanHeader* hdr = reinterpret_cast<const PlanHeader*>(ws + lay.hdr);
     if (!hdr->valid) return;
     const int32_t* blk_prefix = reinterpret_cast<const int32_t*>(ws + lay.blk_prefix);

@@ -37,6 +37,7 @@ constexpr int kCountThreads = 1024;
 __global__ void __launch_bounds__(kCountThreads)
     count_kernel(const int32_t* __restrict__ y, int64_t T, int V, int ignore,
                  int32_t* __restrict__ n_valid) {
+    pdl_entry();
     __shared__ int part[kCountThreads / 32];
     int c = 0;
     bool bad = false;
@@ -88,6 +89,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 __global__ void __launch_bounds__(kRowThreads) row_kernel(RowArgs a) {
+    pdl_entry();
     constexpr float kLog2e = 1.4426950408889634f;
     constexpr float kLn2 = 0.6931471805599453f;
     const int r = blockIdx.x;
@@ -188,6 +190,7 @@ __global__ void __launch_bounds__(kRowThreads) row_kernel(RowArgs a) {
 __global__ void __launch_bounds__(kCountThreads)
     loss_kernel(const float* __restrict__ token_loss, int64_t T, const int32_t* __restrict__ n_valid,
                 float* __restrict__ loss) {
+    pdl_entry();
     __shared__ double part[kCountThreads / 32];
     double acc = 0.0;
     for (int64_t t = threadIdx.x; t < T; t += kCountThreads) acc += (double)token_loss[t];

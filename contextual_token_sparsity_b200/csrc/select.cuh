@@ -50,6 +50,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
                                                     int total_L, int max_seqlen, int block,
                                                     char* __restrict__ ws, WsLayout lay,
                                                     int32_t* zero_word, float* zero_blocks) {
+    pdl_entry();
     PlanHeader* hdr = reinterpret_cast<PlanHeader*>(ws + lay.hdr);
     int64_t* tile_prefix = reinterpret_cast<int64_t*>(ws + lay.tile_prefix);
     int32_t* blk_prefix = reinterpret_cast<int32_t*>(ws + lay.blk_prefix);
@@ -150,6 +151,7 @@ __device__ __forceinline__ uint64_t lb_read(const uint64_t* p) {
 }
 
 __global__ void __launch_bounds__(kSelectThreads) select_kernel(SelectArgs a) {
+    pdl_entry();
     PlanHeader* hdr = reinterpret_cast<PlanHeader*>(a.ws + a.lay.hdr);
     const int32_t* blk_prefix = reinterpret_cast<const int32_t*>(a.ws + a.lay.blk_prefix);
     uint64_t* lookback = reinterpret_cast<uint64_t*>(a.ws + a.lay.lookback);
