@@ -20,19 +20,27 @@
 // rows, 128-byte swizzle) per chunk and 64-column slice brings it from its
 // original position; the kernel checks the run is contiguous.
 //
-// One CTA per (query tile of 128 kept rows, head); 6 warps:
-//   warp 0      TMA producer: Q once, then K and V of each key tile into a
-//               2-stage ring;
-//   warp 1      MMA issuer (tcgen05, cta_group::1, M = 128):
-//               S_j = Q K_j^T into one of two 128-column TMEM buffers, issued
-//               one tile ahead so it overlaps the softmax of tile j-1;
-//               O += P_j V_j into a dh-column TMEM accumulator (V is the
+// One CTA per (pair of consecutive query tiles of 128 kept rows, head);
+// 10 warps:
+//   warp 0      TMA producer: both query tiles once, then K_0, V_0, K_1,
+//               V_1, ... through a 3-slot ring of 32 KB tiles;
+//   warp 1      MMA issuer (tcgen05, cta_group::1, M = 128): for tile t in
+//               {0, 1}, S_t = Q_t K_j^T into TMEM buffer t (128 columns) and
+//               O_t += P_t V_j into a dh-column TMEM accumulator (V is the
 //               MN-major B operand: keys are the contraction dimension);
-//   warps 2-5   softmax: one thread per query row (its TMEM lane), online
-//               max / sum in log2 units; O is rescaled in TMEM only when the
-//               running max grows by more than 8 (2^8), P is written to
-//               shared memory as bf16 in the canonical 128-byte-swizzled
-//               K-major layout; at the end O / l is added into x.
+//               S_t for key tile j + 1 is issued as soon as softmax group t
+//               has read S_t of tile j, so it runs under that group's
+//               exponentials;
+//   warps 2-5   softmax group 0 (query tile 0), warps 6-9 softmax group 1
+//               (query tile 1): one thread per query row (its TMEM lane),
+//               online max / sum in log2 units; O_t is rescaled in TMEM only
+//               when the running max grows by more than 8 (2^8); P_t is
+//               written to shared memory as bf16 in the canonical
+//               128-byte-swizzled K-major layout; at the end O_t / l is added
+//               into x.  The two groups work on different query tiles, so one
+//               group's exponentials overlap the other group's MMAs.
+// A K slot is released when both S MMAs that read it have completed, a V
+// slot when both P V MMAs have.
 //
 // Every wait is bounded in time; a wait that runs out records
 // LEMO_ERR_TIMEOUT and the CTA drains what it issued, frees its tensor
@@ -60,7 +68,7 @@ using score::tc_fence_before;
 using score::tmem_ld16;
 using score::tmem_wait_ld;
 
-constexpr int BM = 128;          // kept query rows per CTA (MMA M, TMEM lanes)
+constexpr int BM = 128;          // kept query rows per query tile (MMA M, TMEM lanes)
 constexpr int BN = 128;          // kept keys per key tile (MMA N of S, K of P V)
 constexpr int CHUNK = 64;        // rows of one TMA box (one contiguous run)
 constexpr int KB = 64;           // elements per 128-byte swizzle row
@@ -69,28 +77,28 @@ constexpr int UMMA_K = 16;
 constexpr int SLICE_BYTES = BM * KB * 2;          // 128 rows x 64 elements: 16 KB
 constexpr int CHUNK_BYTES = CHUNK * KB * 2;       // one box: 8 KB
 constexpr int TILE_BYTES = (MAX_DH / KB) * SLICE_BYTES;  // 32 KB
-constexpr int SOFTMAX_WARPS = 4;
-constexpr int THREADS = 32 * (2 + SOFTMAX_WARPS);
-constexpr int TMEM_COLS = 512;   // S0 [0,128), S1 [128,256), O [256, 256+dh)
+constexpr int SOFTMAX_WARPS = 4;                  // per group
+constexpr int THREADS = 32 * (2 + 2 * SOFTMAX_WARPS);
+constexpr int KV_SLOTS = 3;
+constexpr int TMEM_COLS = 512;   // S_0 [0,128), S_1 [128,256), O_0 [256,+dh), O_1 [384,+dh)
 constexpr int O_COL = 256;
 constexpr float kRescaleLog2 = 8.f;  // rescale O only when the max grows by more
 
-// shared memory: Q | K0 | K1 | V0 | V1 | P | barriers
+// shared memory: Q_0 | Q_1 | P_0 | P_1 | KV ring | barriers
 constexpr int OFF_Q = 0;
-constexpr int OFF_K = OFF_Q + TILE_BYTES;
-constexpr int OFF_V = OFF_K + 2 * TILE_BYTES;
-constexpr int OFF_P = OFF_V + 2 * TILE_BYTES;
-constexpr int OFF_BAR = OFF_P + (BN / KB) * SLICE_BYTES;
+constexpr int OFF_P = OFF_Q + 2 * TILE_BYTES;
+constexpr int OFF_KV = OFF_P + 2 * (BN / KB) * SLICE_BYTES;
+constexpr int OFF_BAR = OFF_KV + KV_SLOTS * TILE_BYTES;
 
 struct Smem {
     uint64_t q_full;
-    uint64_t k_full[2];
-    uint64_t v_full[2];
-    uint64_t kv_empty[2];  // MMA done with stage (both K and V)
-    uint64_t s_full[2];    // S_j in TMEM buffer j % 2
-    uint64_t p_full;       // P_j in shared memory (and O rescaled)
-    uint64_t pv_done;      // O += P_j V_j completed
-    uint64_t done;         // every MMA of the CTA completed
+    uint64_t kv_full[KV_SLOTS];
+    uint64_t kv_empty[KV_SLOTS];  // the MMAs reading the slot completed
+    uint64_t s_full[2];           // S_t of the current key tile in TMEM
+    uint64_t s_free[2];           // softmax group t has read S_t
+    uint64_t p_full[2];           // P_t in shared memory (and O_t rescaled)
+    uint64_t pv_done[2];          // O_t += P_t V_j completed
+    uint64_t done;                // every MMA of the CTA completed
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -109,9 +117,9 @@ constexpr uint32_t kIdescS = idesc(BN, false);
 // Work decomposition written by plan_kernel.
 struct WsHeader {
     int valid;
-    int total_items;  // query tiles over all sequences
+    int total_items;  // query-tile pairs over all sequences
 };
-constexpr size_t kWsPrefix = 256;  // int32 [batch + 1]: query tiles before sequence s
+constexpr size_t kWsPrefix = 256;  // int32 [batch + 1]: query-tile pairs before sequence s
 
 inline size_t ws_bytes(int batch) { return kWsPrefix + align_up(4 * (size_t)(batch + 1), 256); }
 
@@ -133,8 +141,8 @@ struct Args {
 };
 
 // ---------------------------------------------------------------------------
-// Plan: query tiles per sequence from cu_kept, their prefix, and checks of
-// cu_kept against the shape (1 CTA of 1024 threads).
+// Plan: query-tile pairs per sequence from cu_kept, their prefix, and
+// checks of cu_kept against the shape (1 CTA of 1024 threads).
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024)
     plan_kernel(const int32_t* __restrict__ cu_kept, const int32_t* __restrict__ kept_total,
@@ -154,7 +162,7 @@ __global__ void __launch_bounds__(1024)
             const int k0 = cu_kept[s], k1 = cu_kept[s + 1];
             const int L = cu_seqlens[s + 1] - cu_seqlens[s];
             if (k1 < k0 || k1 - k0 > L) bad = 1;
-            else nq = (k1 - k0 + BM - 1) / BM;
+            else nq = ((k1 - k0 + BM - 1) / BM + 1) / 2;
         }
         int tot;
         const int incl = block_scan_incl<int>(nq, sum32, &tot);
@@ -197,6 +205,20 @@ __device__ __noinline__ bool wait_slow(uint64_t* bar, uint32_t parity, Smem* sm,
 __device__ __forceinline__ bool wait(uint64_t* bar, uint32_t parity, Smem* sm, uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     return wait_slow(bar, parity, sm, limit_ns);
+}
+
+// Wait for the phase of the given parity regardless of the abort flag
+// (bounded in time only): used before exit, for copies and MMAs already
+// issued, which always complete.
+__device__ __noinline__ bool wait_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > limit_ns) {
+            raise_error(LEMO_ERR_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
 }
 
 // wait() by every lane of the warp, with a warp-uniform result (the warp
@@ -266,6 +288,14 @@ __device__ __forceinline__ void fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// 2^x with the hardware approximation (flushes subnormal results to 0;
+// exact 0 for x = -inf).
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     const __nv_bfloat162 r = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<const uint32_t*>(&r);
@@ -308,12 +338,15 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int item = blockIdx.x / a.H, h = blockIdx.x % a.H;
     if (item >= hdr->total_items) return;
     const int s = last_le(prefix, a.batch + 1, item);
-    const int nq = prefix[s + 1] - prefix[s];
-    const int qt = nq - 1 - (item - prefix[s]);  // heaviest query tiles first
+    const int npairs = prefix[s + 1] - prefix[s];
+    const int pair = npairs - 1 - (item - prefix[s]);  // heaviest pairs first
     const int kbeg = a.cu_kept[s], kend = a.cu_kept[s + 1];
     const int seq0 = a.cu_seqlens[s], seq1 = a.cu_seqlens[s + 1];
-    const int q0 = kbeg + qt * BM;
-    const int ntiles = qt + 1;
+    const int nq = (kend - kbeg + BM - 1) / BM;
+    const int qa = 2 * pair;                  // query tile of group 0; group 1 has qa + 1
+    const bool two = qa + 1 < nq;
+    const int nt0 = qa + 1;                   // key tiles of query tile t: 0 .. its own index
+    const int nt = two ? qa + 2 : qa + 1;     // key tiles of the pair
     const int kblocks = a.dh / KB;
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -324,14 +357,16 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(&sm->q_full, 1);
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&sm->k_full[b], 1);
-            mbar_init(&sm->v_full[b], 1);
-            mbar_init(&sm->kv_empty[b], 1);
-            mbar_init(&sm->s_full[b], 1);
+        for (int i = 0; i < KV_SLOTS; ++i) {
+            mbar_init(&sm->kv_full[i], 1);
+            mbar_init(&sm->kv_empty[i], 1);
         }
-        mbar_init(&sm->p_full, SOFTMAX_WARPS);
-        mbar_init(&sm->pv_done, 1);
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(&sm->s_full[t], 1);
+            mbar_init(&sm->s_free[t], SOFTMAX_WARPS);
+            mbar_init(&sm->p_full[t], SOFTMAX_WARPS);
+            mbar_init(&sm->pv_done[t], 1);
+        }
         mbar_init(&sm->done, 1);
         sm->abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -355,74 +390,93 @@ __global__ void __launch_bounds__(THREADS, 1)
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_k)) : "memory");
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_v)) : "memory");
             const int col0 = h * a.dh;
-            mbar_arrive_expect_tx(&sm->q_full, chunk_bytes(q0, kend, kblocks));
+            const int q0 = kbeg + qa * BM;
+            mbar_arrive_expect_tx(&sm->q_full, chunk_bytes(q0, kend, kblocks) +
+                                                   (two ? chunk_bytes(q0 + BM, kend, kblocks) : 0u));
             load_tile(&tm_q, base + OFF_Q, q0, kend, a.kept_idx, seq0, seq1, col0, kblocks,
                       &sm->q_full);
-            int j = 0;
-            for (; j < ntiles; ++j) {
-                const int st = j & 1;
-                if (!wait(&sm->kv_empty[st], ((j >> 1) & 1) ^ 1, sm, lim)) break;
-                const int c0 = kbeg + j * BN;
-                const uint32_t bytes = chunk_bytes(c0, kend, kblocks);
-                mbar_arrive_expect_tx(&sm->k_full[st], bytes);
-                load_tile(&tm_k, base + OFF_K + st * TILE_BYTES, c0, kend, a.kept_idx, seq0, seq1,
-                          col0, kblocks, &sm->k_full[st]);
-                mbar_arrive_expect_tx(&sm->v_full[st], bytes);
-                load_tile(&tm_v, base + OFF_V + st * TILE_BYTES, c0, kend, a.kept_idx, seq0, seq1,
-                          col0, kblocks, &sm->v_full[st]);
+            if (two)
+                load_tile(&tm_q, base + OFF_Q + TILE_BYTES, q0 + BM, kend, a.kept_idx, seq0, seq1,
+                          col0, kblocks, &sm->q_full);
+            // loads n = 0, 1, 2, ...: K_{n/2} (n even) or V_{n/2} (n odd)
+            const int nloads = 2 * nt;
+            int n = 0;
+            for (; n < nloads; ++n) {
+                const int slot = n % KV_SLOTS;
+                if (!wait(&sm->kv_empty[slot], ((n / KV_SLOTS) & 1) ^ 1, sm, lim)) break;
+                const int c0 = kbeg + (n >> 1) * BN;
+                mbar_arrive_expect_tx(&sm->kv_full[slot], chunk_bytes(c0, kend, kblocks));
+                load_tile((n & 1) ? &tm_v : &tm_k, base + OFF_KV + slot * TILE_BYTES, c0, kend,
+                          a.kept_idx, seq0, seq1, col0, kblocks, &sm->kv_full[slot]);
             }
-            if (j < ntiles) {
+            if (n < nloads) {
                 // gave up: every load issued lands before the CTA may exit
-                wait(&sm->q_full, 0, sm, lim);
-                for (int i = j > 2 ? j - 2 : 0; i < j; ++i) {
-                    wait(&sm->k_full[i & 1], (i >> 1) & 1, sm, lim);
-                    wait(&sm->v_full[i & 1], (i >> 1) & 1, sm, lim);
-                }
+                wait_drain(&sm->q_full, 0, lim);
+                for (int i = n > KV_SLOTS ? n - KV_SLOTS : 0; i < n; ++i)
+                    wait_drain(&sm->kv_full[i % KV_SLOTS], (i / KV_SLOTS) & 1, lim);
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         const uint32_t idesc_pv = idesc(a.dh, true);
-        const uint32_t sq = smem_u32(base + OFF_Q);
-        bool ok = wait_warp(&sm->q_full, 0, sm, lim);
-        // S_0
-        if (ok) ok = wait_warp(&sm->k_full[0], 0, sm, lim);
-        if (ok) {
-            tc_fence_after();
+        auto slot_of = [](int n) { return n % KV_SLOTS; };
+        auto par_of = [](int n) { return (uint32_t)((n / KV_SLOTS) & 1); };
+        // S_t = Q_t K^T for the K tile in `slot`, into TMEM columns [t * BN, +BN)
+        auto issue_s = [&](int t, int slot) {
             if (lane == 0) {
-                const uint32_t sk = smem_u32(base + OFF_K);
+                const uint32_t sq = smem_u32(base + OFF_Q + t * TILE_BYTES);
+                const uint32_t sk = smem_u32(base + OFF_KV + slot * TILE_BYTES);
                 for (int k = 0; k < a.dh / UMMA_K; ++k) {
                     const uint32_t off = (k >> 2) * SLICE_BYTES + (k & 3) * 32;
-                    umma(tmem, sdesc(sq + off, 16), sdesc(sk + off, 16), kIdescS, k > 0);
+                    umma(tmem + t * BN, sdesc(sq + off, 16), sdesc(sk + off, 16), kIdescS, k > 0);
                 }
-                umma_commit(&sm->s_full[0]);
+                umma_commit(&sm->s_full[t]);
             }
             __syncwarp();
-        }
-        for (int j = 0; ok && j < ntiles; ++j) {
-            const int st = j & 1;
-            if (j + 1 < ntiles) {  // S_{j+1}, overlapping the softmax of tile j
-                const int sn = (j + 1) & 1;
-                if (!(ok = wait_warp(&sm->k_full[sn], ((j + 1) >> 1) & 1, sm, lim))) break;
-                tc_fence_after();
-                if (lane == 0) {
-                    const uint32_t sk = smem_u32(base + OFF_K + sn * TILE_BYTES);
-                    for (int k = 0; k < a.dh / UMMA_K; ++k) {
-                        const uint32_t off = (k >> 2) * SLICE_BYTES + (k & 3) * 32;
-                        umma(tmem + sn * BN, sdesc(sq + off, 16), sdesc(sk + off, 16), kIdescS,
-                             k > 0);
-                    }
-                    umma_commit(&sm->s_full[sn]);
+        };
+        // O_t += P_t V for the V tile in `slot` (accumulate unless j == 0)
+        auto issue_pv = [&](int t, int slot, int j) {
+            if (lane == 0) {
+                const uint32_t sp = smem_u32(base + OFF_P + t * (BN / KB) * SLICE_BYTES);
+                const uint32_t sv = smem_u32(base + OFF_KV + slot * TILE_BYTES);
+                for (int k = 0; k < BN / UMMA_K; ++k) {
+                    const uint32_t offa = (k >> 2) * SLICE_BYTES + (k & 3) * 32;
+                    umma(tmem + O_COL + t * 128, sdesc(sp + offa, 16),
+                         sdesc(sv + k * 2048, SLICE_BYTES), idesc_pv, (j > 0 || k > 0) ? 1u : 0u);
                 }
-                __syncwarp();
+                umma_commit(&sm->pv_done[t]);
             }
-            if (!(ok = wait_warp(&sm->p_full, j & 1, sm, lim))) break;
-            if (!(ok = wait_warp(&sm->v_full[st], (j >> 1) & 1, sm, lim))) break;
+            __syncwarp();
+        };
+        auto release = [&](int slot) {
+            if (lane == 0) umma_commit(&sm->kv_empty[slot]);
+            __syncwarp();
+        };
+        bool ok = wait_warp(&sm->q_full, 0, sm, lim);
+        if (ok) ok = wait_warp(&sm->kv_full[slot_of(0)], par_of(0), sm, lim);
+        if (ok) {
+            tc_fence_after();
+            issue_s(0, slot_of(0));
+            if (two) issue_s(1, slot_of(0));
+            release(slot_of(0));
+        }
+        for (int j = 0; ok && j < nt; ++j) {
+            const int nk = 2 * (j + 1), nv = 2 * j + 1;  // load numbers of K_{j+1} and V_j
+            const bool next0 = j + 1 < nt0, next1 = two && j + 1 < nt;
+            if (next0 || next1) {
+                if (!(ok = wait_warp(&sm->kv_full[slot_of(nk)], par_of(nk), sm, lim))) break;
+                tc_fence_after();
+            }
+            if (next0) {
+                if (!(ok = wait_warp(&sm->s_free[0], j & 1, sm, lim))) break;
+                tc_fence_after();
+                issue_s(0, slot_of(nk));
+            }
+            if (!(ok = wait_warp(&sm->kv_full[slot_of(nv)], par_of(nv), sm, lim))) break;
             // rows of V past the kept set (a short last chunk) are zeroed so
             // that 0-probability keys contribute exactly 0
-            uint8_t* vt = base + OFF_V + st * TILE_BYTES;
-            const int c0 = kbeg + j * BN;
-            const int nvalid = min(BN, kend - c0);
+            uint8_t* vt = base + OFF_KV + slot_of(nv) * TILE_BYTES;
+            const int nvalid = min(BN, kend - (kbeg + j * BN));
             if (nvalid < BN) {
                 for (int kc = 0; kc < kblocks; ++kc) {
                     uint4* p = reinterpret_cast<uint4*>(vt + kc * SLICE_BYTES + nvalid * 128);
@@ -432,98 +486,114 @@ __global__ void __launch_bounds__(THREADS, 1)
                 fence_async_smem();
             }
             __syncwarp();
-            tc_fence_after();
-            if (lane == 0) {
-                const uint32_t sp = smem_u32(base + OFF_P);
-                const uint32_t sv = smem_u32(vt);
-                for (int k = 0; k < BN / UMMA_K; ++k) {
-                    const uint32_t offa = (k >> 2) * SLICE_BYTES + (k & 3) * 32;
-                    umma(tmem + O_COL, sdesc(sp + offa, 16), sdesc(sv + k * 2048, SLICE_BYTES),
-                         idesc_pv, (j > 0 || k > 0) ? 1u : 0u);
-                }
-                umma_commit(&sm->kv_empty[st]);
-                umma_commit(&sm->pv_done);
+            if (j < nt0) {
+                if (!(ok = wait_warp(&sm->p_full[0], j & 1, sm, lim))) break;
+                tc_fence_after();
+                issue_pv(0, slot_of(nv), j);
             }
-            __syncwarp();
+            if (next1) {
+                if (!(ok = wait_warp(&sm->s_free[1], j & 1, sm, lim))) break;
+                tc_fence_after();
+                issue_s(1, slot_of(nk));
+            }
+            if (next0 || next1) release(slot_of(nk));
+            if (two) {
+                if (!(ok = wait_warp(&sm->p_full[1], j & 1, sm, lim))) break;
+                tc_fence_after();
+                issue_pv(1, slot_of(nv), j);
+            }
+            release(slot_of(nv));
         }
         // every MMA completes before the tensor memory is released
         if (lane == 0) umma_commit(&sm->done);
         __syncwarp();
-        wait_warp(&sm->done, 0, sm, lim);
+        wait_drain(&sm->done, 0, lim);
+        __syncwarp();
     } else {
         // ------------------------------------------------------------ softmax + epilogue
-        const int qd = warp & 3;                  // TMEM lane quadrant of this warp
-        const int row = qd * 32 + lane;           // query row of this thread in the tile
-        const int qc = q0 + row;                  // its compact (kept) index
+        const int t = (warp - 2) / SOFTMAX_WARPS;    // query tile of this group
+        const int qd = warp & 3;                     // TMEM lane quadrant of this warp
+        const int row = qd * 32 + lane;              // query row of this thread in the tile
+        const int qc = kbeg + (qa + t) * BM + row;   // its compact (kept) index
+        const int ntt = t == 0 ? nt0 : nt;           // key tiles of this query tile
         const uint32_t lrow = tmem + ((uint32_t)(qd * 32) << 16);
-        uint8_t* prow = base + OFF_P + row * 128; // this row of P in each 64-key slice
-        const int sw = row & 7;                   // 128-byte swizzle phase of the row
-        float m = -CUDART_INF_F, l = 0.f;         // running max (log2 units) and sum
-        bool ok = true;
-        for (int j = 0; j < ntiles; ++j) {
-            if (!(ok = wait_warp(&sm->s_full[j & 1], (j >> 1) & 1, sm, lim))) break;
+        const uint32_t s_col = t * BN, o_col = O_COL + t * 128;
+        uint8_t* prow = base + OFF_P + t * (BN / KB) * SLICE_BYTES + row * 128;
+        const int sw = row & 7;                      // 128-byte swizzle phase of the row
+        const float sl2 = a.scale_log2;
+        float m = -CUDART_INF_F, l = 0.f;            // running max (log2 units) and sum
+        bool ok = t == 0 || two;
+        for (int j = 0; ok && j < ntt; ++j) {
+            if (!(ok = wait_warp(&sm->s_full[t], j & 1, sm, lim))) break;
             tc_fence_after();
             uint32_t r[BN];
 #pragma unroll
-            for (int c = 0; c < BN; c += 16) tmem_ld16(lrow + (j & 1) * BN + c, &r[c]);
+            for (int c = 0; c < BN; c += 16) tmem_ld16(lrow + s_col + c, &r[c]);
             tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm->s_free[t]);  // S_t may be overwritten now
             // keys past the query (causal) or past the kept set are masked
-            const int ncols = min(BN, min(kend, qc + 1) - (kbeg + j * BN));
+            const int c0 = kbeg + j * BN;
+            const int ncols = min(BN, min(kend, qc + 1) - c0);
+            if (__any_sync(0xffffffffu, ncols < BN)) {
+#pragma unroll
+                for (int c = 0; c < BN; ++c)
+                    if (c >= ncols) r[c] = __float_as_uint(-CUDART_INF_F);
+            }
             float mt = -CUDART_INF_F;
 #pragma unroll
-            for (int c = 0; c < BN; ++c) {
-                const float v = c < ncols ? __uint_as_float(r[c]) * a.scale_log2 : -CUDART_INF_F;
-                r[c] = __float_as_uint(v);
-                mt = fmaxf(mt, v);
-            }
+            for (int c = 0; c < BN; ++c) mt = fmaxf(mt, __uint_as_float(r[c]));
+            mt *= sl2;
             bool rescale = false;
             float alpha = 1.f;
             if (j == 0) {
                 m = mt;
             } else if (mt > m + kRescaleLog2) {  // lazy: otherwise p <= 2^8, harmless
-                alpha = exp2f(m - mt);
+                alpha = ex2(m - mt);
                 m = mt;
                 rescale = true;
             }
-            float rs = 0.f;
-            uint32_t pk[BN / 2];
-#pragma unroll
-            for (int c = 0; c < BN; c += 2) {
-                const float p0 = exp2f(__uint_as_float(r[c]) - m);
-                const float p1 = exp2f(__uint_as_float(r[c + 1]) - m);
-                rs += p0 + p1;
-                pk[c / 2] = pack_bf16(p0, p1);
-            }
-            l = l * alpha + rs;
-            if (j > 0) {  // P buffer free and O complete up to tile j-1
-                if (!(ok = wait_warp(&sm->pv_done, (j - 1) & 1, sm, lim))) break;
+            if (j > 0) {  // P_t buffer free and O_t complete up to tile j-1
+                if (!(ok = wait_warp(&sm->pv_done[t], (j - 1) & 1, sm, lim))) break;
                 tc_fence_after();
             }
-            if (__any_sync(0xffffffffu, rescale)) {
-                for (int c = 0; c < a.dh; c += 16) {
-                    uint32_t o[16];
-                    tmem_ld16(lrow + O_COL + c, o);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                    tmem_st16(lrow + O_COL + c, o);
-                }
-                tmem_wait_st();
-            }
+            const float nm = -m;
+            float rs = 0.f;
 #pragma unroll
             for (int kc = 0; kc < BN / KB; ++kc)
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch) {
-                    const uint32_t* v = &pk[kc * 32 + ch * 4];
+                    uint32_t pk[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int c = kc * 64 + ch * 8 + 2 * i;
+                        const float p0 = ex2(fmaf(__uint_as_float(r[c]), sl2, nm));
+                        const float p1 = ex2(fmaf(__uint_as_float(r[c + 1]), sl2, nm));
+                        rs += p0 + p1;
+                        pk[i] = pack_bf16(p0, p1);
+                    }
                     *reinterpret_cast<uint4*>(prow + kc * SLICE_BYTES + ((ch ^ sw) << 4)) =
-                        make_uint4(v[0], v[1], v[2], v[3]);
+                        make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 }
+            l = l * alpha + rs;
+            if (__any_sync(0xffffffffu, rescale)) {
+                for (int c = 0; c < a.dh; c += 16) {
+                    uint32_t o[16];
+                    tmem_ld16(lrow + o_col + c, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                    tmem_st16(lrow + o_col + c, o);
+                }
+                tmem_wait_st();
+            }
             fence_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm->p_full);
+            if (lane == 0) mbar_arrive(&sm->p_full[t]);
         }
-        if (ok) ok = wait_warp(&sm->pv_done, (ntiles - 1) & 1, sm, lim);
+        if (ok) ok = wait_warp(&sm->pv_done[t], (ntt - 1) & 1, sm, lim);
         if (ok) {
             tc_fence_after();
             const float inv = 1.f / l;
@@ -532,12 +602,12 @@ __global__ void __launch_bounds__(THREADS, 1)
             uint16_t* dst = nullptr;
             if (live) {
                 if (add) {
-                    const int64_t t = a.kept_idx[qc];
-                    if (t < 0 || t >= a.x_rows) {
+                    const int64_t tok = a.kept_idx[qc];
+                    if (tok < 0 || tok >= a.x_rows) {
                         raise_error(LEMO_ERR_INVALID_ARG);
                         live = false;
                     } else {
-                        dst = a.x + t * a.ld_x + (int64_t)h * a.dh;
+                        dst = a.x + tok * a.ld_x + (int64_t)h * a.dh;
                     }
                 } else {
                     dst = a.o + (int64_t)qc * a.ld_o + (int64_t)h * a.dh;
@@ -545,7 +615,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
             for (int c = 0; c < a.dh; c += 16) {
                 uint32_t o[16];
-                tmem_ld16(lrow + O_COL + c, o);
+                tmem_ld16(lrow + o_col + c, o);
                 tmem_wait_ld();
                 if (!live) continue;
                 uint4* d4 = reinterpret_cast<uint4*>(dst + c);

@@ -800,7 +800,9 @@ lemo_status lemo_attention_kept(const lemo_shape* shape, const uint16_t* q, cons
         !aligned(kept_total, 4) || !aligned(ws, 256))
         return LEMO_ERR_INVALID_ARG;
     if (ws_bytes < at::ws_bytes(shape->batch)) return LEMO_ERR_INVALID_ARG;
-    const int64_t items = ((int64_t)shape->total_L + (int64_t)shape->batch * (at::BM - 1)) / at::BM;
+    // query-tile pairs: sequence s has ceil(ceil(K_s / BM) / 2) of them
+    const int64_t tiles = ((int64_t)shape->total_L + (int64_t)shape->batch * (at::BM - 1)) / at::BM;
+    const int64_t items = (tiles + shape->batch) / 2;
     if (items * shape->H >= (int64_t)1 << 31) return LEMO_ERR_UNSUPPORTED;
     int dev = 0;
     if (device_sms(&dev) <= 0) return LEMO_ERR_CUDA;
