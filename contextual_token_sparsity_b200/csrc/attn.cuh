@@ -21,26 +21,35 @@
 // original position; the kernel checks the run is contiguous.
 //
 // One CTA per (pair of consecutive query tiles of 128 kept rows, head);
-// 10 warps:
+// 12 warps in 3 warpgroups:
 //   warp 0      TMA producer: both query tiles once, then K_0, V_0, K_1,
-//               V_1, ... through a 3-slot ring of 32 KB tiles;
-//   warp 1      MMA issuer (tcgen05, cta_group::1, M = 128): for tile t in
-//               {0, 1}, S_t = Q_t K_j^T into TMEM buffer t (128 columns) and
-//               O_t += P_t V_j into a dh-column TMEM accumulator (V is the
-//               MN-major B operand: keys are the contraction dimension);
-//               S_t for key tile j + 1 is issued as soon as softmax group t
-//               has read S_t of tile j, so it runs under that group's
-//               exponentials;
-//   warps 2-5   softmax group 0 (query tile 0), warps 6-9 softmax group 1
-//               (query tile 1): one thread per query row (its TMEM lane),
-//               online max / sum in log2 units; O_t is rescaled in TMEM only
-//               when the running max grows by more than 8 (2^8); P_t is
-//               written to shared memory as bf16 in the canonical
-//               128-byte-swizzled K-major layout; at the end O_t / l is added
-//               into x.  The two groups work on different query tiles, so one
-//               group's exponentials overlap the other group's MMAs.
-// A K slot is released when both S MMAs that read it have completed, a V
-// slot when both P V MMAs have.
+//               V_1, ... through a 5-slot ring of 32 KB tiles;
+//   warp 1      MMA issuer (tcgen05, cta_group::1, M = 128).  For query
+//               tile t in {0, 1} and key tile j it issues
+//                 S_t = Q_t K_j^T          into TMEM columns [128 t, +128)
+//                 O_t += P_t V_j           into TMEM columns [256 + 128 t, +dh)
+//               where P_t is read from TMEM (A operand) and V is the MN-major
+//               shared-memory B operand.  It polls both query tiles and
+//               issues whichever MMA is ready, so the tiles never wait on
+//               each other;
+//   warps 2-3   idle (they complete the first warpgroup);
+//   warps 4-7   softmax group 0 (query tile 0), warps 8-11 softmax group 1
+//               (query tile 1): one thread per query row (its TMEM lane).
+//               A thread reads its 128 scores of S_t into registers, keeps an
+//               online max / sum in log2 units, and writes the bf16
+//               probabilities back over the first 64 columns of S_t, where
+//               the P V MMA reads them.  O_t is rescaled in TMEM only when the
+//               running max grows by more than 8 (2^8).  At the end O_t / l
+//               is added into x.  The two groups work on different query
+//               tiles, so one group's exponentials overlap the other group's
+//               MMAs.
+// S_t of key tile j + 1 overwrites P_t of tile j, so it is issued only after
+// O_t += P_t V_j has completed.  A K slot is released when the S MMAs that
+// read it have completed, a V slot when the P V MMAs have.
+//
+// Registers: 384 threads and one CTA per SM leave 168 per thread (three warps
+// share each SM sub-partition's 16K registers); a softmax thread holds its
+// full 128-column row of S in registers.
 //
 // Every wait is bounded in time; a wait that runs out records
 // LEMO_ERR_TIMEOUT and the CTA drains what it issued, frees its tensor
@@ -77,17 +86,16 @@ constexpr int UMMA_K = 16;
 constexpr int SLICE_BYTES = BM * KB * 2;          // 128 rows x 64 elements: 16 KB
 constexpr int CHUNK_BYTES = CHUNK * KB * 2;       // one box: 8 KB
 constexpr int TILE_BYTES = (MAX_DH / KB) * SLICE_BYTES;  // 32 KB
-constexpr int SOFTMAX_WARPS = 4;                  // per group
-constexpr int THREADS = 32 * (2 + 2 * SOFTMAX_WARPS);
-constexpr int KV_SLOTS = 3;
+constexpr int SOFTMAX_WARPS = 4;                  // per group (one warpgroup)
+constexpr int THREADS = 32 * 12;
+constexpr int KV_SLOTS = 5;
 constexpr int TMEM_COLS = 512;   // S_0 [0,128), S_1 [128,256), O_0 [256,+dh), O_1 [384,+dh)
 constexpr int O_COL = 256;
 constexpr float kRescaleLog2 = 8.f;  // rescale O only when the max grows by more
 
-// shared memory: Q_0 | Q_1 | P_0 | P_1 | KV ring | barriers
+// shared memory: Q_0 | Q_1 | KV ring | barriers
 constexpr int OFF_Q = 0;
-constexpr int OFF_P = OFF_Q + 2 * TILE_BYTES;
-constexpr int OFF_KV = OFF_P + 2 * (BN / KB) * SLICE_BYTES;
+constexpr int OFF_KV = OFF_Q + 2 * TILE_BYTES;
 constexpr int OFF_BAR = OFF_KV + KV_SLOTS * TILE_BYTES;
 
 struct Smem {
@@ -95,8 +103,7 @@ struct Smem {
     uint64_t kv_full[KV_SLOTS];
     uint64_t kv_empty[KV_SLOTS];  // the MMAs reading the slot completed
     uint64_t s_full[2];           // S_t of the current key tile in TMEM
-    uint64_t s_free[2];           // softmax group t has read S_t
-    uint64_t p_full[2];           // P_t in shared memory (and O_t rescaled)
+    uint64_t p_full[2];           // P_t in TMEM (and O_t rescaled)
     uint64_t pv_done[2];          // O_t += P_t V_j completed
     uint64_t done;                // every MMA of the CTA completed
     uint32_t tmem_base;
@@ -262,6 +269,17 @@ __device__ __forceinline__ void umma(uint32_t tmem_d, uint64_t da, uint64_t db, 
         "l"(da), "l"(db), "r"(accumulate), "r"(idesc_v));
 }
 
+// Same with the A operand in tensor memory (M rows in lanes, two 16-bit K
+// elements per 32-bit column).
+__device__ __forceinline__ void umma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t db,
+                                        uint32_t idesc_v, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %3, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %4, p;\n\t}\n" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(db), "r"(accumulate), "r"(idesc_v));
+}
+
 // Arrive once on `bar` when every MMA issued so far by this thread is done.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
     asm volatile(
@@ -363,7 +381,6 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(&sm->s_full[t], 1);
-            mbar_init(&sm->s_free[t], SOFTMAX_WARPS);
             mbar_init(&sm->p_full[t], SOFTMAX_WARPS);
             mbar_init(&sm->pv_done[t], 1);
         }
@@ -418,108 +435,116 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
+        // A scheduler over both query tiles: op 2 j is S_t of key tile j,
+        // op 2 j + 1 is O_t += P_t V_j.  S_t(j) needs K_j loaded and (j > 0)
+        // P V of tile j - 1 completed (it overwrites P_t); P V(j) needs V_j
+        // loaded and P_t(j) written by the softmax group.  Lane 0 polls and
+        // issues; a K or V slot is released once every MMA reading it is
+        // issued.
         const uint32_t idesc_pv = idesc(a.dh, true);
-        auto slot_of = [](int n) { return n % KV_SLOTS; };
-        auto par_of = [](int n) { return (uint32_t)((n / KV_SLOTS) & 1); };
-        // S_t = Q_t K^T for the K tile in `slot`, into TMEM columns [t * BN, +BN)
-        auto issue_s = [&](int t, int slot) {
-            if (lane == 0) {
-                const uint32_t sq = smem_u32(base + OFF_Q + t * TILE_BYTES);
-                const uint32_t sk = smem_u32(base + OFF_KV + slot * TILE_BYTES);
-                for (int k = 0; k < a.dh / UMMA_K; ++k) {
-                    const uint32_t off = (k >> 2) * SLICE_BYTES + (k & 3) * 32;
-                    umma(tmem + t * BN, sdesc(sq + off, 16), sdesc(sk + off, 16), kIdescS, k > 0);
-                }
-                umma_commit(&sm->s_full[t]);
-            }
-            __syncwarp();
-        };
-        // O_t += P_t V for the V tile in `slot` (accumulate unless j == 0)
-        auto issue_pv = [&](int t, int slot, int j) {
-            if (lane == 0) {
-                const uint32_t sp = smem_u32(base + OFF_P + t * (BN / KB) * SLICE_BYTES);
-                const uint32_t sv = smem_u32(base + OFF_KV + slot * TILE_BYTES);
-                for (int k = 0; k < BN / UMMA_K; ++k) {
-                    const uint32_t offa = (k >> 2) * SLICE_BYTES + (k & 3) * 32;
-                    umma(tmem + O_COL + t * 128, sdesc(sp + offa, 16),
-                         sdesc(sv + k * 2048, SLICE_BYTES), idesc_pv, (j > 0 || k > 0) ? 1u : 0u);
-                }
-                umma_commit(&sm->pv_done[t]);
-            }
-            __syncwarp();
-        };
-        auto release = [&](int slot) {
-            if (lane == 0) umma_commit(&sm->kv_empty[slot]);
-            __syncwarp();
-        };
+        const uint32_t sq0 = smem_u32(base + OFF_Q);
+        int op[2] = {0, 0};
+        const int nops[2] = {2 * nt0, two ? 2 * nt : 0};
+        uint32_t half_used = 0;  // bit per slot: one of two MMAs on its tile issued
         bool ok = wait_warp(&sm->q_full, 0, sm, lim);
-        if (ok) ok = wait_warp(&sm->kv_full[slot_of(0)], par_of(0), sm, lim);
-        if (ok) {
-            tc_fence_after();
-            issue_s(0, slot_of(0));
-            if (two) issue_s(1, slot_of(0));
-            release(slot_of(0));
-        }
-        for (int j = 0; ok && j < nt; ++j) {
-            const int nk = 2 * (j + 1), nv = 2 * j + 1;  // load numbers of K_{j+1} and V_j
-            const bool next0 = j + 1 < nt0, next1 = two && j + 1 < nt;
-            if (next0 || next1) {
-                if (!(ok = wait_warp(&sm->kv_full[slot_of(nk)], par_of(nk), sm, lim))) break;
-                tc_fence_after();
-            }
-            if (next0) {
-                if (!(ok = wait_warp(&sm->s_free[0], j & 1, sm, lim))) break;
-                tc_fence_after();
-                issue_s(0, slot_of(nk));
-            }
-            if (!(ok = wait_warp(&sm->kv_full[slot_of(nv)], par_of(nv), sm, lim))) break;
-            // rows of V past the kept set (a short last chunk) are zeroed so
-            // that 0-probability keys contribute exactly 0
-            uint8_t* vt = base + OFF_KV + slot_of(nv) * TILE_BYTES;
-            const int nvalid = min(BN, kend - (kbeg + j * BN));
-            if (nvalid < BN) {
-                for (int kc = 0; kc < kblocks; ++kc) {
-                    uint4* p = reinterpret_cast<uint4*>(vt + kc * SLICE_BYTES + nvalid * 128);
-                    const int n16 = (BN - nvalid) * 8;
-                    for (int i = lane; i < n16; i += 32) p[i] = make_uint4(0u, 0u, 0u, 0u);
+        tc_fence_after();
+        uint64_t t_wait = globaltimer_ns();
+        uint32_t spins = 0;
+        while (ok && (op[0] < nops[0] || op[1] < nops[1])) {
+            bool progressed = false;
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                if (op[t] >= nops[t]) continue;
+                const int j = op[t] >> 1;
+                const bool is_pv = op[t] & 1;
+                const int n = is_pv ? 2 * j + 1 : 2 * j;   // load number of the operand
+                const int slot = n % KV_SLOTS;
+                // readiness: operand loaded, and the group's own dependency
+                bool ready = mbar_try_wait(&sm->kv_full[slot], (n / KV_SLOTS) & 1);
+                if (ready) {
+                    if (is_pv) ready = mbar_try_wait(&sm->p_full[t], j & 1);
+                    else if (j > 0) ready = mbar_try_wait(&sm->pv_done[t], (j - 1) & 1);
                 }
-                fence_async_smem();
-            }
-            __syncwarp();
-            if (j < nt0) {
-                if (!(ok = wait_warp(&sm->p_full[0], j & 1, sm, lim))) break;
+                ready = __shfl_sync(0xffffffffu, ready, 0);
+                if (!ready) continue;
                 tc_fence_after();
-                issue_pv(0, slot_of(nv), j);
+                // MMAs that read this tile: one per query tile whose range has it
+                const int need = (j < nt0 ? 1 : 0) + (two ? 1 : 0);
+                const bool first = !((half_used >> slot) & 1u);
+                if (is_pv) {
+                    // rows of V past the kept set (a short last chunk) are
+                    // zeroed so that 0-probability keys contribute exactly 0
+                    // (by the first MMA on this V tile)
+                    const int nvalid = min(BN, kend - (kbeg + j * BN));
+                    if (nvalid < BN && first) {
+                        uint8_t* vt = base + OFF_KV + slot * TILE_BYTES;
+                        for (int kc = 0; kc < kblocks; ++kc) {
+                            uint4* p = reinterpret_cast<uint4*>(vt + kc * SLICE_BYTES + nvalid * 128);
+                            const int n16 = (BN - nvalid) * 8;
+                            for (int i = lane; i < n16; i += 32) p[i] = make_uint4(0u, 0u, 0u, 0u);
+                        }
+                        fence_async_smem();
+                        __syncwarp();
+                        tc_fence_after();
+                    }
+                    if (lane == 0) {
+                        const uint32_t sv = smem_u32(base + OFF_KV + slot * TILE_BYTES);
+                        for (int k = 0; k < BN / UMMA_K; ++k)
+                            umma_ts(tmem + O_COL + t * 128, tmem + t * BN + k * (UMMA_K / 2),
+                                    sdesc(sv + k * 2048, SLICE_BYTES), idesc_pv,
+                                    (j > 0 || k > 0) ? 1u : 0u);
+                        umma_commit(&sm->pv_done[t]);
+                    }
+                } else if (lane == 0) {
+                    const uint32_t sq = sq0 + t * TILE_BYTES;
+                    const uint32_t sk = smem_u32(base + OFF_KV + slot * TILE_BYTES);
+                    for (int k = 0; k < a.dh / UMMA_K; ++k) {
+                        const uint32_t off = (k >> 2) * SLICE_BYTES + (k & 3) * 32;
+                        umma(tmem + t * BN, sdesc(sq + off, 16), sdesc(sk + off, 16), kIdescS,
+                             k > 0);
+                    }
+                    umma_commit(&sm->s_full[t]);
+                }
+                if (need == 1 || !first) {  // last MMA on the tile: free its slot
+                    if (lane == 0) umma_commit(&sm->kv_empty[slot]);
+                    half_used &= ~(1u << slot);
+                } else {
+                    half_used |= 1u << slot;
+                }
+                __syncwarp();
+                ++op[t];
+                progressed = true;
             }
-            if (next1) {
-                if (!(ok = wait_warp(&sm->s_free[1], j & 1, sm, lim))) break;
-                tc_fence_after();
-                issue_s(1, slot_of(nk));
+            if (progressed) {
+                t_wait = globaltimer_ns();
+                spins = 0;
+            } else if ((++spins & 63) == 0) {
+                if (*reinterpret_cast<volatile int*>(&sm->abort_flag)) {
+                    ok = false;
+                } else if (globaltimer_ns() - t_wait > lim) {
+                    if (lane == 0) {
+                        raise_error(LEMO_ERR_TIMEOUT);
+                        abort_cta(sm);
+                    }
+                    ok = false;
+                }
+                ok = __all_sync(0xffffffffu, ok);
             }
-            if (next0 || next1) release(slot_of(nk));
-            if (two) {
-                if (!(ok = wait_warp(&sm->p_full[1], j & 1, sm, lim))) break;
-                tc_fence_after();
-                issue_pv(1, slot_of(nv), j);
-            }
-            release(slot_of(nv));
         }
         // every MMA completes before the tensor memory is released
         if (lane == 0) umma_commit(&sm->done);
         __syncwarp();
         wait_drain(&sm->done, 0, lim);
         __syncwarp();
-    } else {
+    } else if (warp >= 4) {
         // ------------------------------------------------------------ softmax + epilogue
-        const int t = (warp - 2) / SOFTMAX_WARPS;    // query tile of this group
+        const int t = (warp - 4) / SOFTMAX_WARPS;    // query tile of this group
         const int qd = warp & 3;                     // TMEM lane quadrant of this warp
         const int row = qd * 32 + lane;              // query row of this thread in the tile
         const int qc = kbeg + (qa + t) * BM + row;   // its compact (kept) index
         const int ntt = t == 0 ? nt0 : nt;           // key tiles of this query tile
         const uint32_t lrow = tmem + ((uint32_t)(qd * 32) << 16);
         const uint32_t s_col = t * BN, o_col = O_COL + t * 128;
-        uint8_t* prow = base + OFF_P + t * (BN / KB) * SLICE_BYTES + row * 128;
-        const int sw = row & 7;                      // 128-byte swizzle phase of the row
         const float sl2 = a.scale_log2;
         float m = -CUDART_INF_F, l = 0.f;            // running max (log2 units) and sum
         bool ok = t == 0 || two;
@@ -530,9 +555,6 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
             for (int c = 0; c < BN; c += 16) tmem_ld16(lrow + s_col + c, &r[c]);
             tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm->s_free[t]);  // S_t may be overwritten now
             // keys past the query (causal) or past the kept set are masked
             const int c0 = kbeg + j * BN;
             const int ncols = min(BN, min(kend, qc + 1) - c0);
@@ -541,10 +563,17 @@ __global__ void __launch_bounds__(THREADS, 1)
                 for (int c = 0; c < BN; ++c)
                     if (c >= ncols) r[c] = __float_as_uint(-CUDART_INF_F);
             }
-            float mt = -CUDART_INF_F;
+            // row maximum: 8 independent partial maxima, then a tree
+            float mx[8];
 #pragma unroll
-            for (int c = 0; c < BN; ++c) mt = fmaxf(mt, __uint_as_float(r[c]));
-            mt *= sl2;
+            for (int i = 0; i < 8; ++i) mx[i] = __uint_as_float(r[i]);
+#pragma unroll
+            for (int c = 8; c < BN; ++c) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(r[c]));
+#pragma unroll
+            for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+                for (int i = 0; i < w; ++i) mx[i] = fmaxf(mx[i], mx[i + w]);
+            const float mt = mx[0] * sl2;
             bool rescale = false;
             float alpha = 1.f;
             if (j == 0) {
@@ -554,29 +583,24 @@ __global__ void __launch_bounds__(THREADS, 1)
                 m = mt;
                 rescale = true;
             }
-            if (j > 0) {  // P_t buffer free and O_t complete up to tile j-1
-                if (!(ok = wait_warp(&sm->pv_done[t], (j - 1) & 1, sm, lim))) break;
-                tc_fence_after();
-            }
+            // probabilities as bf16 pairs, 4 partial sums
             const float nm = -m;
-            float rs = 0.f;
+            uint32_t pk[BN / 2];
+            float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int kc = 0; kc < BN / KB; ++kc)
+            for (int c = 0; c < BN; c += 2) {
+                const float p0 = ex2(fmaf(__uint_as_float(r[c]), sl2, nm));
+                const float p1 = ex2(fmaf(__uint_as_float(r[c + 1]), sl2, nm));
+                ps[(c >> 1) & 3] += p0 + p1;
+                pk[c >> 1] = pack_bf16(p0, p1);
+            }
+            l = l * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
+            // P_t over the first 64 columns of S_t (S_t is in registers; the
+            // MMA side writes S_t again only after P V of this tile)
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    uint32_t pk[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int c = kc * 64 + ch * 8 + 2 * i;
-                        const float p0 = ex2(fmaf(__uint_as_float(r[c]), sl2, nm));
-                        const float p1 = ex2(fmaf(__uint_as_float(r[c + 1]), sl2, nm));
-                        rs += p0 + p1;
-                        pk[i] = pack_bf16(p0, p1);
-                    }
-                    *reinterpret_cast<uint4*>(prow + kc * SLICE_BYTES + ((ch ^ sw) << 4)) =
-                        make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                }
-            l = l * alpha + rs;
+            for (int c = 0; c < BN / 2; c += 16) tmem_st16(lrow + s_col + c, &pk[c]);
+            // O_t is complete up to tile j - 1 here: S_t(j) was issued after
+            // P V(j - 1) had completed
             if (__any_sync(0xffffffffu, rescale)) {
                 for (int c = 0; c < a.dh; c += 16) {
                     uint32_t o[16];
@@ -586,9 +610,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                     for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
                     tmem_st16(lrow + o_col + c, o);
                 }
-                tmem_wait_st();
             }
-            fence_async_smem();
+            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm->p_full[t]);
