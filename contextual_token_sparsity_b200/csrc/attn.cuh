@@ -23,33 +23,29 @@
 // One CTA per (pair of consecutive query tiles of 128 kept rows, head);
 // 12 warps in 3 warpgroups:
 //   warp 0      TMA producer: both query tiles once, then K_0, V_0, K_1,
-//               V_1, ... through a 5-slot ring of 32 KB tiles;
-//   warp 1      MMA issuer (tcgen05, cta_group::1, M = 128).  For query
-//               tile t in {0, 1} and key tile j it issues
-//                 S_t = Q_t K_j^T          into TMEM columns [128 t, +128)
-//                 O_t += P_t V_j           into TMEM columns [256 + 128 t, +dh)
-//               where P_t is read from TMEM (A operand) and V is the MN-major
-//               shared-memory B operand.  It polls both query tiles and
-//               issues whichever MMA is ready, so the tiles never wait on
-//               each other;
-//   warps 2-3   idle (they complete the first warpgroup);
+//               V_1, ... (key tiles of 64 kept rows, 16 KB each) through a
+//               10-slot ring;
+//   warps 1, 2  MMA issuers (tcgen05, cta_group::1, M = 128), warp 1 for
+//               query tile 0 and warp 2 for query tile 1.  For key tile j:
+//                 S_t(j) = Q_t K_j^T      into TMEM columns [128 t + 64 (j%2), +64)
+//                 O_t += P_t(j) V_j       into TMEM columns [256 + 128 t, +dh)
+//               where P_t(j) is read from TMEM (A operand) and V is the
+//               MN-major shared-memory B operand.  S is double-buffered, so
+//               S_t(j + 1) is computed while the softmax works on tile j;
+//   warp 3      idle (it completes the first warpgroup);
 //   warps 4-7   softmax group 0 (query tile 0), warps 8-11 softmax group 1
 //               (query tile 1): one thread per query row (its TMEM lane).
-//               A thread reads its 128 scores of S_t into registers, keeps an
-//               online max / sum in log2 units, and writes the bf16
-//               probabilities back over the first 64 columns of S_t, where
-//               the P V MMA reads them.  O_t is rescaled in TMEM only when the
-//               running max grows by more than 8 (2^8).  At the end O_t / l
-//               is added into x.  The two groups work on different query
-//               tiles, so one group's exponentials overlap the other group's
-//               MMAs.
-// S_t of key tile j + 1 overwrites P_t of tile j, so it is issued only after
-// O_t += P_t V_j has completed.  A K slot is released when the S MMAs that
-// read it have completed, a V slot when the P V MMAs have.
-//
-// Registers: 384 threads and one CTA per SM leave 168 per thread (three warps
-// share each SM sub-partition's 16K registers); a softmax thread holds its
-// full 128-column row of S in registers.
+//               A thread reads its 64 scores of S_t(j) into registers, keeps
+//               an online max / sum in log2 units, and writes the bf16
+//               probabilities back over the first 32 columns of the same S
+//               buffer, where the P V MMA reads them.  O_t is rescaled in TMEM
+//               only when the running max grows by more than 8 (2^8).  At the
+//               end O_t / l is added into x.
+// S_t(j + 2) overwrites P_t(j), so it is issued only after O_t += P_t(j) V_j
+// has completed.  A K or V slot is released when the MMAs of both query
+// tiles that read it have completed.  The rows of the last, short key tile
+// past the kept set are zeroed by the producer before the tile is handed
+// to the MMAs, so that 0-probability keys contribute exactly 0.
 //
 // Every wait is bounded in time; a wait that runs out records
 // LEMO_ERR_TIMEOUT and the CTA drains what it issued, frees its tensor
@@ -78,34 +74,36 @@ using score::tmem_ld16;
 using score::tmem_wait_ld;
 
 constexpr int BM = 128;          // kept query rows per query tile (MMA M, TMEM lanes)
-constexpr int BN = 128;          // kept keys per key tile (MMA N of S, K of P V)
-constexpr int CHUNK = 64;        // rows of one TMA box (one contiguous run)
+constexpr int BN = 64;           // kept keys per key tile (MMA N of S, K of P V)
 constexpr int KB = 64;           // elements per 128-byte swizzle row
 constexpr int MAX_DH = 128;
 constexpr int UMMA_K = 16;
-constexpr int SLICE_BYTES = BM * KB * 2;          // 128 rows x 64 elements: 16 KB
-constexpr int CHUNK_BYTES = CHUNK * KB * 2;       // one box: 8 KB
-constexpr int TILE_BYTES = (MAX_DH / KB) * SLICE_BYTES;  // 32 KB
-constexpr int SOFTMAX_WARPS = 4;                  // per group (one warpgroup)
+constexpr int Q_SLICE = BM * KB * 2;               // 128 rows x 64 elements: 16 KB
+constexpr int Q_CHUNK = 64 * KB * 2;               // one 64-row box: 8 KB
+constexpr int Q_TILE = (MAX_DH / KB) * Q_SLICE;    // 32 KB
+constexpr int KV_SLICE = BN * KB * 2;              // 64 rows x 64 elements: 8 KB
+constexpr int KV_TILE = (MAX_DH / KB) * KV_SLICE;  // 16 KB
+constexpr int SOFTMAX_WARPS = 4;                   // per group (one warpgroup)
 constexpr int THREADS = 32 * 12;
-constexpr int KV_SLOTS = 5;
+constexpr int KV_SLOTS = 10;
 constexpr int TMEM_COLS = 512;   // S_0 [0,128), S_1 [128,256), O_0 [256,+dh), O_1 [384,+dh)
 constexpr int O_COL = 256;
 constexpr float kRescaleLog2 = 8.f;  // rescale O only when the max grows by more
 
 // shared memory: Q_0 | Q_1 | KV ring | barriers
 constexpr int OFF_Q = 0;
-constexpr int OFF_KV = OFF_Q + 2 * TILE_BYTES;
-constexpr int OFF_BAR = OFF_KV + KV_SLOTS * TILE_BYTES;
+constexpr int OFF_KV = OFF_Q + 2 * Q_TILE;
+constexpr int OFF_BAR = OFF_KV + KV_SLOTS * KV_TILE;
 
 struct Smem {
     uint64_t q_full;
     uint64_t kv_full[KV_SLOTS];
-    uint64_t kv_empty[KV_SLOTS];  // the MMAs reading the slot completed
-    uint64_t s_full[2];           // S_t of the current key tile in TMEM
-    uint64_t p_full[2];           // P_t in TMEM (and O_t rescaled)
-    uint64_t pv_done[2];          // O_t += P_t V_j completed
-    uint64_t done;                // every MMA of the CTA completed
+    uint64_t kv_empty[KV_SLOTS];  // two arrivals: both query tiles' MMAs on the slot done
+    uint64_t s_full[2][2];        // [tile][buffer] S_t(j) in TMEM
+    uint64_t p_full[2][2];        // [tile][buffer] P_t(j) in TMEM (and O_t rescaled)
+    uint64_t pv_done[2][2];       // [tile][buffer] O_t += P_t(j) V_j completed
+    uint64_t vtail;               // the short last V tile has landed (producer only)
+    uint64_t done[2];             // every MMA of issuer t completed
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -113,7 +111,7 @@ constexpr int SMEM_BYTES = OFF_BAR + (int)sizeof(Smem) + 1024 /*align slack*/;
 static_assert(SMEM_BYTES <= 232448, "exceeds the 227 KB of shared memory per CTA");
 
 // Instruction descriptors of tcgen05.mma kind::f16 (D fp32, A and B bf16,
-// M = 128): S = Q K^T with both operands K-major, N = 128; O += P V with V
+// M = 128): S = Q K^T with both operands K-major, N = 64; O += P V with V
 // MN-major (bit 16), N = dh.
 __host__ __device__ constexpr uint32_t idesc(int n, bool b_mn_major) {
     return (1u << 4) | (1u << 7) | (1u << 10) | (b_mn_major ? (1u << 16) : 0u) |
@@ -228,6 +226,20 @@ __device__ __noinline__ bool wait_drain(uint64_t* bar, uint32_t parity, uint64_t
     return true;
 }
 
+// Non-blocking test of a phase (mbarrier.try_wait may suspend the thread
+// for a while; the MMA scheduler must move on to the other query tile).
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // wait() by every lane of the warp, with a warp-uniform result (the warp
 // then runs its collective tensor-memory instructions together or not at all).
 __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, Smem* sm,
@@ -319,31 +331,26 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<const uint32_t*>(&r);
 }
 
-// Issue the TMA boxes of one tile of 128 kept rows starting at compact row
-// c0 (rows at or beyond `end` are not loaded); returns the bytes issued.
-// Each 64-row chunk must be one contiguous run of original rows inside the
-// sequence [seq0, seq1); a chunk that is not is reported (the load stays in
-// bounds: TMA fills rows outside the tensor with zeros).
-__device__ __forceinline__ uint32_t chunk_bytes(int c0, int end, int kblocks) {
-    uint32_t n = 0;
-    for (int c = 0; c < BM / CHUNK; ++c)
-        if (c0 + c * CHUNK < end) n += kblocks * CHUNK_BYTES;
-    return n;
+// TMA boxes (64 columns x 64 rows) of one run of up to 64 kept rows that
+// starts at compact row c0 (rows at or beyond `end` are not loaded).  The
+// run must be contiguous in the original rows and inside the sequence
+// [seq0, seq1); one that is not is reported (the load stays in bounds: TMA
+// fills rows outside the tensor with zeros).  Slice kc of the run goes to
+// dst + kc * slice.  Returns the bytes issued.
+__device__ __forceinline__ uint32_t run_bytes(int c0, int end, int kblocks) {
+    return c0 < end ? (uint32_t)(kblocks * KV_SLICE) : 0u;
 }
 
-__device__ __forceinline__ void load_tile(const CUtensorMap* tm, uint8_t* dst, int c0, int end,
-                                          const int32_t* kept_idx, int seq0, int seq1, int col0,
-                                          int kblocks, uint64_t* bar) {
-    for (int c = 0; c < BM / CHUNK; ++c) {
-        const int start = c0 + c * CHUNK;
-        if (start >= end) break;
-        const int valid = min(CHUNK, end - start);
-        const int row = kept_idx[start];
-        if (kept_idx[start + valid - 1] != row + valid - 1 || row < seq0 || row + valid > seq1)
-            raise_error(LEMO_ERR_INVALID_ARG);
-        for (int kc = 0; kc < kblocks; ++kc)
-            tma_load_2d(dst + kc * SLICE_BYTES + c * CHUNK_BYTES, tm, col0 + kc * KB, row, bar);
-    }
+__device__ __forceinline__ void load_run(const CUtensorMap* tm, uint8_t* dst, int slice, int c0,
+                                         int end, const int32_t* kept_idx, int seq0, int seq1,
+                                         int col0, int kblocks, uint64_t* bar) {
+    if (c0 >= end) return;
+    const int valid = min(64, end - c0);
+    const int row = kept_idx[c0];
+    if (kept_idx[c0 + valid - 1] != row + valid - 1 || row < seq0 || row + valid > seq1)
+        raise_error(LEMO_ERR_INVALID_ARG);
+    for (int kc = 0; kc < kblocks; ++kc)
+        tma_load_2d(dst + kc * slice, tm, col0 + kc * KB, row, bar);
 }
 
 __global__ void __launch_bounds__(THREADS, 1)
@@ -360,11 +367,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int pair = npairs - 1 - (item - prefix[s]);  // heaviest pairs first
     const int kbeg = a.cu_kept[s], kend = a.cu_kept[s + 1];
     const int seq0 = a.cu_seqlens[s], seq1 = a.cu_seqlens[s + 1];
-    const int nq = (kend - kbeg + BM - 1) / BM;
-    const int qa = 2 * pair;                  // query tile of group 0; group 1 has qa + 1
+    const int nq = (kend - kbeg + BM - 1) / BM;      // query tiles of the sequence
+    const int nk = (kend - kbeg + BN - 1) / BN;      // key tiles of the sequence
+    const int qa = 2 * pair;                         // query tile of group 0; group 1 has qa + 1
     const bool two = qa + 1 < nq;
-    const int nt0 = qa + 1;                   // key tiles of query tile t: 0 .. its own index
-    const int nt = two ? qa + 2 : qa + 1;     // key tiles of the pair
+    // key tiles of query tile t: those up to the end of its rows
+    const int ntk[2] = {min(2 * qa + 2, nk), two ? min(2 * qa + 4, nk) : 0};
+    const int nt = two ? ntk[1] : ntk[0];            // key tiles loaded for the pair
     const int kblocks = a.dh / KB;
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -377,14 +386,17 @@ __global__ void __launch_bounds__(THREADS, 1)
         mbar_init(&sm->q_full, 1);
         for (int i = 0; i < KV_SLOTS; ++i) {
             mbar_init(&sm->kv_full[i], 1);
-            mbar_init(&sm->kv_empty[i], 1);
+            mbar_init(&sm->kv_empty[i], 2);
         }
-        for (int t = 0; t < 2; ++t) {
-            mbar_init(&sm->s_full[t], 1);
-            mbar_init(&sm->p_full[t], SOFTMAX_WARPS);
-            mbar_init(&sm->pv_done[t], 1);
-        }
-        mbar_init(&sm->done, 1);
+        for (int t = 0; t < 2; ++t)
+            for (int b = 0; b < 2; ++b) {
+                mbar_init(&sm->s_full[t][b], 1);
+                mbar_init(&sm->p_full[t][b], SOFTMAX_WARPS);
+                mbar_init(&sm->pv_done[t][b], 1);
+            }
+        mbar_init(&sm->vtail, 1);
+        mbar_init(&sm->done[0], 1);
+        mbar_init(&sm->done[1], 1);
         sm->abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -408,13 +420,12 @@ __global__ void __launch_bounds__(THREADS, 1)
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_v)) : "memory");
             const int col0 = h * a.dh;
             const int q0 = kbeg + qa * BM;
-            mbar_arrive_expect_tx(&sm->q_full, chunk_bytes(q0, kend, kblocks) +
-                                                   (two ? chunk_bytes(q0 + BM, kend, kblocks) : 0u));
-            load_tile(&tm_q, base + OFF_Q, q0, kend, a.kept_idx, seq0, seq1, col0, kblocks,
-                      &sm->q_full);
-            if (two)
-                load_tile(&tm_q, base + OFF_Q + TILE_BYTES, q0 + BM, kend, a.kept_idx, seq0, seq1,
-                          col0, kblocks, &sm->q_full);
+            uint32_t qbytes = 0;
+            for (int r = 0; r < (two ? 4 : 2); ++r) qbytes += run_bytes(q0 + 64 * r, kend, kblocks);
+            mbar_arrive_expect_tx(&sm->q_full, qbytes);
+            for (int r = 0; r < (two ? 4 : 2); ++r)   // query tile r / 2, 64-row half r % 2
+                load_run(&tm_q, base + OFF_Q + (r >> 1) * Q_TILE + (r & 1) * Q_CHUNK, Q_SLICE,
+                         q0 + 64 * r, kend, a.kept_idx, seq0, seq1, col0, kblocks, &sm->q_full);
             // loads n = 0, 1, 2, ...: K_{n/2} (n even) or V_{n/2} (n odd)
             const int nloads = 2 * nt;
             int n = 0;
@@ -422,9 +433,26 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const int slot = n % KV_SLOTS;
                 if (!wait(&sm->kv_empty[slot], ((n / KV_SLOTS) & 1) ^ 1, sm, lim)) break;
                 const int c0 = kbeg + (n >> 1) * BN;
-                mbar_arrive_expect_tx(&sm->kv_full[slot], chunk_bytes(c0, kend, kblocks));
-                load_tile((n & 1) ? &tm_v : &tm_k, base + OFF_KV + slot * TILE_BYTES, c0, kend,
-                          a.kept_idx, seq0, seq1, col0, kblocks, &sm->kv_full[slot]);
+                uint8_t* dst = base + OFF_KV + slot * KV_TILE;
+                const int nvalid = min(BN, kend - c0);
+                if ((n & 1) && nvalid < BN) {
+                    // the short last V tile: land it, zero the rows past the
+                    // kept set, then hand it to the MMAs
+                    mbar_arrive_expect_tx(&sm->vtail, run_bytes(c0, kend, kblocks));
+                    load_run(&tm_v, dst, KV_SLICE, c0, kend, a.kept_idx, seq0, seq1, col0,
+                             kblocks, &sm->vtail);
+                    if (!wait_drain(&sm->vtail, 0, lim)) break;
+                    for (int kc = 0; kc < kblocks; ++kc) {
+                        uint4* z = reinterpret_cast<uint4*>(dst + kc * KV_SLICE + nvalid * 128);
+                        for (int i = 0; i < (BN - nvalid) * 8; ++i) z[i] = make_uint4(0u, 0u, 0u, 0u);
+                    }
+                    fence_async_smem();
+                    mbar_arrive(&sm->kv_full[slot]);
+                    continue;
+                }
+                mbar_arrive_expect_tx(&sm->kv_full[slot], run_bytes(c0, kend, kblocks));
+                load_run((n & 1) ? &tm_v : &tm_k, dst, KV_SLICE, c0, kend, a.kept_idx, seq0, seq1,
+                         col0, kblocks, &sm->kv_full[slot]);
             }
             if (n < nloads) {
                 // gave up: every load issued lands before the CTA may exit
@@ -433,123 +461,91 @@ __global__ void __launch_bounds__(THREADS, 1)
                     wait_drain(&sm->kv_full[i % KV_SLOTS], (i / KV_SLOTS) & 1, lim);
             }
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        // A scheduler over both query tiles: op 2 j is S_t of key tile j,
-        // op 2 j + 1 is O_t += P_t V_j.  S_t(j) needs K_j loaded and (j > 0)
-        // P V of tile j - 1 completed (it overwrites P_t); P V(j) needs V_j
-        // loaded and P_t(j) written by the softmax group.  Lane 0 polls and
-        // issues; a K or V slot is released once every MMA reading it is
-        // issued.
+    } else if (warp == 1 || warp == 2) {
+        // ------------------------------------------------------------ MMA issuer of tile t
+        // Order: S(0), S(1), PV(0), S(2), PV(1), ..., S(n-1), PV(n-2), PV(n-1).
+        // S(j) needs K_j loaded and, for j >= 2, PV(j - 2) completed (it
+        // reuses that buffer); PV(j) needs V_j loaded and P(j) written.
+        const int t = warp - 1;
+        const int n = ntk[t];
+        bool ok = n > 0;
+        if (ok) ok = wait_warp(&sm->q_full, 0, sm, lim);
         const uint32_t idesc_pv = idesc(a.dh, true);
-        const uint32_t sq0 = smem_u32(base + OFF_Q);
-        int op[2] = {0, 0};
-        const int nops[2] = {2 * nt0, two ? 2 * nt : 0};
-        uint32_t half_used = 0;  // bit per slot: one of two MMAs on its tile issued
-        bool ok = wait_warp(&sm->q_full, 0, sm, lim);
-        tc_fence_after();
-        uint64_t t_wait = globaltimer_ns();
-        uint32_t spins = 0;
-        while (ok && (op[0] < nops[0] || op[1] < nops[1])) {
-            bool progressed = false;
-#pragma unroll
-            for (int t = 0; t < 2; ++t) {
-                if (op[t] >= nops[t]) continue;
-                const int j = op[t] >> 1;
-                const bool is_pv = op[t] & 1;
-                const int n = is_pv ? 2 * j + 1 : 2 * j;   // load number of the operand
-                const int slot = n % KV_SLOTS;
-                // readiness: operand loaded, and the group's own dependency
-                bool ready = mbar_try_wait(&sm->kv_full[slot], (n / KV_SLOTS) & 1);
-                if (ready) {
-                    if (is_pv) ready = mbar_try_wait(&sm->p_full[t], j & 1);
-                    else if (j > 0) ready = mbar_try_wait(&sm->pv_done[t], (j - 1) & 1);
-                }
-                ready = __shfl_sync(0xffffffffu, ready, 0);
-                if (!ready) continue;
-                tc_fence_after();
-                // MMAs that read this tile: one per query tile whose range has it
-                const int need = (j < nt0 ? 1 : 0) + (two ? 1 : 0);
-                const bool first = !((half_used >> slot) & 1u);
-                if (is_pv) {
-                    // rows of V past the kept set (a short last chunk) are
-                    // zeroed so that 0-probability keys contribute exactly 0
-                    // (by the first MMA on this V tile)
-                    const int nvalid = min(BN, kend - (kbeg + j * BN));
-                    if (nvalid < BN && first) {
-                        uint8_t* vt = base + OFF_KV + slot * TILE_BYTES;
-                        for (int kc = 0; kc < kblocks; ++kc) {
-                            uint4* p = reinterpret_cast<uint4*>(vt + kc * SLICE_BYTES + nvalid * 128);
-                            const int n16 = (BN - nvalid) * 8;
-                            for (int i = lane; i < n16; i += 32) p[i] = make_uint4(0u, 0u, 0u, 0u);
-                        }
-                        fence_async_smem();
-                        __syncwarp();
-                        tc_fence_after();
-                    }
-                    if (lane == 0) {
-                        const uint32_t sv = smem_u32(base + OFF_KV + slot * TILE_BYTES);
-                        for (int k = 0; k < BN / UMMA_K; ++k)
-                            umma_ts(tmem + O_COL + t * 128, tmem + t * BN + k * (UMMA_K / 2),
-                                    sdesc(sv + k * 2048, SLICE_BYTES), idesc_pv,
-                                    (j > 0 || k > 0) ? 1u : 0u);
-                        umma_commit(&sm->pv_done[t]);
-                    }
-                } else if (lane == 0) {
-                    const uint32_t sq = sq0 + t * TILE_BYTES;
-                    const uint32_t sk = smem_u32(base + OFF_KV + slot * TILE_BYTES);
-                    for (int k = 0; k < a.dh / UMMA_K; ++k) {
-                        const uint32_t off = (k >> 2) * SLICE_BYTES + (k & 3) * 32;
-                        umma(tmem + t * BN, sdesc(sq + off, 16), sdesc(sk + off, 16), kIdescS,
-                             k > 0);
-                    }
-                    umma_commit(&sm->s_full[t]);
-                }
-                if (need == 1 || !first) {  // last MMA on the tile: free its slot
-                    if (lane == 0) umma_commit(&sm->kv_empty[slot]);
-                    half_used &= ~(1u << slot);
-                } else {
-                    half_used |= 1u << slot;
-                }
-                __syncwarp();
-                ++op[t];
-                progressed = true;
+        const uint32_t sq = smem_u32(base + OFF_Q + t * Q_TILE);
+        // the other query tile does not read key tile j: release its share too
+        auto release = [&](int ld_no, int j) {
+            if (lane == 0) {
+                umma_commit(&sm->kv_empty[ld_no % KV_SLOTS]);
+                if (j >= ntk[t ^ 1]) umma_commit(&sm->kv_empty[ld_no % KV_SLOTS]);
             }
-            if (progressed) {
-                t_wait = globaltimer_ns();
-                spins = 0;
-            } else if ((++spins & 63) == 0) {
-                if (*reinterpret_cast<volatile int*>(&sm->abort_flag)) {
-                    ok = false;
-                } else if (globaltimer_ns() - t_wait > lim) {
-                    if (lane == 0) {
-                        raise_error(LEMO_ERR_TIMEOUT);
-                        abort_cta(sm);
-                    }
-                    ok = false;
+        };
+        auto issue_s = [&](int j) -> bool {
+            const int ld_no = 2 * j;
+            if (!wait_warp(&sm->kv_full[ld_no % KV_SLOTS], (ld_no / KV_SLOTS) & 1, sm, lim))
+                return false;
+            if (j >= 2 && !wait_warp(&sm->pv_done[t][j & 1], ((j - 2) >> 1) & 1, sm, lim))
+                return false;
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t sk = smem_u32(base + OFF_KV + (ld_no % KV_SLOTS) * KV_TILE);
+                const uint32_t d = tmem + t * 128 + (j & 1) * BN;
+                for (int k = 0; k < a.dh / UMMA_K; ++k) {
+                    const uint32_t qo = (k >> 2) * Q_SLICE + (k & 3) * 32;
+                    const uint32_t ko = (k >> 2) * KV_SLICE + (k & 3) * 32;
+                    umma(d, sdesc(sq + qo, 16), sdesc(sk + ko, 16), kIdescS, k > 0);
                 }
-                ok = __all_sync(0xffffffffu, ok);
+                umma_commit(&sm->s_full[t][j & 1]);
             }
+            release(ld_no, j);
+            __syncwarp();
+            return true;
+        };
+        auto issue_pv = [&](int j) -> bool {
+            const int ld_no = 2 * j + 1;
+            if (!wait_warp(&sm->kv_full[ld_no % KV_SLOTS], (ld_no / KV_SLOTS) & 1, sm, lim))
+                return false;
+            if (!wait_warp(&sm->p_full[t][j & 1], (j >> 1) & 1, sm, lim)) return false;
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t sv = smem_u32(base + OFF_KV + (ld_no % KV_SLOTS) * KV_TILE);
+                const uint32_t pa = tmem + t * 128 + (j & 1) * BN;
+                for (int k = 0; k < BN / UMMA_K; ++k)
+                    umma_ts(tmem + O_COL + t * 128, pa + k * (UMMA_K / 2),
+                            sdesc(sv + k * 2048, KV_SLICE), idesc_pv, (j > 0 || k > 0) ? 1u : 0u);
+                umma_commit(&sm->pv_done[t][j & 1]);
+            }
+            release(ld_no, j);
+            __syncwarp();
+            return true;
+        };
+        if (ok) ok = issue_s(0);
+        for (int j = 0; ok && j < n; ++j) {
+            if (j + 1 < n && !(ok = issue_s(j + 1))) break;
+            ok = issue_pv(j);
         }
         // every MMA completes before the tensor memory is released
-        if (lane == 0) umma_commit(&sm->done);
-        __syncwarp();
-        wait_drain(&sm->done, 0, lim);
-        __syncwarp();
+        if (n > 0) {
+            if (lane == 0) umma_commit(&sm->done[t]);
+            __syncwarp();
+            wait_drain(&sm->done[t], 0, lim);
+            __syncwarp();
+        }
     } else if (warp >= 4) {
         // ------------------------------------------------------------ softmax + epilogue
         const int t = (warp - 4) / SOFTMAX_WARPS;    // query tile of this group
         const int qd = warp & 3;                     // TMEM lane quadrant of this warp
         const int row = qd * 32 + lane;              // query row of this thread in the tile
         const int qc = kbeg + (qa + t) * BM + row;   // its compact (kept) index
-        const int ntt = t == 0 ? nt0 : nt;           // key tiles of this query tile
+        const int ntt = ntk[t];                      // key tiles of this query tile
         const uint32_t lrow = tmem + ((uint32_t)(qd * 32) << 16);
-        const uint32_t s_col = t * BN, o_col = O_COL + t * 128;
+        const uint32_t o_col = O_COL + t * 128;
         const float sl2 = a.scale_log2;
         float m = -CUDART_INF_F, l = 0.f;            // running max (log2 units) and sum
-        bool ok = t == 0 || two;
+        bool ok = ntt > 0;
         for (int j = 0; ok && j < ntt; ++j) {
-            if (!(ok = wait_warp(&sm->s_full[t], j & 1, sm, lim))) break;
+            const int b = j & 1;
+            const uint32_t s_col = t * 128 + b * BN;
+            if (!(ok = wait_warp(&sm->s_full[t][b], (j >> 1) & 1, sm, lim))) break;
             tc_fence_after();
             uint32_t r[BN];
 #pragma unroll
@@ -595,13 +591,16 @@ __global__ void __launch_bounds__(THREADS, 1)
                 pk[c >> 1] = pack_bf16(p0, p1);
             }
             l = l * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
-            // P_t over the first 64 columns of S_t (S_t is in registers; the
-            // MMA side writes S_t again only after P V of this tile)
+            // P_t(j) over the first 32 columns of its S buffer (S_t(j) is in
+            // registers; that buffer is written again only after P V(j))
 #pragma unroll
             for (int c = 0; c < BN / 2; c += 16) tmem_st16(lrow + s_col + c, &pk[c]);
-            // O_t is complete up to tile j - 1 here: S_t(j) was issued after
-            // P V(j - 1) had completed
             if (__any_sync(0xffffffffu, rescale)) {
+                // O_t must hold P V up to tile j - 1 before it is scaled
+                if (j > 0 && !(ok = wait_warp(&sm->pv_done[t][(j - 1) & 1], ((j - 1) >> 1) & 1,
+                                              sm, lim)))
+                    break;
+                tc_fence_after();
                 for (int c = 0; c < a.dh; c += 16) {
                     uint32_t o[16];
                     tmem_ld16(lrow + o_col + c, o);
@@ -614,9 +613,10 @@ __global__ void __launch_bounds__(THREADS, 1)
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm->p_full[t]);
+            if (lane == 0) mbar_arrive(&sm->p_full[t][b]);
         }
-        if (ok) ok = wait_warp(&sm->pv_done[t], (ntt - 1) & 1, sm, lim);
+        // the last P V of the tile (its commit covers every earlier MMA)
+        if (ok) ok = wait_warp(&sm->pv_done[t][(ntt - 1) & 1], ((ntt - 1) >> 1) & 1, sm, lim);
         if (ok) {
             tc_fence_after();
             const float inv = 1.f / l;

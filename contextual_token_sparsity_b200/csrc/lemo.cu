@@ -152,7 +152,7 @@ bool encode_rows(CUtensorMap* tm, const uint16_t* base, int64_t rows, int64_t wi
     if (!enc) return false;
     const cuuint64_t dims[2] = {(cuuint64_t)width, (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
-    const cuuint32_t box[2] = {(cuuint32_t)lemo::attn::KB, (cuuint32_t)lemo::attn::CHUNK};
+    const cuuint32_t box[2] = {(cuuint32_t)lemo::attn::KB, 64u};
     const cuuint32_t estr[2] = {1, 1};
     return enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(base), dims,
                strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
