@@ -461,61 +461,56 @@ __global__ void __launch_bounds__(THREADS, 1)
                     wait_drain(&sm->kv_full[i % KV_SLOTS], (i / KV_SLOTS) & 1, lim);
             }
         }
-    } else if (warp == 1 || warp == 2) {
+    } else if ((warp == 1 || warp == 2) && lane == 0) {
         // ------------------------------------------------------------ MMA issuer of tile t
-        // Order: S(0), S(1), PV(0), S(2), PV(1), ..., S(n-1), PV(n-2), PV(n-1).
-        // S(j) needs K_j loaded and, for j >= 2, PV(j - 2) completed (it
-        // reuses that buffer); PV(j) needs V_j loaded and P(j) written.
+        // One thread issues, waits and commits (no warp-wide votes or
+        // reconvergence between MMAs).  Order: S(0), S(1), PV(0), S(2),
+        // PV(1), ..., S(n-1), PV(n-2), PV(n-1).  S(j) needs K_j loaded and,
+        // for j >= 2, PV(j - 2) completed (it reuses that buffer); PV(j)
+        // needs V_j loaded and P(j) written.
         const int t = warp - 1;
         const int n = ntk[t];
         bool ok = n > 0;
-        if (ok) ok = wait_warp(&sm->q_full, 0, sm, lim);
+        if (ok) ok = wait(&sm->q_full, 0, sm, lim);
         const uint32_t idesc_pv = idesc(a.dh, true);
         const uint32_t sq = smem_u32(base + OFF_Q + t * Q_TILE);
+        const int nko = ntk[t ^ 1];
         // the other query tile does not read key tile j: release its share too
         auto release = [&](int ld_no, int j) {
-            if (lane == 0) {
-                umma_commit(&sm->kv_empty[ld_no % KV_SLOTS]);
-                if (j >= ntk[t ^ 1]) umma_commit(&sm->kv_empty[ld_no % KV_SLOTS]);
-            }
+            umma_commit(&sm->kv_empty[ld_no % KV_SLOTS]);
+            if (j >= nko) umma_commit(&sm->kv_empty[ld_no % KV_SLOTS]);
         };
         auto issue_s = [&](int j) -> bool {
             const int ld_no = 2 * j;
-            if (!wait_warp(&sm->kv_full[ld_no % KV_SLOTS], (ld_no / KV_SLOTS) & 1, sm, lim))
+            if (!wait(&sm->kv_full[ld_no % KV_SLOTS], (ld_no / KV_SLOTS) & 1, sm, lim))
                 return false;
-            if (j >= 2 && !wait_warp(&sm->pv_done[t][j & 1], ((j - 2) >> 1) & 1, sm, lim))
+            if (j >= 2 && !wait(&sm->pv_done[t][j & 1], ((j - 2) >> 1) & 1, sm, lim))
                 return false;
             tc_fence_after();
-            if (lane == 0) {
-                const uint32_t sk = smem_u32(base + OFF_KV + (ld_no % KV_SLOTS) * KV_TILE);
-                const uint32_t d = tmem + t * 128 + (j & 1) * BN;
-                for (int k = 0; k < a.dh / UMMA_K; ++k) {
-                    const uint32_t qo = (k >> 2) * Q_SLICE + (k & 3) * 32;
-                    const uint32_t ko = (k >> 2) * KV_SLICE + (k & 3) * 32;
-                    umma(d, sdesc(sq + qo, 16), sdesc(sk + ko, 16), kIdescS, k > 0);
-                }
-                umma_commit(&sm->s_full[t][j & 1]);
+            const uint32_t sk = smem_u32(base + OFF_KV + (ld_no % KV_SLOTS) * KV_TILE);
+            const uint32_t d = tmem + t * 128 + (j & 1) * BN;
+            for (int k = 0; k < a.dh / UMMA_K; ++k) {
+                const uint32_t qo = (k >> 2) * Q_SLICE + (k & 3) * 32;
+                const uint32_t ko = (k >> 2) * KV_SLICE + (k & 3) * 32;
+                umma(d, sdesc(sq + qo, 16), sdesc(sk + ko, 16), kIdescS, k > 0);
             }
+            umma_commit(&sm->s_full[t][j & 1]);
             release(ld_no, j);
-            __syncwarp();
             return true;
         };
         auto issue_pv = [&](int j) -> bool {
             const int ld_no = 2 * j + 1;
-            if (!wait_warp(&sm->kv_full[ld_no % KV_SLOTS], (ld_no / KV_SLOTS) & 1, sm, lim))
+            if (!wait(&sm->kv_full[ld_no % KV_SLOTS], (ld_no / KV_SLOTS) & 1, sm, lim))
                 return false;
-            if (!wait_warp(&sm->p_full[t][j & 1], (j >> 1) & 1, sm, lim)) return false;
+            if (!wait(&sm->p_full[t][j & 1], (j >> 1) & 1, sm, lim)) return false;
             tc_fence_after();
-            if (lane == 0) {
-                const uint32_t sv = smem_u32(base + OFF_KV + (ld_no % KV_SLOTS) * KV_TILE);
-                const uint32_t pa = tmem + t * 128 + (j & 1) * BN;
-                for (int k = 0; k < BN / UMMA_K; ++k)
-                    umma_ts(tmem + O_COL + t * 128, pa + k * (UMMA_K / 2),
-                            sdesc(sv + k * 2048, KV_SLICE), idesc_pv, (j > 0 || k > 0) ? 1u : 0u);
-                umma_commit(&sm->pv_done[t][j & 1]);
-            }
+            const uint32_t sv = smem_u32(base + OFF_KV + (ld_no % KV_SLOTS) * KV_TILE);
+            const uint32_t pa = tmem + t * 128 + (j & 1) * BN;
+            for (int k = 0; k < BN / UMMA_K; ++k)
+                umma_ts(tmem + O_COL + t * 128, pa + k * (UMMA_K / 2),
+                        sdesc(sv + k * 2048, KV_SLICE), idesc_pv, (j > 0 || k > 0) ? 1u : 0u);
+            umma_commit(&sm->pv_done[t][j & 1]);
             release(ld_no, j);
-            __syncwarp();
             return true;
         };
         if (ok) ok = issue_s(0);
@@ -525,10 +520,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         // every MMA completes before the tensor memory is released
         if (n > 0) {
-            if (lane == 0) umma_commit(&sm->done[t]);
-            __syncwarp();
+            umma_commit(&sm->done[t]);
             wait_drain(&sm->done[t], 0, lim);
-            __syncwarp();
         }
     } else if (warp >= 4) {
         // ------------------------------------------------------------ softmax + epilogue
