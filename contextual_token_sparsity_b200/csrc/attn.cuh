@@ -25,8 +25,9 @@
 //   warp 0      TMA producer: both query tiles once, then K_0, V_0, K_1,
 //               V_1, ... (key tiles of 64 kept rows, 16 KB each) through a
 //               10-slot ring;
-//   warps 1, 2  MMA issuers (tcgen05, cta_group::1, M = 128), warp 1 for
-//               query tile 0 and warp 2 for query tile 1.  For key tile j:
+//   warps 1, 2  S issuers for query tiles 0 and 1, warps 3, 12 P V issuers
+//               for query tiles 0 and 1 (one thread each; tcgen05,
+//               cta_group::1, M = 128).  For key tile j:
 //                 S_t(j) = Q_t K_j^T      into TMEM columns [128 t + 64 (j%2), +64)
 //                 O_t += P_t(j) V_j       into TMEM columns [256 + 128 t, +dh)
 //               where P_t(j) is read from TMEM (A operand) and V is the
@@ -84,7 +85,7 @@ constexpr int Q_TILE = (MAX_DH / KB) * Q_SLICE;    // 32 KB
 constexpr int KV_SLICE = BN * KB * 2;              // 64 rows x 64 elements: 8 KB
 constexpr int KV_TILE = (MAX_DH / KB) * KV_SLICE;  // 16 KB
 constexpr int SOFTMAX_WARPS = 4;                   // per group (one warpgroup)
-constexpr int THREADS = 32 * 12;
+constexpr int THREADS = 32 * 16;
 constexpr int KV_SLOTS = 10;
 constexpr int TMEM_COLS = 512;   // S_0 [0,128), S_1 [128,256), O_0 [256,+dh), O_1 [384,+dh)
 constexpr int O_COL = 256;
@@ -103,7 +104,7 @@ struct Smem {
     uint64_t p_full[2][2];        // [tile][buffer] P_t(j) in TMEM (and O_t rescaled)
     uint64_t pv_done[2][2];       // [tile][buffer] O_t += P_t(j) V_j completed
     uint64_t vtail;               // the short last V tile has landed (producer only)
-    uint64_t done[2];             // every MMA of issuer t completed
+    uint64_t done[4];             // every MMA of issuer i completed
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -395,8 +396,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 mbar_init(&sm->pv_done[t][b], 1);
             }
         mbar_init(&sm->vtail, 1);
-        mbar_init(&sm->done[0], 1);
-        mbar_init(&sm->done[1], 1);
+        for (int i = 0; i < 4; ++i) mbar_init(&sm->done[i], 1);
         sm->abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -461,69 +461,57 @@ __global__ void __launch_bounds__(THREADS, 1)
                     wait_drain(&sm->kv_full[i % KV_SLOTS], (i / KV_SLOTS) & 1, lim);
             }
         }
-    } else if ((warp == 1 || warp == 2) && lane == 0) {
-        // ------------------------------------------------------------ MMA issuer of tile t
-        // One thread issues, waits and commits (no warp-wide votes or
-        // reconvergence between MMAs).  Order: S(0), S(1), PV(0), S(2),
-        // PV(1), ..., S(n-1), PV(n-2), PV(n-1).  S(j) needs K_j loaded and,
-        // for j >= 2, PV(j - 2) completed (it reuses that buffer); PV(j)
-        // needs V_j loaded and P(j) written.
-        const int t = warp - 1;
+    } else if ((warp == 1 || warp == 2 || warp == 3 || warp == 12) && lane == 0) {
+        // ------------------------------------------------------------ MMA issuers
+        // One thread per chain, waiting, issuing and committing alone.
+        //   S issuer of tile t:   S(j) needs K_j loaded and, for j >= 2,
+        //                         PV(j - 2) completed (it reuses that buffer);
+        //   P V issuer of tile t: PV(j) needs V_j loaded and P(j) written.
+        // A K slot is released by the S issuers, a V slot by the P V issuers;
+        // a chain releases the other tile's share of a key tile that the
+        // other tile does not read.
+        const bool is_s = warp <= 2;
+        const int t = (warp == 1 || warp == 3) ? 0 : 1;
+        const int id = is_s ? t : 2 + t;
         const int n = ntk[t];
+        const int nko = ntk[t ^ 1];
         bool ok = n > 0;
-        if (ok) ok = wait(&sm->q_full, 0, sm, lim);
+        if (ok && is_s) ok = wait(&sm->q_full, 0, sm, lim);
         const uint32_t idesc_pv = idesc(a.dh, true);
         const uint32_t sq = smem_u32(base + OFF_Q + t * Q_TILE);
-        const int nko = ntk[t ^ 1];
-        // the other query tile does not read key tile j: release its share too
-        auto release = [&](int ld_no, int j) {
-            umma_commit(&sm->kv_empty[ld_no % KV_SLOTS]);
-            if (j >= nko) umma_commit(&sm->kv_empty[ld_no % KV_SLOTS]);
-        };
-        auto issue_s = [&](int j) -> bool {
-            const int ld_no = 2 * j;
-            if (!wait(&sm->kv_full[ld_no % KV_SLOTS], (ld_no / KV_SLOTS) & 1, sm, lim))
-                return false;
-            if (j >= 2 && !wait(&sm->pv_done[t][j & 1], ((j - 2) >> 1) & 1, sm, lim))
-                return false;
-            tc_fence_after();
-            const uint32_t sk = smem_u32(base + OFF_KV + (ld_no % KV_SLOTS) * KV_TILE);
-            const uint32_t d = tmem + t * 128 + (j & 1) * BN;
-            for (int k = 0; k < a.dh / UMMA_K; ++k) {
-                const uint32_t qo = (k >> 2) * Q_SLICE + (k & 3) * 32;
-                const uint32_t ko = (k >> 2) * KV_SLICE + (k & 3) * 32;
-                umma(d, sdesc(sq + qo, 16), sdesc(sk + ko, 16), kIdescS, k > 0);
-            }
-            umma_commit(&sm->s_full[t][j & 1]);
-            release(ld_no, j);
-            return true;
-        };
-        auto issue_pv = [&](int j) -> bool {
-            const int ld_no = 2 * j + 1;
-            if (!wait(&sm->kv_full[ld_no % KV_SLOTS], (ld_no / KV_SLOTS) & 1, sm, lim))
-                return false;
-            if (!wait(&sm->p_full[t][j & 1], (j >> 1) & 1, sm, lim)) return false;
-            tc_fence_after();
-            const uint32_t sv = smem_u32(base + OFF_KV + (ld_no % KV_SLOTS) * KV_TILE);
-            const uint32_t pa = tmem + t * 128 + (j & 1) * BN;
-            for (int k = 0; k < BN / UMMA_K; ++k)
-                umma_ts(tmem + O_COL + t * 128, pa + k * (UMMA_K / 2),
-                        sdesc(sv + k * 2048, KV_SLICE), idesc_pv, (j > 0 || k > 0) ? 1u : 0u);
-            umma_commit(&sm->pv_done[t][j & 1]);
-            release(ld_no, j);
-            return true;
-        };
-        if (ok) ok = issue_s(0);
         for (int j = 0; ok && j < n; ++j) {
-            if (j + 1 < n && !(ok = issue_s(j + 1))) break;
-            ok = issue_pv(j);
+            const int ld_no = 2 * j + (is_s ? 0 : 1);
+            const int slot = ld_no % KV_SLOTS;
+            if (!(ok = wait(&sm->kv_full[slot], (ld_no / KV_SLOTS) & 1, sm, lim))) break;
+            const uint32_t tile = smem_u32(base + OFF_KV + slot * KV_TILE);
+            const uint32_t sbuf = tmem + t * 128 + (j & 1) * BN;
+            if (is_s) {
+                if (j >= 2 && !(ok = wait(&sm->pv_done[t][j & 1], ((j - 2) >> 1) & 1, sm, lim)))
+                    break;
+                tc_fence_after();
+                for (int k = 0; k < a.dh / UMMA_K; ++k) {
+                    const uint32_t qo = (k >> 2) * Q_SLICE + (k & 3) * 32;
+                    const uint32_t ko = (k >> 2) * KV_SLICE + (k & 3) * 32;
+                    umma(sbuf, sdesc(sq + qo, 16), sdesc(tile + ko, 16), kIdescS, k > 0);
+                }
+                umma_commit(&sm->s_full[t][j & 1]);
+            } else {
+                if (!(ok = wait(&sm->p_full[t][j & 1], (j >> 1) & 1, sm, lim))) break;
+                tc_fence_after();
+                for (int k = 0; k < BN / UMMA_K; ++k)
+                    umma_ts(tmem + O_COL + t * 128, sbuf + k * (UMMA_K / 2),
+                            sdesc(tile + k * 2048, KV_SLICE), idesc_pv, (j > 0 || k > 0) ? 1u : 0u);
+                umma_commit(&sm->pv_done[t][j & 1]);
+            }
+            umma_commit(&sm->kv_empty[slot]);
+            if (j >= nko) umma_commit(&sm->kv_empty[slot]);
         }
         // every MMA completes before the tensor memory is released
         if (n > 0) {
-            umma_commit(&sm->done[t]);
-            wait_drain(&sm->done[t], 0, lim);
+            umma_commit(&sm->done[id]);
+            wait_drain(&sm->done[id], 0, lim);
         }
-    } else if (warp >= 4) {
+    } else if (warp >= 4 && warp < 12) {
         // ------------------------------------------------------------ softmax + epilogue
         const int t = (warp - 4) / SOFTMAX_WARPS;    // query tile of this group
         const int qd = warp & 3;                     // TMEM lane quadrant of this warp
