@@ -855,9 +855,10 @@ def run_predict(args):
     out["movement"] = {"gather_gbs": round(g_b / (us["gather"] * 1e-6) / 1e9, 1),
                        "scatter_gbs": round(s_b / (us["scatter"] * 1e-6) / 1e9, 1),
                        "hbm_peak_gbs": bw}
-    # predict: plan, pool, 2 x (gemm, reduce, gemm), products, column sum;
-    # select: plan, select; gather; scatter
-    out["gpu_launches"] = 14 * args.steps
+    # predict: plan, pool, both predictors' first GEMM, split-K reduce, both
+    # second GEMMs, block products, head-group reduce, column sum; select:
+    # plan, select; gather; scatter
+    out["gpu_launches"] = 12 * args.steps
     out["clocks"] = clk
     if not args.no_e2e:
         pin = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).pin_memory()  # noqa

@@ -765,13 +765,11 @@ lemo_status lemo_predict_scores(const lemo_shape* shape, int32_t d, const uint16
     launch(pr::products_kernel, dim3((unsigned)p.ptiles, (unsigned)p.groups), pr::kMmaThreads, 0,
            st, pa, w, lay);
     if ((e = launch_status()) != LEMO_OK) return e;
+    if (p.groups > 1) launch(pr::products_reduce_kernel, sms * 2, 256, 0, st, pa, w, lay);
     const int64_t cs_ctas = (p.tb + 7) / 8;
     const int cs_grid = (int)(cs_ctas < (int64_t)sms * 8 ? cs_ctas : sms * 8);
-    if (p.groups > 1)
-        launch(pr::plane_column_sum_kernel, cs_grid, 256, 0, st, pa, w, lay, block_scores);
-    else
-        launch(lemo::score::column_sum_kernel, cs_grid, 256, 0, st, P, w, lay, shape->batch,
-               block_scores);
+    launch(lemo::score::column_sum_kernel, cs_grid, 256, 0, st, P, w, lay, shape->batch,
+           block_scores);
     return launch_status();
 }
 

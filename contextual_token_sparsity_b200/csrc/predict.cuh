@@ -393,35 +393,29 @@ __global__ void __launch_bounds__(kMmaThreads)
     }
 }
 
-// Column sums straight from the partial planes (head groups > 1):
-// score[m] = inv_h * sum_{n >= m, same sequence} sum_g part[g][n][m].  One
-// warp per token block; lane l takes rows n = m + l, m + l + 32, ... in
-// increasing order and the groups in increasing order, then a fixed
-// butterfly combines the lanes: the same bits on every run.
+// P[n][m] = inv_h * sum_g part[g][n][m], g in increasing order, for the
+// pairs of one sequence with n >= m (head groups > 1).  Threads run along
+// m, so the partial planes are read with coalesced loads.
 __global__ void __launch_bounds__(256)
-    plane_column_sum_kernel(const ProductsArgs a, const char* __restrict__ ws, WsLayout lay,
-                            float* __restrict__ scores) {
+    products_reduce_kernel(const ProductsArgs a, const char* __restrict__ ws, WsLayout lay) {
     pdl_entry();
     const PlanHeader* hdr = reinterpret_cast<const PlanHeader*>(ws + lay.hdr);
     if (!hdr->valid) return;
     const int32_t* blk_prefix = reinterpret_cast<const int32_t*>(ws + lay.blk_prefix);
-    const int total = hdr->total_blocks;
+    const int64_t* m_prefix = reinterpret_cast<const int64_t*>(ws + lay.m_prefix);
+    const int TB = hdr->total_blocks;
+    const int64_t total = (int64_t)TB * TB;
     const int64_t plane = a.tb_cap * a.tb_cap;
-    const int lane = threadIdx.x & 31;
-    const int warps = (gridDim.x * blockDim.x) >> 5;
-    for (int m = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; m < total; m += warps) {
-        const int s = last_le(blk_prefix, a.batch + 1, m);
-        const int end = blk_prefix[s + 1];
-        float sum = 0.f;
-        for (int n = m + lane; n < end; n += 32) {
-            const float* src = a.part + (int64_t)n * a.tb_cap + m;
-            float v = 0.f;
-            for (int g = 0; g < a.groups; ++g) v += src[g * plane];
-            sum += v;
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-        if (lane == 0) scores[m] = sum * a.inv_h;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int n = (int)(i / TB), m = (int)(i % TB);
+        if (m > n) continue;
+        const int s = last_le(blk_prefix, a.batch + 1, n);
+        if (m < blk_prefix[s]) continue;
+        const int64_t o = (int64_t)n * a.tb_cap + m;
+        float v = 0.f;
+        for (int g = 0; g < a.groups; ++g) v += a.part[g * plane + o];
+        store_pair(a, blk_prefix, m_prefix, s, n, m, v);
     }
 }
 
