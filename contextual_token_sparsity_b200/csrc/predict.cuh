@@ -281,8 +281,17 @@ __global__ void __launch_bounds__(256)
     float* dst = hid + blockIdx.y * hid_side_stride;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
          i += (int64_t)gridDim.x * blockDim.x) {
+        // loads in batches of 8 (in flight together), added in z order
         float v = 0.f;
-        for (int z = 0; z < splits; ++z) v += src[(int64_t)z * plane + i];
+        int z = 0;
+        for (; z + 8 <= splits; z += 8) {
+            float t[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) t[u] = src[(int64_t)(z + u) * plane + i];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v += t[u];
+        }
+        for (; z < splits; ++z) v += src[(int64_t)z * plane + i];
         dst[i] = fmaxf(v, 0.f);
     }
 }
@@ -413,8 +422,17 @@ __global__ void __launch_bounds__(256)
         const int s = last_le(blk_prefix, a.batch + 1, n);
         if (m < blk_prefix[s]) continue;
         const int64_t o = (int64_t)n * a.tb_cap + m;
+        // loads in batches of 8 (in flight together), added in g order
         float v = 0.f;
-        for (int g = 0; g < a.groups; ++g) v += a.part[g * plane + o];
+        int g = 0;
+        for (; g + 8 <= a.groups; g += 8) {
+            float t[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) t[u] = a.part[(g + u) * plane + o];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v += t[u];
+        }
+        for (; g < a.groups; ++g) v += a.part[g * plane + o];
         store_pair(a, blk_prefix, m_prefix, s, n, m, v);
     }
 }

@@ -538,8 +538,17 @@ __global__ void __launch_bounds__(256) column_sum_kernel(const float* __restrict
         const int m = g - blk_prefix[s];
         const int nb = blk_prefix[s + 1] - blk_prefix[s];
         const float* col = mblk + m_prefix[s] + m;
+        // rows in batches of 4 per lane (loads in flight together), added in n order
         float sum = 0.f;
-        for (int n = m + lane; n < nb; n += 32) sum += col[(int64_t)n * nb];
+        int n = m + lane;
+        for (; n + 96 < nb; n += 128) {
+            float t[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) t[u] = col[(int64_t)(n + 32 * u) * nb];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) sum += t[u];
+        }
+        for (; n < nb; n += 32) sum += col[(int64_t)n * nb];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
         if (lane == 0) scores[g] = sum;
