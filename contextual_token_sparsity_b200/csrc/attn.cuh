@@ -327,6 +327,32 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// Packed fp32 pairs (one instruction for two lanes of work) and the
+// three-input maximum of sm_100.
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+    uint64_t v;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "f"(lo), "f"(hi));
+    return v;
+}
+__device__ __forceinline__ void unf2(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     const __nv_bfloat162 r = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<const uint32_t*>(&r);
@@ -540,17 +566,17 @@ __global__ void __launch_bounds__(THREADS, 1)
                 for (int c = 0; c < BN; ++c)
                     if (c >= ncols) r[c] = __float_as_uint(-CUDART_INF_F);
             }
-            // row maximum: 8 independent partial maxima, then a tree
+            // row maximum: 8 independent chains of three-input maxima, then a tree
             float mx[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) mx[i] = __uint_as_float(r[i]);
 #pragma unroll
-            for (int c = 8; c < BN; ++c) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(r[c]));
+            for (int c = 8; c < BN; c += 16)
 #pragma unroll
-            for (int w = 4; w > 0; w >>= 1)
-#pragma unroll
-                for (int i = 0; i < w; ++i) mx[i] = fmaxf(mx[i], mx[i + w]);
-            const float mt = mx[0] * sl2;
+                for (int i = 0; i < 8; ++i)
+                    mx[i] = max3(mx[i], __uint_as_float(r[c + i]), __uint_as_float(r[c + 8 + i]));
+            const float mt =
+                max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * sl2;
             bool rescale = false;
             float alpha = 1.f;
             if (j == 0) {
@@ -560,18 +586,23 @@ __global__ void __launch_bounds__(THREADS, 1)
                 m = mt;
                 rescale = true;
             }
-            // probabilities as bf16 pairs, 4 partial sums
-            const float nm = -m;
+            // probabilities as bf16 pairs; exponent arguments and partial
+            // sums on packed fp32 pairs (2 pair sums x 2 lanes)
+            const uint64_t sc2 = f2(sl2, sl2), nm2 = f2(-m, -m);
             uint32_t pk[BN / 2];
-            float ps[4] = {0.f, 0.f, 0.f, 0.f};
+            uint64_t ps2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
 #pragma unroll
             for (int c = 0; c < BN; c += 2) {
-                const float p0 = ex2(fmaf(__uint_as_float(r[c]), sl2, nm));
-                const float p1 = ex2(fmaf(__uint_as_float(r[c + 1]), sl2, nm));
-                ps[(c >> 1) & 3] += p0 + p1;
+                float x0, x1;
+                unf2(fma_f32x2(f2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), sc2, nm2), x0, x1);
+                const float p0 = ex2(x0), p1 = ex2(x1);
+                ps2[(c >> 1) & 1] = add_f32x2(ps2[(c >> 1) & 1], f2(p0, p1));
                 pk[c >> 1] = pack_bf16(p0, p1);
             }
-            l = l * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
+            float a0, a1, b0, b1;
+            unf2(ps2[0], a0, a1);
+            unf2(ps2[1], b0, b1);
+            l = l * alpha + ((a0 + a1) + (b0 + b1));
             // P_t(j) over the first 32 columns of its S buffer (S_t(j) is in
             // registers; that buffer is written again only after P V(j))
 #pragma unroll
