@@ -311,6 +311,33 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
         : "memory");
 }
 
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+        "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+        "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -555,8 +582,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (!(ok = wait_warp(&sm->s_full[t][b], (j >> 1) & 1, sm, lim))) break;
             tc_fence_after();
             uint32_t r[BN];
-#pragma unroll
-            for (int c = 0; c < BN; c += 16) tmem_ld16(lrow + s_col + c, &r[c]);
+            tmem_ld32(lrow + s_col, &r[0]);
+            tmem_ld32(lrow + s_col + 32, &r[32]);
             tmem_wait_ld();
             // keys past the query (causal) or past the kept set are masked
             const int c0 = kbeg + j * BN;
@@ -605,8 +632,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             l = l * alpha + ((a0 + a1) + (b0 + b1));
             // P_t(j) over the first 32 columns of its S buffer (S_t(j) is in
             // registers; that buffer is written again only after P V(j))
-#pragma unroll
-            for (int c = 0; c < BN / 2; c += 16) tmem_st16(lrow + s_col + c, &pk[c]);
+            tmem_st32(lrow + s_col, pk);
             if (__any_sync(0xffffffffu, rescale)) {
                 // O_t must hold P V up to tile j - 1 before it is scaled
                 if (j > 0 && !(ok = wait_warp(&sm->pv_done[t][(j - 1) & 1], ((j - 1) >> 1) & 1,
