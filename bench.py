@@ -423,17 +423,38 @@ def run_e2e(args, host, layers, thetas, dev, world, local, tokens_per_step):
     h2d = sum(t.numel() * 2 for t in hq + hk + hy) + hx.numel() * 2
     d2h = hx_out.numel() * 2 + sum(t.numel() * 4 for t in hs_out)
 
+    # Host -> device copies run on their own stream, ordered by events: layer
+    # l + 1's inputs upload while layer l computes, and a layer's device
+    # buffers are refilled only after the previous step's use of them.
+    cs = torch.cuda.Stream(device=dev)
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    ready, used = [ev() for _ in range(nl)], [ev() for _ in range(nl)]
+    x_ready, x_used = ev(), ev()
+    for e in used + [x_used]:
+        e.record(stream)
+
     def step():
-        dx.copy_(hx, non_blocking=True)
+        with torch.cuda.stream(cs):
+            for l in range(nl):
+                cs.wait_event(used[l])
+                dq[l].copy_(hq[l], non_blocking=True)
+                dk[l].copy_(hk[l], non_blocking=True)
+                dy[l].copy_(hy[l], non_blocking=True)
+                ready[l].record(cs)
+                if l == 0:  # the residual stream right after the first layer's inputs
+                    cs.wait_event(x_used)
+                    dx.copy_(hx, non_blocking=True)
+                    x_ready.record(cs)
+        stream.wait_event(x_ready)
         for l in range(nl):
-            dq[l].copy_(hq[l], non_blocking=True)
-            dk[l].copy_(hk[l], non_blocking=True)
-            dy[l].copy_(hy[l], non_blocking=True)
+            stream.wait_event(ready[l])
             L_ = layers[l]
             L_.step(dq[l].view(torch.bfloat16), dk[l].view(torch.bfloat16), thetas[l],
                     dx.view(torch.bfloat16), dy[l].view(torch.bfloat16))
+            used[l].record(stream)
             hs_out[l].copy_(L_.block_scores, non_blocking=True)
         hx_out.copy_(dx, non_blocking=True)
+        x_used.record(stream)
 
     steps = max(3, min(args.steps, args.e2e_steps))
     for _ in range(2):
@@ -444,6 +465,7 @@ def run_e2e(args, host, layers, thetas, dev, world, local, tokens_per_step):
     barrier(world, local)
     torch.cuda.synchronize()
     a.record(stream)
+    cs.wait_event(a)  # no copy of the timed steps starts before the clock
     for _ in range(steps):
         step()
     b.record(stream)
@@ -453,7 +475,8 @@ def run_e2e(args, host, layers, thetas, dev, world, local, tokens_per_step):
     return {"value": round(whole_job_rate(tokens_per_step, world, s / steps), 1), "unit": UNIT,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
             "ms_per_step": round(1e3 * s / steps, 3),
-            "path": "pinned host -> device copies, lemo_* calls, device -> pinned host copies"}
+            "path": "pinned host -> device copies (own stream, overlapping the previous layer), "
+                    "lemo_* calls, device -> pinned host copies"}
 
 
 # ----------------------------------------------------------------------------
