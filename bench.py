@@ -561,6 +561,8 @@ def run_segloss(args):
         "gpu_launches": (2 + -(-T // S)) * args.steps,
         "clocks": clk,
     }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = ext_cpu_baseline("lmhead-7b", args.cpu_seconds)
     if world > 1:
         import torch.distributed as dist
         dist.barrier(device_ids=[local])
@@ -785,6 +787,8 @@ def run_attention(args):
                           list(zip(hq, dq)) + list(zip(hk, dk)) + list(zip(hv, dv)) + [(hxp, dx)],
                           [(dx, hx_out)],
                           lambda: call(dx.view(torch.bfloat16), bf(dq), bf(dk), bf(dv)))
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = ext_cpu_baseline("attn-c3", args.cpu_seconds)
     _finish(out, world, local, rank)
 
 
@@ -893,6 +897,8 @@ def run_predict(args):
         out["e2e"] = _e2e(max(3, min(args.steps, args.e2e_steps)), world, local, dev, L,
                           [(hxp, dx), (hyp, dy)], [(dx, hx_out), (layer.block_scores, hs)],
                           lambda: call(dx.view(torch.bfloat16), dy.view(torch.bfloat16)))
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = ext_cpu_baseline("predict-c5", args.cpu_seconds)
     _finish(out, world, local, rank)
 
 
@@ -980,6 +986,8 @@ def run_mlp(args):
         out["e2e"] = _e2e(max(3, min(args.steps, args.e2e_steps)), world, local, dev, L,
                           list(zip((hg, hu, hxp, hyp), dd)), [(dd[2], hx_out)],
                           lambda: call(*[t.view(torch.bfloat16) for t in dd]))
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = ext_cpu_baseline("mlp-7b", args.cpu_seconds)
     _finish(out, world, local, rank)
 
 
@@ -1076,6 +1084,125 @@ def cpu_baseline(key: str, budget_s: float = 20.0, layer: int = 0):
             "seconds_per_layer_estimate": round(t_layer, 2)}
 
 
+def oracle_sample(workload: str, budget_s: float = 20.0, seed: int = 0):
+    """The CPU oracle, as it stands, on a bounded sample of an extension
+    workload.  Returns (estimated seconds per layer / call, tokens it covers,
+    description of the sample)."""
+    import oracle
+    from contextual_token_sparsity_b200 import synth
+    rng = np.random.default_rng(seed)
+    if workload == "predict-c5":
+        w = synth.WORKLOADS["c5"]
+        sd, L, d, hd = int(w.seeds[0]), w.total_L, w.d, w.H * w.dh
+        with open(os.path.join(ROOT, "tests", "golden", "c5.json")) as f:
+            theta = float(json.load(f)["layers"][0]["pred_theta"])
+        xb, _ = synth.projected_x(L, d, float(w.salient), sd)
+        w1q, w2q, lq = synth.predictor_weights(d, w.predictor_rank, hd, 0.4, sd, 10)
+        w1k, w2k, lk = synth.predictor_weights(d, w.predictor_rank, hd, 0.4, sd, 11)
+        y = synth.normal_bf16(L, d, sd, 8)
+        cu = np.array([0, L], dtype=np.int32)
+        t0 = time.perf_counter()
+        reps = oracle.block_representatives(xb, cu, w.block)
+        qh = oracle.predictor_embeddings(reps, w1q[:, lq], w2q[lq])
+        kh = oracle.predictor_embeddings(reps, w1k[:, lk], w2k[lk])
+        _, ps = oracle.predict_scores(qh, kh, cu, w.block, w.H, w.dh)
+        idx, _, _ = oracle.compact(oracle.keep_mask(ps, theta), cu, w.block)
+        oracle.gather_pad(xb, idx, PAD_TO)
+        oracle.scatter_residual(xb, y, idx)
+        t = time.perf_counter() - t0
+        return t, L, (f"predict-c5 in full ({t:.1f} s): block means, both predictors, Eq. 3 block "
+                      "products, threshold, compaction, gather and scatter; float64 numpy")
+    if workload == "attn-c3":
+        w = synth.WORKLOADS["c3"]
+        with open(os.path.join(ROOT, "tests", "golden", "c3.json")) as f:
+            g = json.load(f)["layers"][1]
+        inp = synth.make_workload("c3", 1, with_x=False)
+        hd = w.H * w.dh
+        v = synth.normal_bf16(w.total_L, hd, int(w.seeds[1]), 22)
+        mask = oracle.keep_mask(np.array([float(x) for x in g["scores"]]), float(g["theta"]))
+        idx, cu_k, K = oracle.compact(mask, inp["cu_seqlens"], w.block)
+        order = rng.permutation(K)
+        t0 = time.perf_counter()
+        pairs = rows = 0
+        for r in order:
+            oracle.attention_kept_rows(inp["q"], inp["k"], v, idx[:K], cu_k, w.H, w.dh, [int(r)])
+            pairs += int(r) + 1
+            rows += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
+        t = time.perf_counter() - t0
+        all_pairs = K * (K + 1) // 2
+        return t * all_pairs / pairs, w.total_L, (
+            f"layer 1 of attn-c3 (K = {K}): {rows} of {K} query rows ({pairs} of {all_pairs} "
+            f"query-key pairs, {t:.1f} s) by the oracle, scaled by pairs; float64 numpy")
+    if workload == "mlp-7b":
+        L, d_ff, d, b = 16384, 11008, 4096, 64
+        gate, up = synth.mlp_activations(L, d_ff, 0.1, seed=0, gated=True)
+        chunk, t_sc, done = 512, 0.0, 0
+        while done < L and t_sc < budget_s:
+            t0 = time.perf_counter()
+            oracle.mlp_token_scores(gate_bits=gate[done:done + chunk], up_bits=up[done:done + chunk])
+            t_sc += time.perf_counter() - t0
+            done += chunk
+        cu = np.array([0, L], dtype=np.int32)
+        x, y = synth.normal_bf16(L, d, 0, 7), synth.normal_bf16(L, d, 0, 8)
+        t0 = time.perf_counter()
+        bs = oracle.mlp_block_scores(np.linspace(1.0, 0.0, L), cu, b)  # costs do not depend on values
+        idx, _, _ = oracle.compact(oracle.keep_mask(bs, float(np.median(bs))), cu, b)
+        oracle.gather_pad(x, idx, PAD_TO)
+        oracle.scatter_residual(x, y, idx)
+        t_rest = time.perf_counter() - t0
+        return t_sc * L / done + t_rest, L, (
+            f"mlp-7b: token scores of {done} of {L} tokens ({t_sc:.1f} s) scaled by tokens; block "
+            f"scores, threshold, compaction, gather and scatter in full ({t_rest:.1f} s); float64 numpy")
+    if workload == "lmhead-7b":
+        cfg = synth.LM_HEAD_WORKLOADS["lmhead-7b"]
+        T, d, V = cfg["T"], cfg["d"], cfg["V"]
+        h, wt, y = synth.lm_head_inputs(T, d, V, cfg["seed"])
+        R = 64
+        t0 = time.perf_counter()
+        oracle.lm_head_loss(h[:R], wt, y[:R])
+        t = time.perf_counter() - t0
+        return t * T / R, T, (f"lmhead-7b: the oracle's full definition (logits, loss, dh and dW) on "
+                              f"the first {R} of {T} tokens ({t:.1f} s), scaled by tokens; float64 numpy")
+    raise ValueError(workload)
+
+
+def ext_cpu_baseline(workload: str, budget_s: float):
+    t, tokens, desc = oracle_sample(workload, budget_s)
+    return {"value": round(tokens / t, 3), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": desc, "seconds_per_layer_estimate": round(t, 2)}
+
+
+def run_reference_ext(args):
+    world, rank, local = dist_env()
+    if rank != 0:
+        return  # the reference arm runs on rank 0 only
+    per_step = max(0.3, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    vals, desc, tokens = [], "", 0
+    for i in range(args.warmup + args.steps):
+        t, tokens, d = oracle_sample(args.workload, per_step, seed=i)
+        if i >= args.warmup:
+            vals.append(t)
+            desc = d
+    t = statistics.fmean(vals)
+    value = tokens / t
+    metric = {"attn-c3": ATTN_METRIC, "predict-c5": PREDICT_METRIC, "mlp-7b": MLP_METRIC,
+              "lmhead-7b": SEGLOSS_METRIC}[args.workload]
+    out = {
+        "metric": metric, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t * 1e3, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": args.workload, "parallelism": "CPU oracle, rank 0 only"},
+        "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": blas_threads(),
+                         "kind": "oracle", "sample": f"per step: {desc}"},
+        "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
 def run_reference(args):
     world, rank, local = dist_env()
     if rank != 0:
@@ -1133,8 +1260,7 @@ def main(argv=None):
                   "predict-c5": run_predict, "mlp-7b": run_mlp}
     if args.workload in extensions:
         if args.impl == "reference":
-            print(json.dumps({"impl": "reference", "unavailable": "the oracle arm covers the "
-                              "per-layer path workloads only"}), flush=True)
+            run_reference_ext(args)
         else:
             extensions[args.workload](args)
     elif args.impl == "reference":
