@@ -227,20 +227,6 @@ __device__ __noinline__ bool wait_drain(uint64_t* bar, uint32_t parity, uint64_t
     return true;
 }
 
-// Non-blocking test of a phase (mbarrier.try_wait may suspend the thread
-// for a while; the MMA scheduler must move on to the other query tile).
-__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
 // wait() by every lane of the warp, with a warp-uniform result (the warp
 // then runs its collective tensor-memory instructions together or not at all).
 __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, Smem* sm,
