@@ -663,7 +663,7 @@ lemo_status lemo_mlp_block_scores(const lemo_shape* shape, int32_t d_ff, const u
     if (sms <= 0) return LEMO_ERR_CUDA;
     const int64_t ctas_needed =
         ((int64_t)shape->total_L + lemo::mlp::kThreads / 32 - 1) / (lemo::mlp::kThreads / 32);
-    const int64_t grid = ctas_needed < (int64_t)sms * 4 ? ctas_needed : (int64_t)sms * 4;
+    const int64_t grid = ctas_needed < (int64_t)sms * 2 ? ctas_needed : (int64_t)sms * 2;
     launch(lemo::mlp::block_scores_kernel, (unsigned)grid, lemo::mlp::kThreads, 0, st, a);
     return launch_status();
 }

@@ -4,8 +4,9 @@
 // a token block scores the maximum over its tokens (the block rule of Eq. 2).
 // The selection, gather and scatter kernels then apply unchanged.
 //
-// One warp per token row over a persistent grid, 16-byte loads with four in
-// flight per lane (HBM-bound); per-lane partial sums in a fixed order and a
+// One warp per token row over a persistent grid (two CTAs of 512 threads per
+// SM, 64 registers each), 16-byte loads with eight per operand in flight per
+// lane (HBM-bound); per-lane partial sums in a fixed order and a
 // fixed butterfly make each token score deterministic, and the block maximum
 // does not depend on the order its tokens finish.
 #pragma once
@@ -16,7 +17,7 @@ namespace lemo {
 namespace mlp {
 
 constexpr int kThreads = 512;
-constexpr int kUnroll = 4;
+constexpr int kUnroll = 8;
 
 __device__ __forceinline__ float pos_sum8(uint4 v) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -68,7 +69,7 @@ struct Args {
 // is the maximum of its tokens' scores; every score is >= 0, so the maxima
 // combine with an integer atomicMax on the float bit patterns (order does
 // not change a maximum: deterministic).  block_scores must be zeroed first.
-__global__ void __launch_bounds__(kThreads) block_scores_kernel(const Args a) {
+__global__ void __launch_bounds__(kThreads, 2) block_scores_kernel(const Args a) {
     pdl_entry();
     const PlanHeader* hdr = reinterpret_cast<const PlanHeader*>(a.ws + a.lay.hdr);
     if (!hdr->valid) return;
