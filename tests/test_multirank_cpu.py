@@ -62,3 +62,20 @@ def test_single_rank_is_identity():
     import bench
     assert bench.max_over_ranks(3.5, 1) == 3.5
     assert bench.whole_job_rate(100, 1, 2.0) == 50.0
+
+
+@pytest.mark.parametrize("workload", ["c3", "attn-c3", "lmhead-7b"])
+def test_reference_arm_other_ranks_exit_without_work(workload, monkeypatch, capsys):
+    """Under torchrun the reference arm runs on rank 0 only: any other rank
+    prints nothing and returns at once (no oracle work, no collective)."""
+    import time
+
+    import bench
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setenv("LOCAL_RANK", "1")
+    t0 = time.perf_counter()
+    bench.main(["--impl", "reference", "--gpus", "2", "--workload", workload, "--steps", "1",
+                "--warmup", "3"])
+    assert time.perf_counter() - t0 < 5.0
+    assert capsys.readouterr().out == ""
