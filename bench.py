@@ -1,7 +1,7 @@
 """Throughput of the contextual-token-sparsity hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lemo|reference]
-                    [--workload c3]
+                    [--workload llama7b-16k]
 
 One step is one pass of the whole path - block scores, threshold, compaction,
 gather, scatter with residual add - over every layer of the workload (default:
@@ -131,10 +131,10 @@ def score_source_digest() -> str:
 
 def profiled_traffic(workload: str):
     """DRAM bytes per scorer launch from the committed ncu summary
-    (profiles/score_tiles_*.md), if it was taken on the current scorer source
+    (profiles/score_tiles_llama7b.md), if it was taken on the current scorer source
     (else None)."""
-    path = os.path.join(ROOT, "profiles", "score_tiles_c2.md")
-    if workload != "c3" or not os.path.exists(path):
+    path = os.path.join(ROOT, "profiles", "score_tiles_llama7b.md")
+    if workload != "llama7b-16k" or not os.path.exists(path):
         return None
     rec = {}
     with open(path) as f:
@@ -562,7 +562,7 @@ def run_segloss(args):
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = ext_cpu_baseline("lmhead-7b", args.cpu_seconds)
+        out["cpu_baseline"] = ext_cpu_baseline("lmhead-llama7b-16k", args.cpu_seconds)
     if world > 1:
         import torch.distributed as dist
         dist.barrier(device_ids=[local])
@@ -685,7 +685,7 @@ def attention_flops(kept_per_seq, H, dh) -> float:
 
 
 def run_attention(args):
-    """Attention over the kept tokens of the three c3 layers (keep 30/50/70 %),
+    """Attention over the kept tokens of the three llama7b-16k layers (keep 30/50/70 %),
     added in place into the residual stream.  The keep masks come from the
     path itself (score + select at set-up, with the stored thresholds)."""
     import torch
@@ -696,12 +696,12 @@ def run_attention(args):
     world, rank, local = dist_env()
     dev, gpu_id = _setup_device(world, local)
     lemo.load()
-    key = "c3"
+    key = "llama7b-16k"
     w = synth.WORKLOADS[key]
     nl = w.layers
     thetas = thresholds(key, nl)
     if thetas is None:
-        raise RuntimeError("stored thresholds tests/golden/c3.json are missing")
+        raise RuntimeError("stored thresholds tests/golden/llama7b-16k.json are missing")
     hd = w.H * w.dh
     host = []
     for l in range(nl):
@@ -755,8 +755,8 @@ def run_attention(args):
     tot_f = sum(flops)
     tot_ach = tot_f / (sum(per_layer_us) * 1e-6) / 1e12
     out = _header(ATTN_METRIC, args, world, step_s, whole_job_rate(nl * w.total_L, world, step_s))
-    out["config"] = {"workload": f"attn-c3: attention over the kept tokens of the {key} layers "
-                                 f"(L={w.total_L}, H={w.H}, dh={w.dh}, b={w.block}, keep "
+    out["config"] = {"workload": f"attn-llama7b-16k: attention over the kept tokens of the {key} "
+                                 f"layers (L={w.total_L}, H={w.H}, dh={w.dh}, b={w.block}, keep "
                                  f"30/50/70%), output added into the residual in place",
                      "layers": nl, "kept_tokens": kept, "softmax_scale": "1/sqrt(dh)",
                      "l2": "not flushed; each step reads 3 x 3 x 134 MB of Q/K/V rows "
@@ -788,12 +788,12 @@ def run_attention(args):
                           [(dx, hx_out)],
                           lambda: call(dx.view(torch.bfloat16), bf(dq), bf(dk), bf(dv)))
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = ext_cpu_baseline("attn-c3", args.cpu_seconds)
+        out["cpu_baseline"] = ext_cpu_baseline("attn-llama7b-16k", args.cpu_seconds)
     _finish(out, world, local, rank)
 
 
 def run_predict(args):
-    """The predicted path at the Llama-2-13B layer (c5): block means of X,
+    """The predicted path at the Llama-2-13B layer (llama13b-32k): block means of X,
     the two rank-256 ReLU predictors (pruned neurons left out: rank 154),
     block products and column sums, then select / gather / scatter with the
     stored predicted-score threshold."""
@@ -805,12 +805,12 @@ def run_predict(args):
     world, rank, local = dist_env()
     dev, gpu_id = _setup_device(world, local)
     lemo.load()
-    key = "c5"
+    key = "llama13b-32k"
     w = synth.WORKLOADS[key]
     seed = int(w.seeds[0])
     path = os.path.join(ROOT, "tests", "golden", f"{key}.json")
     if not os.path.exists(path):
-        raise RuntimeError("stored thresholds tests/golden/c5.json are missing")
+        raise RuntimeError("stored thresholds tests/golden/llama13b-32k.json are missing")
     with open(path) as f:
         theta = float(json.load(f)["layers"][0]["pred_theta"])
     L, d, hd = w.total_L, w.d, w.H * w.dh
@@ -865,7 +865,7 @@ def run_predict(args):
     pred_flops = 2 * 2 * tb * (d * rank_eff + rank_eff * hd) + tb * (tb + 1) * hd
     bw = peaks["hbm_gbs"]
     out = _header(PREDICT_METRIC, args, world, step_s, whole_job_rate(L, world, step_s))
-    out["config"] = {"workload": f"predict-c5: {w.name}", "seq_lens": list(w.lengths),
+    out["config"] = {"workload": f"predict-llama13b-32k: {w.name}", "seq_lens": list(w.lengths),
                      "heads": w.H, "head_dim": w.dh, "block": w.block, "d": d,
                      "predictor_rank": w.predictor_rank, "live_neurons": [len(liveq), len(livek)],
                      "keep": 0.5, "kept_tokens": K, "threshold_source":
@@ -898,7 +898,7 @@ def run_predict(args):
                           [(hxp, dx), (hyp, dy)], [(dx, hx_out), (layer.block_scores, hs)],
                           lambda: call(dx.view(torch.bfloat16), dy.view(torch.bfloat16)))
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = ext_cpu_baseline("predict-c5", args.cpu_seconds)
+        out["cpu_baseline"] = ext_cpu_baseline("predict-llama13b-32k", args.cpu_seconds)
     _finish(out, world, local, rank)
 
 
@@ -963,7 +963,7 @@ def run_mlp(args):
     gbs = score_bytes / (us["mlp_score"] * 1e-6) / 1e9
     g_b, s_b = move_bytes(K, d)
     out = _header(MLP_METRIC, args, world, step_s, whole_job_rate(L, world, step_s))
-    out["config"] = {"workload": f"mlp-7b: L={L}, SiLU-gated d_ff={d_ff}, b={b}, d={d}, "
+    out["config"] = {"workload": f"mlp-llama7b-16k: L={L}, SiLU-gated d_ff={d_ff}, b={b}, d={d}, "
                                  "keep 50%", "kept_tokens": K,
                      "threshold_source": "keep ratio on the kernel's own block scores",
                      "l2": "not flushed; each step reads 721 MB of activations (> 126 MB L2)",
@@ -987,7 +987,7 @@ def run_mlp(args):
                           list(zip((hg, hu, hxp, hyp), dd)), [(dd[2], hx_out)],
                           lambda: call(*[t.view(torch.bfloat16) for t in dd]))
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = ext_cpu_baseline("mlp-7b", args.cpu_seconds)
+        out["cpu_baseline"] = ext_cpu_baseline("mlp-llama7b-16k", args.cpu_seconds)
     _finish(out, world, local, rank)
 
 
@@ -1091,10 +1091,10 @@ def oracle_sample(workload: str, budget_s: float = 20.0, seed: int = 0):
     import oracle
     from contextual_token_sparsity_b200 import synth
     rng = np.random.default_rng(seed)
-    if workload == "predict-c5":
-        w = synth.WORKLOADS["c5"]
+    if workload == "predict-llama13b-32k":
+        w = synth.WORKLOADS["llama13b-32k"]
         sd, L, d, hd = int(w.seeds[0]), w.total_L, w.d, w.H * w.dh
-        with open(os.path.join(ROOT, "tests", "golden", "c5.json")) as f:
+        with open(os.path.join(ROOT, "tests", "golden", "llama13b-32k.json")) as f:
             theta = float(json.load(f)["layers"][0]["pred_theta"])
         xb, _ = synth.projected_x(L, d, float(w.salient), sd)
         w1q, w2q, lq = synth.predictor_weights(d, w.predictor_rank, hd, 0.4, sd, 10)
@@ -1110,13 +1110,13 @@ def oracle_sample(workload: str, budget_s: float = 20.0, seed: int = 0):
         oracle.gather_pad(xb, idx, PAD_TO)
         oracle.scatter_residual(xb, y, idx)
         t = time.perf_counter() - t0
-        return t, L, (f"predict-c5 in full ({t:.1f} s): block means, both predictors, Eq. 3 block "
-                      "products, threshold, compaction, gather and scatter; float64 numpy")
-    if workload == "attn-c3":
-        w = synth.WORKLOADS["c3"]
-        with open(os.path.join(ROOT, "tests", "golden", "c3.json")) as f:
+        return t, L, (f"predict-llama13b-32k in full ({t:.1f} s): block means, both predictors, "
+                      "Eq. 3 block products, threshold, compaction, gather and scatter; float64 numpy")
+    if workload == "attn-llama7b-16k":
+        w = synth.WORKLOADS["llama7b-16k"]
+        with open(os.path.join(ROOT, "tests", "golden", "llama7b-16k.json")) as f:
             g = json.load(f)["layers"][1]
-        inp = synth.make_workload("c3", 1, with_x=False)
+        inp = synth.make_workload("llama7b-16k", 1, with_x=False)
         hd = w.H * w.dh
         v = synth.normal_bf16(w.total_L, hd, int(w.seeds[1]), 22)
         mask = oracle.keep_mask(np.array([float(x) for x in g["scores"]]), float(g["theta"]))
@@ -1133,9 +1133,9 @@ def oracle_sample(workload: str, budget_s: float = 20.0, seed: int = 0):
         t = time.perf_counter() - t0
         all_pairs = K * (K + 1) // 2
         return t * all_pairs / pairs, w.total_L, (
-            f"layer 1 of attn-c3 (K = {K}): {rows} of {K} query rows ({pairs} of {all_pairs} "
-            f"query-key pairs, {t:.1f} s) by the oracle, scaled by pairs; float64 numpy")
-    if workload == "mlp-7b":
+            f"layer 1 of attn-llama7b-16k (K = {K}): {rows} of {K} query rows "
+            f"({pairs} of {all_pairs} query-key pairs, {t:.1f} s) by the oracle, scaled by pairs; float64 numpy")
+    if workload == "mlp-llama7b-16k":
         L, d_ff, d, b = 16384, 11008, 4096, 64
         gate, up = synth.mlp_activations(L, d_ff, 0.1, seed=0, gated=True)
         chunk, t_sc, done = 512, 0.0, 0
@@ -1153,18 +1153,18 @@ def oracle_sample(workload: str, budget_s: float = 20.0, seed: int = 0):
         oracle.scatter_residual(x, y, idx)
         t_rest = time.perf_counter() - t0
         return t_sc * L / done + t_rest, L, (
-            f"mlp-7b: token scores of {done} of {L} tokens ({t_sc:.1f} s) scaled by tokens; block "
-            f"scores, threshold, compaction, gather and scatter in full ({t_rest:.1f} s); float64 numpy")
-    if workload == "lmhead-7b":
-        cfg = synth.LM_HEAD_WORKLOADS["lmhead-7b"]
+            f"mlp-llama7b-16k: token scores of {done} of {L} tokens ({t_sc:.1f} s) scaled by "
+            f"tokens; block scores, threshold, compaction, gather and scatter in full ({t_rest:.1f} s); float64 numpy")
+    if workload == "lmhead-llama7b-16k":
+        cfg = synth.LM_HEAD_WORKLOADS["lmhead-llama7b-16k"]
         T, d, V = cfg["T"], cfg["d"], cfg["V"]
         h, wt, y = synth.lm_head_inputs(T, d, V, cfg["seed"])
         R = 64
         t0 = time.perf_counter()
         oracle.lm_head_loss(h[:R], wt, y[:R])
         t = time.perf_counter() - t0
-        return t * T / R, T, (f"lmhead-7b: the oracle's full definition (logits, loss, dh and dW) on "
-                              f"the first {R} of {T} tokens ({t:.1f} s), scaled by tokens; float64 numpy")
+        return t * T / R, T, (f"lmhead-llama7b-16k: the oracle's full definition (logits, loss, "
+                              f"dh and dW) on the first {R} of {T} tokens ({t:.1f} s), scaled by tokens; float64 numpy")
     raise ValueError(workload)
 
 
@@ -1187,8 +1187,8 @@ def run_reference_ext(args):
             desc = d
     t = statistics.fmean(vals)
     value = tokens / t
-    metric = {"attn-c3": ATTN_METRIC, "predict-c5": PREDICT_METRIC, "mlp-7b": MLP_METRIC,
-              "lmhead-7b": SEGLOSS_METRIC}[args.workload]
+    metric = {"attn-llama7b-16k": ATTN_METRIC, "predict-llama13b-32k": PREDICT_METRIC,
+              "mlp-llama7b-16k": MLP_METRIC, "lmhead-llama7b-16k": SEGLOSS_METRIC}[args.workload]
     out = {
         "metric": metric, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t * 1e3, 1),
@@ -1243,9 +1243,10 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["lemo", "reference"], default="lemo")
-    ap.add_argument("--workload", default="c3",
-                    choices=["c1", "c2", "c3", "c4", "c5", "lmhead-7b", "attn-c3",
-                             "predict-c5", "mlp-7b"])
+    ap.add_argument("--workload", default="llama7b-16k",
+                    choices=["small-1k", "llama7b-8k", "llama7b-16k", "varlen-10k", "llama13b-32k",
+                             "lmhead-llama7b-16k", "attn-llama7b-16k", "predict-llama13b-32k",
+                             "mlp-llama7b-16k"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -1256,8 +1257,8 @@ def main(argv=None):
     world = dist_env()[0]
     if args.gpus != world and world > 1:
         ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}")
-    extensions = {"lmhead-7b": run_segloss, "attn-c3": run_attention,
-                  "predict-c5": run_predict, "mlp-7b": run_mlp}
+    extensions = {"lmhead-llama7b-16k": run_segloss, "attn-llama7b-16k": run_attention,
+                  "predict-llama13b-32k": run_predict, "mlp-llama7b-16k": run_mlp}
     if args.workload in extensions:
         if args.impl == "reference":
             run_reference_ext(args)

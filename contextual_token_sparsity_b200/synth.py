@@ -190,7 +190,7 @@ def lm_head_inputs(T: int, d: int, V: int, seed: int, logit_std: float = 2.0,
 # Segmented lm-head loss at the Llama-2-7B head (d = 4096, V = 32000) over
 # the 16384 tokens of one long sequence, 16 segments of 1024 tokens.
 LM_HEAD_WORKLOADS = {
-    "lmhead-7b": dict(T=16384, d=4096, V=32000, seg_rows=1024, seed=0),
+    "lmhead-llama7b-16k": dict(T=16384, d=4096, V=32000, seg_rows=1024, seed=0),
 }
 
 
@@ -219,16 +219,17 @@ class Workload:
 
 
 WORKLOADS = {
-    "c1": Workload("single layer L=1024 d=512 H=8 dh=64 b=64", (1024,), 512, 8, 64, 64,
+    "small-1k": Workload("single layer L=1024 d=512 H=8 dh=64 b=64", (1024,), 512, 8, 64, 64,
                    (0.5,), (0,), "projected"),
-    "c2": Workload("llama2-7b layer L=8192 d=4096 H=32 dh=128 b=64 keep 50%", (8192,), 4096,
-                   32, 128, 64, (0.5,), (0,), "direct"),
-    "c3": Workload("llama2-7b layers L=16384 d=4096 H=32 dh=128 b=64 keep 30/50/70%",
+    "llama7b-8k": Workload("llama2-7b layer L=8192 d=4096 H=32 dh=128 b=64 keep 50%", (8192,),
+                           4096, 32, 128, 64, (0.5,), (0,), "direct"),
+    "llama7b-16k": Workload("llama2-7b layers L=16384 d=4096 H=32 dh=128 b=64 keep 30/50/70%",
                    (16384,), 4096, 32, 128, 64, (0.3, 0.5, 0.7), (0, 1, 2), "direct"),
-    "c4": Workload("varlen L={4096,3072,2048,1024} d=4096 H=32 dh=128 b=64 keep 50%",
+    "varlen-10k": Workload("varlen L={4096,3072,2048,1024} d=4096 H=32 dh=128 b=64 keep 50%",
                    (4096, 3072, 2048, 1024), 4096, 32, 128, 64, (0.5,), (0,), "direct",
                    salient="uniform-5-20"),
-    "c5": Workload("llama2-13b layer L=32768 d=5120 H=40 dh=128 b=128 keep 50% + predictor",
+    "llama13b-32k": Workload("llama2-13b layer L=32768 d=5120 H=40 dh=128 b=128 keep 50% "
+                             "+ predictor",
                    (32768,), 5120, 40, 128, 128, (0.5,), (0,), "projected",
                    predictor_rank=256),
 }

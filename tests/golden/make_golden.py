@@ -1,6 +1,6 @@
 """Write the stored expected values of the full-size workloads.
 
-    python tests/golden/make_golden.py [c2 c3 c4 c5]
+    python tests/golden/make_golden.py [llama7b-8k llama7b-16k varlen-10k llama13b-32k]
 
 Calls only the CPU oracle (``oracle/``) and the seeded input generators
 (``contextual_token_sparsity_b200.synth``); nothing here touches the GPU
@@ -72,4 +72,4 @@ def main(keys):
 
 
 if __name__ == "__main__":
-    main(sys.argv[1:] or ["c2", "c4", "c3", "c5"])
+    main(sys.argv[1:] or ["llama7b-8k", "varlen-10k", "llama7b-16k", "llama13b-32k"])

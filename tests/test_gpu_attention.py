@@ -181,13 +181,13 @@ def test_non_block_kept_set_is_reported():
     assert st == lemo.LEMO_ERR_INVALID_ARG
 
 
-def test_c3_layer_sampled_rows():
+def test_llama7b_16k_layer_sampled_rows():
     """Llama-2-7B layer shape (L = 16384, H = 32, dh = 128, b = 64) with the
-    c3 layer-1 keep mask (50 %): sampled kept rows against the oracle."""
+    llama7b-16k layer-1 keep mask (50 %): sampled kept rows against the oracle."""
     import json
     import os
     L, H, dh, b = 16384, 32, 128, 64
-    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "c3.json")
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "llama7b-16k.json")
     with open(path) as f:
         g = json.load(f)["layers"][1]
     mask = oracle.keep_mask(np.array([float(s) for s in g["scores"]]), float(g["theta"]))

@@ -41,7 +41,8 @@ def _golden(key):
         return json.load(f)
 
 
-CASES = [("c2", 0), ("c4", 0), ("c3", 0), ("c3", 1), ("c3", 2), ("c5", 0)]
+CASES = [("llama7b-8k", 0), ("varlen-10k", 0), ("llama7b-16k", 0), ("llama7b-16k", 1),
+         ("llama7b-16k", 2), ("llama13b-32k", 0)]
 
 
 @pytest.mark.parametrize("key,layer", CASES, ids=[f"{k}-layer{l}" for k, l in CASES])

@@ -110,10 +110,10 @@ def test_keep_all_and_none(theta, expect):
     check_movement(res, cu, b, x, y, 128)
 
 
-def test_config_c1_full():
+def test_small_1k_full():
     """Single layer L=1024, d=512, H=8, dh=64, b=64, projected Q/K, 50th pct."""
-    w = synth.WORKLOADS["c1"]
-    inp = synth.make_workload("c1")
+    w = synth.WORKLOADS["small-1k"]
+    inp = synth.make_workload("small-1k")
     cu = inp["cu_seqlens"]
     s_ref = oracle.column_scores(oracle.score_blocks(inp["q"], inp["k"], cu, w.H, w.dh, w.block))
     theta = oracle.threshold_for_keep_ratio(s_ref, 0.5)

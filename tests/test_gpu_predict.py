@@ -105,8 +105,8 @@ def test_pruned_neurons_can_be_left_out():
     np.testing.assert_allclose(compact, full, rtol=1e-5, atol=1e-6 * np.abs(full).max())
 
 
-def test_predictor_workload_c5_against_stored_oracle():
-    key = "c5"
+def test_predictor_llama13b_32k_against_stored_oracle():
+    key = "llama13b-32k"
     path = os.path.join(GOLDEN, f"{key}.json")
     if not os.path.exists(path):
         pytest.skip("no stored oracle values")
@@ -121,7 +121,7 @@ def test_predictor_workload_c5_against_stored_oracle():
     assert synth.digest(w1q, w2q, w1k, w2k) == g["digest_pred"]
     got, cu = run_predict(list(w.lengths), w.H, w.dh, w.block, x, w1q, w2q, w1k, w2k)
     want = np.array([float(v) for v in g["pred_scores"]])
-    assert_scores_close(got, want, "predicted scores c5")
+    assert_scores_close(got, want, "predicted scores llama13b-32k")
     ptheta = float(g["pred_theta"])
     mask_gpu = oracle.keep_mask(got.astype(np.float32), np.float32(ptheta))
     band = np.abs(want - ptheta) <= BAND * abs(ptheta)

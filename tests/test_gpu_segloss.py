@@ -161,7 +161,7 @@ def test_lmhead_7b_workload_sampled_rows():
     """Llama-2-7B head over 16384 tokens in 16 segments: sampled token rows
     against the oracle row by row, the loss against the mean of the token
     terms, and sum_v dW[v, :] = 0 (rows of dz sum to zero)."""
-    cfg = synth.LM_HEAD_WORKLOADS["lmhead-7b"]
+    cfg = synth.LM_HEAD_WORKLOADS["lmhead-llama7b-16k"]
     T, d, V, S = cfg["T"], cfg["d"], cfg["V"], cfg["seg_rows"]
     h, w, y = synth.lm_head_inputs(T, d, V, cfg["seed"])
     got = run(h, w, y, S)

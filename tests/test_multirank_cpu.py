@@ -64,7 +64,7 @@ def test_single_rank_is_identity():
     assert bench.whole_job_rate(100, 1, 2.0) == 50.0
 
 
-@pytest.mark.parametrize("workload", ["c3", "attn-c3", "lmhead-7b"])
+@pytest.mark.parametrize("workload", ["llama7b-16k", "attn-llama7b-16k", "lmhead-llama7b-16k"])
 def test_reference_arm_other_ranks_exit_without_work(workload, monkeypatch, capsys):
     """Under torchrun the reference arm runs on rank 0 only: any other rank
     prints nothing and returns at once (no oracle work, no collective)."""
