@@ -166,18 +166,26 @@ def thresholds(key: str, layers: int):
 # ----------------------------------------------------------------------------
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples of one GPU (every 100 ms)."""
+    """Clock, power and throttle-reason samples of one GPU while a timed
+    region runs: NVML polled from a thread every 10 ms (read-only queries),
+    or nvidia-smi every 100 ms where NVML cannot be loaded."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+    PERIOD_S = 0.01
 
     def __init__(self, index):
-        self.index = index  # nvidia-smi id: a GPU UUID or an index
+        self.index = index  # a GPU UUID ("GPU-...") or an index
         self.proc = None
+        self.nv = None
+        self.rows = []
         self.path = os.path.join("/tmp", f"lemo_clocks_{os.getpid()}_{index}.csv")
 
     def start(self):
+        if self._start_nvml():
+            return
         try:
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
@@ -187,7 +195,48 @@ class ClockSampler:
         except OSError:
             self.proc = None
 
+    def _start_nvml(self) -> bool:
+        import threading
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+        except Exception:
+            return False
+        try:
+            idx = str(self.index)
+            h = (nv.nvmlDeviceGetHandleByUUID(idx) if idx.startswith("GPU-")
+                 else nv.nvmlDeviceGetHandleByIndex(int(idx)))
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+        except Exception:
+            nv.nvmlShutdown()
+            return False
+        self.nv, self.h = nv, h
+        self.bits = (nv.nvmlClocksEventReasonHwSlowdown, nv.nvmlClocksEventReasonHwThermalSlowdown,
+                     nv.nvmlClocksEventReasonSwThermalSlowdown, nv.nvmlClocksEventReasonSwPowerCap)
+        self.halt = threading.Event()
+        self.thread = threading.Thread(target=self._poll, daemon=True)
+        self.thread.start()
+        return True
+
+    def _poll(self):
+        nv, h = self.nv, self.h
+        while not self.halt.is_set():
+            try:
+                sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.rows.append((sm, self.max_mhz, pw,
+                                  [self.REASONS[i] for i, b in enumerate(self.bits) if rs & b]))
+            except Exception:
+                pass
+            self.halt.wait(self.PERIOD_S)
+
     def stop(self):
+        if self.nv is not None:
+            self.halt.set()
+            self.thread.join(timeout=5)
+            self.nv.nvmlShutdown()
+            return self.summary(self.rows, "nvml")
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -206,24 +255,33 @@ class ClockSampler:
             os.remove(self.path)
         except OSError:
             pass
-        if not rows:
-            return None
+        return self.summary([self.parse_smi(r) for r in rows], "nvidia-smi")
 
+    @classmethod
+    def parse_smi(cls, r):
+        """One nvidia-smi CSV row -> (sm MHz, max MHz, power W, active reasons)."""
         def num(v):
             try:
                 return float(v)
             except ValueError:
                 return float("nan")
-        sm = [num(r[0]) for r in rows]
-        mx = [num(r[1]) for r in rows]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower() == "active"})
-        loaded = [s for s in sm if not math.isnan(s)]
-        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+        return (num(r[0]), num(r[1]), num(r[2]),
+                [cls.REASONS[i] for i in range(4) if r[4 + i].lower() == "active"])
+
+    @staticmethod
+    def summary(rows, source):
+        if not rows:
+            return None
+        sm = [r[0] for r in rows if not math.isnan(r[0])]
+        mx = [r[1] for r in rows if not math.isnan(r[1])]
+        pw = [r[2] for r in rows if not math.isnan(r[2])]
+        return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(mx) if mx else None,
                 "samples": len(rows),
-                "power_w_max": max(num(r[2]) for r in rows),
-                "reasons": reasons}
+                "power_w_median": statistics.median(pw) if pw else None,
+                "power_w_max": max(pw) if pw else None,
+                "reasons": sorted({x for r in rows for x in r[3]}),
+                "source": source}
 
 
 # ----------------------------------------------------------------------------

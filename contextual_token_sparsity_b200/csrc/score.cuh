@@ -18,15 +18,18 @@
 //                            overlaps the read-out of head h; commits are
 //                            multicast to both CTAs;
 //   epilogue (8 warps)       tcgen05.ld pulls S^h into registers and folds it
-//                            into the running sum A += max(S^h, 0) (128 fp32
-//                            per thread; max on the min/max unit, the adds as
-//                            packed fp32x2), then frees the accumulator on the
-//                            leader's barrier.
+//                            into the running sum 2A += S^h + |S^h| (128 fp32
+//                            per thread; s + |s| is exactly 2 max(s, 0), and
+//                            both adds are packed fp32x2, so no instruction
+//                            runs on the half-rate min/max unit), then frees
+//                            the accumulator on the leader's barrier.
 //
 // After the last head the epilogue applies the causal mask (j < i, rows
-// inside the sequence), takes the maximum of A over each b x b block and
-// writes M[n][m] = max * scale / H.  S is never written to memory.  A second
-// small kernel sums M's columns in a fixed order (deterministic).
+// inside the sequence), takes the maximum of 2A over each b x b block and
+// writes M[n][m] = max * (scale / H) / 2.  Doubling every addend doubles
+// every rounded partial sum, so M has the same bits as summing max(S^h, 0)
+// directly.  S is never written to memory.  A second small kernel sums M's
+// columns in a fixed order (deterministic).
 //
 // Splitting the key operand across the pair cuts the bytes each SM loads per
 // head from 96 KB (one-SM 128 x 256 tile) to 64 KB, and loading a whole head
@@ -34,9 +37,13 @@
 // MMA fed.  Ten warps per CTA (not more) leave 168 registers per thread for
 // the 128 running sums.  No TMA load uses multicast.
 //
-// Sustained, the kernel runs at the board's power limit, so fewer issued
-// instructions per score element (about 2.4, 1.5 of them arithmetic) turn
-// directly into speed.
+// One 256 x 256 x 16 MMA keeps the tensor pipe busy for ~137 cycles and the
+// pipe queues only about two of them, so the issuing thread tests the
+// barriers of the next head while the last MMAs of the current one are
+// queued (blocking only when they are not complete) instead of leaving the
+// pipe idle between heads.  Sustained, the kernel runs at the board's power
+// limit, so fewer issued instructions per score element turn directly into
+// speed.
 //
 // Every mbarrier wait is bounded in time; a wait that runs out records
 // LEMO_ERR_TIMEOUT and makes both CTAs of the pair drain what they issued,
@@ -273,6 +280,58 @@ __device__ __forceinline__ void add_f32x2(float& a0, float& a1, float b0, float 
         : "f"(b0), "f"(b1));
 }
 
+// MMAs k = K0 .. K1-1 of one head (16 bf16 of K each): 16 bf16 (32 bytes)
+// along K inside a swizzle row, every 4 steps the next 16 KB slice.
+template <int K0, int K1>
+__device__ __forceinline__ void issue_mmas(uint32_t d_tmem, uint64_t da, uint64_t db) {
+#pragma unroll
+    for (int k = K0; k < K1; ++k) {
+        const uint64_t off = (uint64_t)((k >> 2) * (KB_BYTES >> 4) + (k & 3) * 2);
+        umma_bf16_pair(d_tmem, da + off, db + off, k > 0 ? 1u : 0u);
+    }
+}
+
+// Whether the phases with parities p0 of b0 and p1 of b1 are both complete.
+// test_wait never suspends the thread, so both tests are in flight together.
+__device__ __forceinline__ bool mbar_test_wait2(uint64_t* b0, uint32_t p0, uint64_t* b1,
+                                                uint32_t p1) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred q0, q1, q;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 q0, [%1], %2;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 q1, [%3], %4;\n\t"
+        "and.pred q, q0, q1;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(b0)), "r"(p0), "r"(smem_u32(b1)), "r"(p1)
+        : "memory");
+    return ok != 0;
+}
+
+// Whether both barriers the issuer waits on before head g are complete
+// (never blocks).
+__device__ __forceinline__ bool head_ready(Smem* sm, uint32_t g) {
+    return mbar_test_wait2(&sm->acc_empty[g & 1], ((g >> 1) & 1) ^ 1, &sm->full[g % STAGES],
+                           (g / STAGES) & 1);
+}
+
+// The issuer's two waits before head g: accumulator g & 1 drained by both
+// epilogues, stage g % STAGES loaded by both producers.
+__device__ __forceinline__ bool wait_head(Smem* sm, uint32_t g, uint64_t limit_ns) {
+    uint64_t* ae = &sm->acc_empty[g & 1];
+    uint64_t* fu = &sm->full[g % STAGES];
+    const uint32_t pae = ((g >> 1) & 1) ^ 1, pfu = (g / STAGES) & 1;
+    if (mbar_test_wait2(ae, pae, fu, pfu)) return true;
+    return mbar_wait_slow(ae, pae, sm, limit_ns) && mbar_wait(fu, pfu, sm, limit_ns);
+}
+
+// max(a, b, c) in one three-input min/max instruction.
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 struct TileCoord {
     int seq;
     int qi, kj;
@@ -373,37 +432,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
+        // Heads are issued back to back over all tiles of the pair (the MMAs
+        // need no tile coordinates).  The tensor pipe queues only about two
+        // MMAs, so the barriers of head g + 1 are tested (without blocking)
+        // while the last MMAs of head g are queued; only when they are not
+        // complete yet does the thread block on them, after its commits.
         if (lane == 0 && leader) {
-            uint32_t it = 0, acc_it = 0;
-            bool ok = true;
-            for (int64_t t = pair; ok && t < total_tiles; t += npairs) {
-                for (int h = 0; ok && h < a.H; ++h, ++acc_it) {
-                    const uint32_t buf = acc_it & 1, aph = (acc_it >> 1) & 1;
-                    if (!mbar_wait(&sm->acc_empty[buf], aph ^ 1, sm, a.spin_limit_ns)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t d_tmem = tmem_base + buf * ACC_COLS;
-                    const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
-                    if (!mbar_wait(&sm->full[s], ph, sm, a.spin_limit_ns)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t sa = smem_u32(tiles + s * STAGE_BYTES);
-                    const uint64_t da = sdesc_sw128(sa);
-                    const uint64_t db = sdesc_sw128(sa + A_BYTES);
-                    for (int k = 0; k < a.dh / UMMA_K; ++k) {
-                        // 16 bf16 (32 bytes) along K inside a swizzle row; every 4 steps
-                        // move on to the next 16 KB slice
-                        const uint64_t off = (uint64_t)((k >> 2) * (KB_BYTES >> 4) + (k & 3) * 2);
-                        umma_bf16_pair(d_tmem, da + off, db + off, k > 0 ? 1u : 0u);
-                    }
-                    umma_commit_pair(&sm->empty[s]);  // both CTAs' stage s is free again
-                    ++it;
-                    umma_commit_pair(&sm->acc_full[buf]);  // both CTAs' accumulators are ready
+            const int64_t my_tiles = (total_tiles - pair + npairs - 1) / npairs;
+            const uint32_t heads = (uint32_t)(my_tiles * a.H);
+            bool ok = heads > 0 && wait_head(sm, 0, a.spin_limit_ns);
+            for (uint32_t g = 0; ok && g < heads; ++g) {
+                const uint32_t buf = g & 1, s = g % STAGES;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + buf * ACC_COLS;
+                const uint32_t sa = smem_u32(tiles + s * STAGE_BYTES);
+                const uint64_t da = sdesc_sw128(sa);
+                const uint64_t db = sdesc_sw128(sa + A_BYTES);
+                const bool more = g + 1 < heads;
+                bool ready = false;
+                if (a.dh == 128) {  // head dimensions 64 and 128 are accepted
+                    issue_mmas<0, 4>(d_tmem, da, db);
+                    ready = more && head_ready(sm, g + 1);
+                    issue_mmas<4, 8>(d_tmem, da, db);
+                } else {
+                    issue_mmas<0, 2>(d_tmem, da, db);
+                    ready = more && head_ready(sm, g + 1);
+                    issue_mmas<2, 4>(d_tmem, da, db);
                 }
+                umma_commit_pair(&sm->empty[s]);       // both CTAs' stage s is free again
+                umma_commit_pair(&sm->acc_full[buf]);  // both CTAs' accumulators are ready
+                if (more && !ready) ok = wait_head(sm, g + 1, a.spin_limit_ns);
             }
             // Every MMA completes before either CTA releases its tensor memory.
             umma_commit_pair(&sm->done);
@@ -448,7 +506,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 #pragma unroll
                     for (int j = 0; j < 32; j += 2) {
                         const float s0 = __uint_as_float(r[j]), s1 = __uint_as_float(r[j + 1]);
-                        add_f32x2(acc[ch + j], acc[ch + j + 1], fmaxf(s0, 0.f), fmaxf(s1, 0.f));
+                        float t0 = s0, t1 = s1;
+                        add_f32x2(t0, t1, fabsf(s0), fabsf(s1));  // 2 max(s, 0), exactly
+                        add_f32x2(acc[ch + j], acc[ch + j + 1], t0, t1);
                     }
                 }
                 tc_fence_before();
@@ -468,8 +528,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             const int col0 = c.kj * TN + colhalf * COLS_PER_THREAD;
             const int jlim = (i_loc < c.L) ? (i_loc - col0) : 0;  // local cols < jlim are valid
             float mx[2] = {0.f, 0.f};
+            if (jlim >= COLS_PER_THREAD) {  // every column of this thread's slice is valid
 #pragma unroll
-            for (int j = 0; j < COLS_PER_THREAD; ++j) mx[j / 64] = fmaxf(mx[j / 64], (j < jlim) ? acc[j] : 0.f);
+                for (int g = 0; g < 2; ++g) {
+                    float m0 = 0.f, m1 = 0.f;
+#pragma unroll
+                    for (int j = g * 64; j < g * 64 + 64; j += 4) {
+                        m0 = max3(m0, acc[j], acc[j + 1]);
+                        m1 = max3(m1, acc[j + 2], acc[j + 3]);
+                    }
+                    mx[g] = fmaxf(m0, m1);
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < COLS_PER_THREAD; ++j)
+                    mx[j / 64] = fmaxf(mx[j / 64], (j < jlim) ? acc[j] : 0.f);
+            }
 #pragma unroll
             for (int g = 0; g < 2; ++g)
 #pragma unroll
@@ -491,7 +565,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     const float v = fmaxf(sm->red[tile_par][2 * qb][kslot],
                                           sm->red[tile_par][2 * qb + 1][kslot]);
                     const int n = row0 / 64 + qb, m = c.kj * (TN / 64) + kslot;
-                    if (n < nb && m <= n) M[(int64_t)n * nb + m] = v * a.out_scale;
+                    if (n < nb && m <= n) M[(int64_t)n * nb + m] = v * (0.5f * a.out_scale);
                 }
             } else {  // block == 128: 1 query block x 2 key blocks
                 if (etid < 2) {
@@ -501,7 +575,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                         v = fmaxf(v, fmaxf(sm->red[tile_par][qq][etid * 2],
                                            sm->red[tile_par][qq][etid * 2 + 1]));
                     const int n = row0 / 128, m = c.kj * (TN / 128) + etid;
-                    if (n < nb && m <= n) M[(int64_t)n * nb + m] = v * a.out_scale;
+                    if (n < nb && m <= n) M[(int64_t)n * nb + m] = v * (0.5f * a.out_scale);
                 }
             }
         }

@@ -79,3 +79,16 @@ def test_reference_arm_other_ranks_exit_without_work(workload, monkeypatch, caps
                 "--warmup", "3"])
     assert time.perf_counter() - t0 < 5.0
     assert capsys.readouterr().out == ""
+
+
+def test_clock_summary_reports_load_clocks_and_reasons():
+    """The clock record of a bench line: median SM clock, the maximum, power
+    and every throttle reason seen in any sample (nvidia-smi rows parsed)."""
+    import bench
+    rows = [["1965", "1965", "410.0", "0x0", "Not Active", "Not Active", "Not Active", "Not Active"],
+            ["1500", "1965", "990.5", "0x4", "Not Active", "Not Active", "Not Active", "Active"],
+            ["1450", "1965", "995.0", "0x4", "Not Active", "Not Active", "Not Active", "Active"]]
+    s = bench.ClockSampler.summary([bench.ClockSampler.parse_smi(r) for r in rows], "nvidia-smi")
+    assert s["sm_mhz"] == 1500 and s["sm_max_mhz"] == 1965 and s["samples"] == 3
+    assert s["power_w_max"] == 995.0 and s["reasons"] == ["sw_power_cap"]
+    assert bench.ClockSampler.summary([], "nvml") is None
