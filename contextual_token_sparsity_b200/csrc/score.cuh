@@ -38,12 +38,13 @@
 // the 128 running sums.  No TMA load uses multicast.
 //
 // One 256 x 256 x 16 MMA keeps the tensor pipe busy for ~137 cycles and the
-// pipe queues only about two of them, so the issuing thread tests the
-// barriers of the next head while the last MMAs of the current one are
-// queued (blocking only when they are not complete) instead of leaving the
-// pipe idle between heads.  Sustained, the kernel runs at the board's power
-// limit, so fewer issued instructions per score element turn directly into
-// speed.
+// pipe queues only about two of them, so every cycle between the epilogue
+// freeing an accumulator and the next MMA shows up as idle tensor time: the
+// issuer prepares head g + 1 before it blocks, and the epilogue frees the
+// accumulator as soon as its last tensor-memory load has landed (before the
+// arithmetic on that chunk).  Sustained, the kernel runs at the board's power
+// limit (the SM clock settles near 1.4-1.6 GHz), so fewer issued
+// instructions per score element turn directly into speed.
 //
 // Every mbarrier wait is bounded in time; a wait that runs out records
 // LEMO_ERR_TIMEOUT and makes both CTAs of the pair drain what they issued,
@@ -291,40 +292,6 @@ __device__ __forceinline__ void issue_mmas(uint32_t d_tmem, uint64_t da, uint64_
     }
 }
 
-// Whether the phases with parities p0 of b0 and p1 of b1 are both complete.
-// test_wait never suspends the thread, so both tests are in flight together.
-__device__ __forceinline__ bool mbar_test_wait2(uint64_t* b0, uint32_t p0, uint64_t* b1,
-                                                uint32_t p1) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred q0, q1, q;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 q0, [%1], %2;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 q1, [%3], %4;\n\t"
-        "and.pred q, q0, q1;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}\n"
-        : "=r"(ok)
-        : "r"(smem_u32(b0)), "r"(p0), "r"(smem_u32(b1)), "r"(p1)
-        : "memory");
-    return ok != 0;
-}
-
-// Whether both barriers the issuer waits on before head g are complete
-// (never blocks).
-__device__ __forceinline__ bool head_ready(Smem* sm, uint32_t g) {
-    return mbar_test_wait2(&sm->acc_empty[g & 1], ((g >> 1) & 1) ^ 1, &sm->full[g % STAGES],
-                           (g / STAGES) & 1);
-}
-
-// The issuer's two waits before head g: accumulator g & 1 drained by both
-// epilogues, stage g % STAGES loaded by both producers.
-__device__ __forceinline__ bool wait_head(Smem* sm, uint32_t g, uint64_t limit_ns) {
-    uint64_t* ae = &sm->acc_empty[g & 1];
-    uint64_t* fu = &sm->full[g % STAGES];
-    const uint32_t pae = ((g >> 1) & 1) ^ 1, pfu = (g / STAGES) & 1;
-    if (mbar_test_wait2(ae, pae, fu, pfu)) return true;
-    return mbar_wait_slow(ae, pae, sm, limit_ns) && mbar_wait(fu, pfu, sm, limit_ns);
-}
-
 // max(a, b, c) in one three-input min/max instruction.
 __device__ __forceinline__ float max3(float a, float b, float c) {
     float d;
@@ -433,35 +400,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         // Heads are issued back to back over all tiles of the pair (the MMAs
-        // need no tile coordinates).  The tensor pipe queues only about two
-        // MMAs, so the barriers of head g + 1 are tested (without blocking)
-        // while the last MMAs of head g are queued; only when they are not
-        // complete yet does the thread block on them, after its commits.
+        // need no tile coordinates).  The stage, parities and descriptors of
+        // head g + 1 are computed before the thread blocks on its barriers, so
+        // that once the epilogue frees the accumulator only a fence stands
+        // between the wake-up and the next MMA.
         if (lane == 0 && leader) {
             const int64_t my_tiles = (total_tiles - pair + npairs - 1) / npairs;
             const uint32_t heads = (uint32_t)(my_tiles * a.H);
-            bool ok = heads > 0 && wait_head(sm, 0, a.spin_limit_ns);
+            const uint32_t sa0 = smem_u32(tiles);
+            uint32_t s = 0, fph = 0;  // stage of head g and the parity of its full phase
+            uint64_t da = sdesc_sw128(sa0), db = sdesc_sw128(sa0 + A_BYTES);
+            bool ok = heads > 0 && mbar_wait(&sm->acc_empty[0], 1, sm, a.spin_limit_ns) &&
+                      mbar_wait(&sm->full[0], 0, sm, a.spin_limit_ns);
             for (uint32_t g = 0; ok && g < heads; ++g) {
-                const uint32_t buf = g & 1, s = g % STAGES;
-                tc_fence_after();
+                const uint32_t buf = g & 1;
                 const uint32_t d_tmem = tmem_base + buf * ACC_COLS;
-                const uint32_t sa = smem_u32(tiles + s * STAGE_BYTES);
-                const uint64_t da = sdesc_sw128(sa);
-                const uint64_t db = sdesc_sw128(sa + A_BYTES);
+                // head g + 1: its stage, the parities of its two waits
+                const uint32_t s1 = s + 1 == STAGES ? 0 : s + 1;
+                const uint32_t fph1 = s1 == 0 ? fph ^ 1 : fph;
+                const uint32_t aph1 = (((g + 1) >> 1) & 1) ^ 1;
                 const bool more = g + 1 < heads;
-                bool ready = false;
-                if (a.dh == 128) {  // head dimensions 64 and 128 are accepted
+                tc_fence_after();
+                if (a.dh == 128)  // head dimensions 64 and 128 are accepted
+                    issue_mmas<0, 8>(d_tmem, da, db);
+                else
                     issue_mmas<0, 4>(d_tmem, da, db);
-                    ready = more && head_ready(sm, g + 1);
-                    issue_mmas<4, 8>(d_tmem, da, db);
-                } else {
-                    issue_mmas<0, 2>(d_tmem, da, db);
-                    ready = more && head_ready(sm, g + 1);
-                    issue_mmas<2, 4>(d_tmem, da, db);
-                }
                 umma_commit_pair(&sm->empty[s]);       // both CTAs' stage s is free again
                 umma_commit_pair(&sm->acc_full[buf]);  // both CTAs' accumulators are ready
-                if (more && !ready) ok = wait_head(sm, g + 1, a.spin_limit_ns);
+                // everything head g + 1 needs except its barriers, before blocking on them
+                const uint32_t sa1 = sa0 + s1 * STAGE_BYTES;
+                da = sdesc_sw128(sa1);
+                db = sdesc_sw128(sa1 + A_BYTES);
+                if (more)
+                    ok = mbar_wait(&sm->acc_empty[buf ^ 1], aph1, sm, a.spin_limit_ns) &&
+                         mbar_wait(&sm->full[s1], fph1, sm, a.spin_limit_ns);
+                s = s1;
+                fph = fph1;
             }
             // Every MMA completes before either CTA releases its tensor memory.
             umma_commit_pair(&sm->done);
@@ -503,6 +477,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     tmem_ld16(base + ch, &r[0]);
                     tmem_ld16(base + ch + 16, &r[16]);
                     tmem_wait_ld();
+                    if (ch + 32 == COLS_PER_THREAD) {
+                        // every read of this accumulator has landed: free it
+                        // before folding the last chunk
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive_cluster(acc_empty_c[buf]);
+                    }
 #pragma unroll
                     for (int j = 0; j < 32; j += 2) {
                         const float s0 = __uint_as_float(r[j]), s1 = __uint_as_float(r[j + 1]);
@@ -511,9 +492,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                         add_f32x2(acc[ch + j], acc[ch + j + 1], t0, t1);
                     }
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(acc_empty_c[buf]);
             }
             if (!ok) break;
 
