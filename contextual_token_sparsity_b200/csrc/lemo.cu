@@ -230,7 +230,11 @@ lemo_status check_move(const void* x, int64_t ld_x, int64_t x_rows, int32_t d, c
 // region holds the block products P) followed by the predictor buffers.
 struct PredictLayout {
     lemo::WsLayout base;
-    size_t xbar, part, hid, qh, kh, ppart, total;
+    // byte offsets: block-mean planes, padded weight planes, split-K
+    // partials, hidden-activation planes, Qhat / Khat planes, partial products
+    size_t xb_hi, xb_lo, w1p[2], w2p[2], part, hid_hi, hid_lo, q_hi, q_lo, k_hi, k_lo, ppart, total;
+    int ldr;         // rank padded to a multiple of 8
+    int ldh;         // head dimension padded to a multiple of 8
     int64_t tb;      // upper bound of the number of token blocks
     int splits;      // split-K factor of the first predictor GEMM
     int k_chunk;     // K range of one split
@@ -251,9 +255,11 @@ PredictLayout predict_layout(const lemo_shape* s, int d, int rank) {
     p.base = layout_of(s);
     p.tb = ((int64_t)s->total_L + (int64_t)s->batch * (s->block - 1)) / s->block;
     if (p.tb < 1) p.tb = 1;
-    const int64_t hd = (int64_t)s->H * s->dh;
+    p.ldr = (rank + 7) / 8 * 8;
+    p.ldh = (s->dh + 7) / 8 * 8;
+    const int64_t hdp = (int64_t)s->H * p.ldh;
     const int64_t mt = (p.tb + pr::TM - 1) / pr::TM;
-    const int64_t tiles = 2 * ((rank + pr::TN - 1) / pr::TN) * mt;
+    const int64_t tiles = 2 * ((p.ldr + pr::TN - 1) / pr::TN) * mt;
     const int64_t kst = (d + pr::TK - 1) / pr::TK;        // K stages of the first GEMM
     int64_t splits = (kGemmCtas + tiles - 1) / tiles;
     const int64_t max_splits = (kst + 3) / 4;              // at least 4 stages per split
@@ -269,11 +275,22 @@ PredictLayout predict_layout(const lemo_shape* s, int d, int rank) {
     p.hpg = (int)((s->H + groups - 1) / groups);
     p.groups = (s->H + p.hpg - 1) / p.hpg;
     size_t off = p.base.total;
-    p.xbar = off;  off = lemo::align_up(off + 4 * (size_t)p.tb * d, 256);
-    p.part = off;  off = lemo::align_up(off + 4 * (size_t)2 * p.splits * p.tb * rank, 256);
-    p.hid = off;   off = lemo::align_up(off + 4 * (size_t)2 * p.tb * rank, 256);
-    p.qh = off;    off = lemo::align_up(off + 4 * (size_t)p.tb * hd, 256);
-    p.kh = off;    off = lemo::align_up(off + 4 * (size_t)p.tb * hd, 256);
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = lemo::align_up(off + bytes, 256);
+        return o;
+    };
+    p.xb_hi = take(2 * (size_t)p.tb * d);
+    p.xb_lo = take(2 * (size_t)p.tb * d);
+    for (int i = 0; i < 2; ++i) p.w1p[i] = take(2 * (size_t)d * p.ldr);
+    for (int i = 0; i < 2; ++i) p.w2p[i] = take(2 * (size_t)p.ldr * hdp);
+    p.part = take(4 * (size_t)2 * p.splits * p.tb * p.ldr);
+    p.hid_hi = take(2 * (size_t)2 * p.tb * p.ldr);
+    p.hid_lo = take(2 * (size_t)2 * p.tb * p.ldr);
+    p.q_hi = take(2 * (size_t)p.tb * hdp);
+    p.q_lo = take(2 * (size_t)p.tb * hdp);
+    p.k_hi = take(2 * (size_t)p.tb * hdp);
+    p.k_lo = take(2 * (size_t)p.tb * hdp);
     p.ppart = off;
     if (p.groups > 1) off = lemo::align_up(off + 4 * (size_t)p.groups * p.tb * p.tb, 256);
     p.total = off;
@@ -694,67 +711,114 @@ lemo_status lemo_predict_scores(const lemo_shape* shape, int32_t d, const uint16
     char* w = static_cast<char*>(ws);
     const lemo::WsLayout& lay = p.base;
     const lemo::PlanHeader* hdr = reinterpret_cast<const lemo::PlanHeader*>(w + lay.hdr);
-    float* xbar = reinterpret_cast<float*>(w + p.xbar);
     float* part = reinterpret_cast<float*>(w + p.part);
-    float* hid = reinterpret_cast<float*>(w + p.hid);
     float* P = reinterpret_cast<float*>(w + lay.mblk);
-    const int hd = shape->H * shape->dh;
+    auto plane = [&](size_t off) { return reinterpret_cast<uint16_t*>(w + off); };
+    const int hdp = shape->H * p.ldh;  // columns of the Qhat / Khat planes (heads padded)
 
     launch_plan(shape, w, lay, nullptr, st);
     if ((e = launch_status()) != LEMO_OK) return e;
     if (shape->total_L == 0) return LEMO_OK;
+    // weights whose rows are not 16-byte aligned: padded copies
+    const bool w1_vec16 = rank % 8 == 0 && aligned(w1q, 16) && aligned(w1k, 16);
+    const bool w1_vec4 = !w1_vec16 && rank % 2 == 0 && aligned(w1q, 4) && aligned(w1k, 4);
+    const bool pad_w1 = !w1_vec16 && !w1_vec4;
+    const bool pad_w2 = shape->dh % 8 != 0 || !aligned(w2q, 16) || !aligned(w2k, 16);
+    if (pad_w1) {
+        pr::PadArgs pa1 = {};
+        pa1.src[0] = w1q;
+        pa1.src[1] = w1k;
+        pa1.dst[0] = plane(p.w1p[0]);
+        pa1.dst[1] = plane(p.w1p[1]);
+        pa1.rows = pa1.rows_out = d;
+        pa1.cols = pa1.run = rank;
+        pa1.run_ld = p.ldr;
+        pa1.ld_out = p.ldr;
+        launch(pr::pad_kernel, dim3((unsigned)((d + 7) / 8), 2u), 256, 0, st, pa1);
+    }
+    if (pad_w2) {
+        pr::PadArgs pa2 = {};
+        pa2.src[0] = w2q;
+        pa2.src[1] = w2k;
+        pa2.dst[0] = plane(p.w2p[0]);
+        pa2.dst[1] = plane(p.w2p[1]);
+        pa2.rows = pa2.rows_out = rank;
+        pa2.cols = shape->H * shape->dh;
+        pa2.run = shape->dh;
+        pa2.run_ld = p.ldh;
+        pa2.ld_out = hdp;
+        launch(pr::pad_kernel, dim3((unsigned)((rank + 7) / 8), 2u), 256, 0, st, pa2);
+    }
+    const uint16_t* w1s[2] = {pad_w1 ? plane(p.w1p[0]) : w1q, pad_w1 ? plane(p.w1p[1]) : w1k};
+    const uint16_t* w2s[2] = {pad_w2 ? plane(p.w2p[0]) : w2q, pad_w2 ? plane(p.w2p[1]) : w2k};
+    // block means, as hi / lo planes
     launch(pr::pool_kernel,
            dim3((unsigned)p.tb, (unsigned)((d + pr::kPoolCols - 1) / pr::kPoolCols)),
            pr::kPoolThreads, 0, st, x, ld_x, d, shape->cu_seqlens, shape->batch, shape->block, w,
-           lay, xbar);
+           lay, plane(p.xb_hi), plane(p.xb_lo));
     if ((e = launch_status()) != LEMO_OK) return e;
     const unsigned mtiles = (unsigned)((p.tb + pr::TM - 1) / pr::TM);
     // hidden layers of both predictors: split-K partials, then relu of their sum
-    pr::GemmArgs g1;
-    g1.a[0] = g1.a[1] = xbar;
+    pr::GemmArgs g1 = {};
+    g1.a_hi[0] = g1.a_hi[1] = plane(p.xb_hi);
+    g1.a_lo[0] = g1.a_lo[1] = plane(p.xb_lo);
     g1.lda = d;
-    g1.w[0] = w1q;
-    g1.w[1] = w1k;
-    g1.ldw = rank;
+    g1.w[0] = w1s[0];
+    g1.w[1] = w1s[1];
+    g1.ldw = pad_w1 ? p.ldr : rank;
     g1.c[0] = part;
-    g1.c[1] = part + (int64_t)p.splits * p.tb * rank;
-    g1.ldc = rank;
-    g1.c_split = p.tb * rank;
+    g1.c[1] = part + (int64_t)p.splits * p.tb * p.ldr;
+    g1.ldc = p.ldr;
+    g1.c_split = p.tb * p.ldr;
     g1.hdr = hdr;
-    g1.N = rank;
+    g1.N = p.ldr;
     g1.K = d;
+    g1.w_rows = d;
+    g1.w_cols = pad_w1 ? p.ldr : rank;
+    g1.w_vec4 = w1_vec4;
     g1.k_chunk = p.k_chunk;
     g1.splits = p.splits;
-    launch(pr::gemm_kernel, dim3((unsigned)((rank + pr::TN - 1) / pr::TN), mtiles, 2u * p.splits),
-           pr::kMmaThreads, 0, st, g1);
+    launch(pr::gemm_kernel<false>,
+           dim3((unsigned)((p.ldr + pr::TN - 1) / pr::TN), mtiles, 2u * p.splits), pr::kMmaThreads,
+           0, st, g1);
     launch(pr::reduce_kernel, dim3((unsigned)sms, 2u), 256, 0, st, part,
-           (int64_t)p.splits * p.tb * rank, p.tb * rank, p.splits, hdr, rank, hid, p.tb * rank);
-    // block embeddings of both predictors
-    pr::GemmArgs g2;
-    g2.a[0] = hid;
-    g2.a[1] = hid + p.tb * rank;
-    g2.lda = rank;
-    g2.w[0] = w2q;
-    g2.w[1] = w2k;
-    g2.ldw = hd;
-    g2.c[0] = reinterpret_cast<float*>(w + p.qh);
-    g2.c[1] = reinterpret_cast<float*>(w + p.kh);
-    g2.ldc = hd;
+           (int64_t)p.splits * p.tb * p.ldr, p.tb * p.ldr, p.splits, hdr, p.ldr, plane(p.hid_hi),
+           plane(p.hid_lo), p.tb * p.ldr);
+    // block embeddings of both predictors, as hi / lo planes
+    pr::GemmArgs g2 = {};
+    g2.a_hi[0] = plane(p.hid_hi);
+    g2.a_hi[1] = plane(p.hid_hi) + p.tb * p.ldr;
+    g2.a_lo[0] = plane(p.hid_lo);
+    g2.a_lo[1] = plane(p.hid_lo) + p.tb * p.ldr;
+    g2.lda = p.ldr;
+    g2.w[0] = w2s[0];
+    g2.w[1] = w2s[1];
+    g2.ldw = hdp;
+    g2.c_hi[0] = plane(p.q_hi);
+    g2.c_lo[0] = plane(p.q_lo);
+    g2.c_hi[1] = plane(p.k_hi);
+    g2.c_lo[1] = plane(p.k_lo);
+    g2.ldc = hdp;
     g2.c_split = 0;
     g2.hdr = hdr;
-    g2.N = hd;
-    g2.K = rank;
-    g2.k_chunk = (rank + pr::TK - 1) / pr::TK * pr::TK;
+    g2.N = hdp;
+    g2.K = p.ldr;
+    g2.w_rows = rank;
+    g2.w_cols = hdp;
+    g2.w_vec4 = false;
+    g2.k_chunk = (p.ldr + pr::TK - 1) / pr::TK * pr::TK;
     g2.splits = 1;
-    launch(pr::gemm_kernel, dim3((unsigned)((hd + pr::TN - 1) / pr::TN), mtiles, 2u),
+    launch(pr::gemm_kernel<true>, dim3((unsigned)((hdp + pr::TN - 1) / pr::TN), mtiles, 2u),
            pr::kMmaThreads, 0, st, g2);
     if ((e = launch_status()) != LEMO_OK) return e;
     // block products, mean over heads of the positive parts
     pr::ProductsArgs pa;
-    pa.qh = g2.c[0];
-    pa.kh = g2.c[1];
+    pa.q_hi = plane(p.q_hi);
+    pa.q_lo = plane(p.q_lo);
+    pa.k_hi = plane(p.k_hi);
+    pa.k_lo = plane(p.k_lo);
     pa.H = shape->H;
-    pa.dh = shape->dh;
+    pa.ldh = p.ldh;
     pa.hpg = p.hpg;
     pa.groups = p.groups;
     pa.batch = shape->batch;
