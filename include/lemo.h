@@ -291,9 +291,11 @@ LEMO_API lemo_status lemo_mlp_block_scores(const lemo_shape* shape, int32_t d_ff
 
 /*
  * Workspace bytes of lemo_predict_scores for `shape`, residual width d and
- * predictor rank (the plan arrays, block means, hidden activations, split-K
- * partial sums, predicted Q/K block embeddings and the block-product
- * matrices).  Returns 0 for invalid arguments.  HOST-only computation.
+ * predictor rank (the plan arrays; the block means, hidden activations and
+ * predicted Q/K block embeddings, each as a pair of bf16 planes hi + lo; row-
+ * padded copies of the weights for shapes whose rows are not aligned; the
+ * split-K partial sums and the block-product matrices).  Returns 0 for
+ * invalid arguments.  HOST-only computation.
  */
 LEMO_API size_t lemo_predict_workspace_size(const lemo_shape* shape, int32_t d, int32_t rank);
 
@@ -320,8 +322,12 @@ LEMO_API size_t lemo_predict_workspace_size(const lemo_shape* shape, int32_t d, 
  * block_scores DEVICE fp32 [total_blocks].
  * ws, ws_bytes DEVICE workspace of lemo_predict_workspace_size bytes,
  *              256-byte aligned.
- * Computed in fp32 on the CUDA cores; split-K sums are reduced in a fixed
- * order, so the result is deterministic.
+ * fp32 accuracy on the tensor cores: every fp32 operand is split into
+ * bf16 hi + lo and a product is taken as hi*b + lo*b (+ hi*lo' when both
+ * operands are fp32), with fp32 accumulation; split-K and head-group sums
+ * are reduced in a fixed order, so the result is deterministic.  Weights
+ * need only 2-byte alignment (rows that are not 16-byte aligned are read
+ * with smaller copies or through a padded copy in the workspace).
  */
 LEMO_API lemo_status lemo_predict_scores(const lemo_shape* shape, int32_t d, const uint16_t* x,
                                          int64_t ld_x, const uint16_t* w1q, const uint16_t* w2q,
