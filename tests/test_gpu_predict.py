@@ -38,7 +38,16 @@ def _dev(bits):
     return to_device_bf16(bits)
 
 
-def run_predict(lengths, H, dh, b, x_bits, w1q, w2q, w1k, w2k):
+def _dev_misaligned(bits):
+    """Device copy whose data pointer is 2 bytes past a 256-byte boundary."""
+    import torch
+    flat = np.zeros(bits.size + 1, np.uint16)
+    flat[1:] = np.ascontiguousarray(bits).ravel()
+    t = torch.from_numpy(flat.view(np.int16)).cuda()
+    return t[1:].view(bits.shape)
+
+
+def run_predict(lengths, H, dh, b, x_bits, w1q, w2q, w1k, w2k, misaligned=False):
     import torch
     cu = np.zeros(len(lengths) + 1, dtype=np.int32)
     cu[1:] = np.cumsum(lengths)
@@ -49,7 +58,8 @@ def run_predict(lengths, H, dh, b, x_bits, w1q, w2q, w1k, w2k):
                      device="cuda")
     nblk = sum(-(-L // b) for L in lengths)
     out = torch.full((max(nblk, 1),), float("nan"), dtype=torch.float32, device="cuda")
-    lemo.lemo_predict_scores(shape, _dev(x_bits), _dev(w1q), _dev(w2q), _dev(w1k), _dev(w2k),
+    wdev = _dev_misaligned if misaligned else _dev
+    lemo.lemo_predict_scores(shape, _dev(x_bits), wdev(w1q), wdev(w2q), wdev(w1k), wdev(w2k),
                              out, ws)
     st = lemo.lemo_get_error()
     assert st == lemo.LEMO_OK, lemo.STATUS.get(st, st)
@@ -67,7 +77,9 @@ def oracle_predict(lengths, H, dh, b, x_bits, w1q, w2q, w1k, w2k):
 
 CASES = [([300, 0, 517, 64, 1], 2, 64, 64, 64, 48),
          ([1000], 3, 128, 128, 256, 40),
-         ([2049, 640], 4, 32, 64, 136, 100)]
+         ([2049, 640], 4, 32, 64, 136, 100),   # rank % 8 != 0: W1 rows read 4 bytes at a time
+         ([700, 130], 3, 20, 64, 64, 37),       # odd rank and dh % 8 != 0: padded weight copies
+         ([513], 2, 24, 128, 40, 6)]
 
 
 @pytest.mark.parametrize("lengths,H,dh,b,d,rank", CASES, ids=[str(c[0]) for c in CASES])
@@ -80,6 +92,20 @@ def test_predictor_matches_oracle(lengths, H, dh, b, d, rank):
     want = oracle_predict(lengths, H, dh, b, x, w1q, w2q, w1k, w2k)
     err = assert_scores_close(got, want, "predicted scores")
     assert err < 1e-4
+
+
+def test_weights_with_only_2_byte_alignment():
+    """Weight pointers 2 bytes off a 16-byte boundary go through padded
+    copies; the arithmetic is the same, so the scores are the same bits."""
+    lengths, H, dh, b, d, rank = [640, 200], 2, 64, 64, 128, 48
+    x = synth.normal_bf16(sum(lengths), d, 9, 7)
+    w1q, w2q, _ = synth.predictor_weights(d, rank, H * dh, 0.4, 9, 10)
+    w1k, w2k, _ = synth.predictor_weights(d, rank, H * dh, 0.4, 9, 11)
+    aligned, _ = run_predict(lengths, H, dh, b, x, w1q, w2q, w1k, w2k)
+    shifted, _ = run_predict(lengths, H, dh, b, x, w1q, w2q, w1k, w2k, misaligned=True)
+    assert np.array_equal(aligned, shifted)
+    assert_scores_close(shifted, oracle_predict(lengths, H, dh, b, x, w1q, w2q, w1k, w2k),
+                        "predicted scores, misaligned weights")
 
 
 def test_pruned_neurons_can_be_left_out():
