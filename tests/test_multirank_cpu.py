@@ -92,3 +92,25 @@ def test_clock_summary_reports_load_clocks_and_reasons():
     assert s["sm_mhz"] == 1500 and s["sm_max_mhz"] == 1965 and s["samples"] == 3
     assert s["power_w_max"] == 995.0 and s["reasons"] == ["sw_power_cap"]
     assert bench.ClockSampler.summary([], "nvml") is None
+
+
+def test_scorer_traffic_record_is_tied_to_the_scorer_source(tmp_path, monkeypatch):
+    """roofline.traffic comes from the committed ncu summary only while that
+    summary was taken on the current scorer source; any other workload, a
+    stale digest or a missing file give null."""
+    import bench
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.profiled_traffic("llama7b-16k") is None            # no summary
+    src = tmp_path / "contextual_token_sparsity_b200" / "csrc"
+    src.mkdir(parents=True)
+    for name in bench.SCORE_SOURCES:
+        (src / name).write_text("// " + name)
+    digest = bench.score_source_digest()
+    (prof / "score_tiles_llama7b.md").write_text(
+        f"text\n\n    source_digest = {digest}\n    dram_bytes_per_launch = 476498261\n")
+    assert bench.profiled_traffic("llama7b-16k") == 476498261
+    assert bench.profiled_traffic("llama7b-8k") is None              # other workload
+    (src / bench.SCORE_SOURCES[0]).write_text("// changed")
+    assert bench.profiled_traffic("llama7b-16k") is None            # source changed since
