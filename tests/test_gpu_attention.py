@@ -120,6 +120,20 @@ def test_compact_output_matches_oracle(lengths, H, dh, b, p):
     check_compact(got, want, v, H, dh)
 
 
+def test_many_short_sequences():
+    """600 sequences with 0 to 5 kept blocks each (ragged last blocks,
+    empty sequences): query-tile pairs and key tiles per sequence."""
+    rng = np.random.default_rng(31)
+    lengths = [int(v) for v in rng.choice([0, 1, 64, 65, 200, 300], size=600)]
+    H, dh, b = 2, 64, 64
+    L = sum(lengths)
+    q, k, v = (synth.normal_bf16(L, H * dh, 31, st) for st in (20, 21, 22))
+    cu, idx, cu_kept, K = random_kept(lengths, b, 31, 0.6)
+    st, got, _ = run_attention(lengths, H, dh, b, q, k, v, idx, cu_kept, K)
+    assert st == lemo.LEMO_OK, lemo.STATUS.get(st, st)
+    check_compact(got, oracle.attention_kept(q, k, v, idx, cu_kept, H, dh), v, H, dh)
+
+
 def test_in_place_residual_and_untouched_rows():
     lengths, H, dh, b = [700, 333], 2, 128, 64
     L = sum(lengths)

@@ -124,6 +124,20 @@ def test_small_1k_full():
     assert int(res["mask"].sum()) == 8
 
 
+def test_many_short_sequences():
+    """1500 sequences (empty, shorter than a block, a block and a token,
+    a few blocks): the plan's prefix loop runs in two chunks and every
+    kernel maps tiles, blocks and rows to their sequences by search."""
+    rng = np.random.default_rng(21)
+    lengths = [int(v) for v in rng.choice([0, 1, 5, 63, 64, 65, 130, 200], size=1500)]
+    H, dh, b, d = 2, 64, 64, 16
+    q, k, cu, x, y = _inputs(lengths, H, dh, d, seed=21)
+    s_ref = oracle.column_scores(oracle.score_blocks(q, k, cu, H, dh, b))
+    theta = oracle.threshold_for_keep_ratio(s_ref, 0.5)
+    res = run_layer(lengths, H, dh, b, d, q, k, x, y, theta)
+    check_all(res, q, k, cu, H, dh, b, x, y, theta)
+
+
 def test_varlen_packing_equals_separate_calls():
     """A packed batch gives the same scores as each sequence on its own."""
     lengths, H, dh, b, d = [512, 130, 700], 2, 128, 64, 8
