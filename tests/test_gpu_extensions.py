@@ -91,8 +91,13 @@ def _mlp_gpu(lengths, b, mats, gated):
         layer.block_scores[: layer.total_blocks].cpu().numpy().astype(np.float64), cu
 
 
+# 400 sequences of 0 to 200 tokens: every token row finds its sequence and block by search
+MANY = [int(v) for v in np.random.default_rng(51).choice([0, 1, 63, 64, 65, 200], size=400)]
+
+
 @pytest.mark.parametrize("gated", [False, True], ids=["relu", "silu-gated"])
-@pytest.mark.parametrize("lengths,b,d_ff", [([300, 0, 517, 1], 64, 136), ([1000, 257], 128, 512)])
+@pytest.mark.parametrize("lengths,b,d_ff", [([300, 0, 517, 1], 64, 136), ([1000, 257], 128, 512),
+                                            (MANY, 64, 64)])
 def test_mlp_scores_match_oracle_and_select(lengths, b, d_ff, gated):
     mats = synth.mlp_activations(sum(lengths), d_ff, 0.1, seed=len(lengths), gated=gated)
     layer, tok, blk, cu = _mlp_gpu(lengths, b, mats, gated)

@@ -94,6 +94,29 @@ def test_predictor_matches_oracle(lengths, H, dh, b, d, rank):
     assert err < 1e-4
 
 
+def test_many_short_sequences():
+    """300 sequences: 64 x 64 tiles of block pairs span several sequences,
+    whose cross pairs the block products must leave out."""
+    rng = np.random.default_rng(41)
+    lengths = [int(v) for v in rng.choice([0, 1, 63, 128, 129, 300], size=300)]
+    H, dh, b, d, rank = 2, 32, 64, 64, 24
+    x = synth.normal_bf16(sum(lengths), d, 41, 7)
+    w1q, w2q, _ = synth.predictor_weights(d, rank, H * dh, 0.4, 41, 10)
+    w1k, w2k, _ = synth.predictor_weights(d, rank, H * dh, 0.4, 41, 11)
+    got, _ = run_predict(lengths, H, dh, b, x, w1q, w2q, w1k, w2k)
+    want = oracle_predict(lengths, H, dh, b, x, w1q, w2q, w1k, w2k)
+    assert_scores_close(got, want, "predicted scores, 300 sequences")
+    # fp32 accuracy: one-token sequences give scores near 0, and a block pair's
+    # 32-term dot products cancel (each product is exact to 2^-16, so the error
+    # follows the size of the terms, not of the result); the error is measured
+    # against the scale of the scores, and relatively (10x inside the 1e-2
+    # bar) only for the scores that are not near 0
+    scale = np.abs(want).max()
+    assert np.abs(got - want).max() <= 1e-5 * scale
+    big = np.abs(want) >= 1e-3 * scale
+    assert (np.abs(got - want)[big] / np.abs(want[big])).max() < 1e-3
+
+
 def test_weights_with_only_2_byte_alignment():
     """Weight pointers 2 bytes off a 16-byte boundary go through padded
     copies; the arithmetic is the same, so the scores are the same bits."""
