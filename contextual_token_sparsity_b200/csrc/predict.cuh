@@ -15,7 +15,10 @@
 // hi = bf16(v) and lo = bf16(v - hi); a product a.b is taken as
 // a_hi b_hi + a_lo b_hi + a_hi b_lo (the weights are bf16 already, so for
 // the GEMMs only a_hi b + a_lo b is needed).  The dropped term is below
-// 2^-16 of the product, so the predicted scores stay at fp32 accuracy.
+// 2^-16 of each product, so a score's error is about 2^-16 of the sum of
+// the magnitudes of its products: near fp32 accuracy, except where a block
+// pair's dot products cancel (then it stays small against the scores'
+// scale, not against that one score).
 //
 // Every fp32 intermediate (block means, hidden activations, Qhat, Khat) is
 // split once, by the kernel that produces it, and stored as two bf16 planes
