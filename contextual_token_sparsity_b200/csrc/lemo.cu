@@ -161,6 +161,7 @@ bool encode_rows(CUtensorMap* tm, const uint16_t* base, int64_t rows, int64_t wi
 }
 
 bool g_attn_smem_set[kMaxDevices];
+bool g_prod_smem_set[kMaxDevices];
 
 // CTA pairs of the scoring kernel that fit on the device at once (one
 // persistent wave).  Sets the kernel's shared-memory limit on first use.
@@ -826,8 +827,18 @@ lemo_status lemo_predict_scores(const lemo_shape* shape, int32_t d, const uint16
     pa.inv_h = 1.f / (float)shape->H;
     pa.part = reinterpret_cast<float*>(w + p.ppart);
     pa.P = P;
-    launch(pr::products_kernel, dim3((unsigned)p.ptiles, (unsigned)p.groups), pr::kMmaThreads, 0,
-           st, pa, w, lay);
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!g_prod_smem_set[dev]) {
+            if (cudaFuncSetAttribute(pr::products_kernel,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     pr::PROD_SMEM) != cudaSuccess)
+                return LEMO_ERR_CUDA;
+            g_prod_smem_set[dev] = true;
+        }
+    }
+    launch(pr::products_kernel, dim3((unsigned)p.ptiles, (unsigned)p.groups), pr::kMmaThreads,
+           pr::PROD_SMEM, st, pa, w, lay);
     if ((e = launch_status()) != LEMO_OK) return e;
     if (p.groups > 1) launch(pr::products_reduce_kernel, sms * 2, 256, 0, st, pa, w, lay);
     const int64_t cs_ctas = (p.tb + 7) / 8;

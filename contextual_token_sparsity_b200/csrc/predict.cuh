@@ -169,8 +169,9 @@ constexpr int B_PITCH = 144;                // bytes per row of a [32][64] bf16 
 constexpr int B_PLANE = TK * B_PITCH;       // 4608 bytes
 constexpr int GEMM_STAGES = 3;
 constexpr int GEMM_STAGE = 2 * A_PLANE + B_PLANE;
-constexpr int PROD_STAGES = 2;
+constexpr int PROD_STAGES = 3;
 constexpr int PROD_STAGE = 4 * A_PLANE;
+constexpr int PROD_SMEM = PROD_STAGES * PROD_STAGE;  // dynamic shared memory (60 KB)
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
     return (uint32_t)__cvta_generic_to_shared(p);
@@ -532,7 +533,7 @@ __global__ void __launch_bounds__(kMmaThreads)
     const int n0 = tn * TM, mb0 = tm * TN;
     if (n0 >= TB) return;
     const int64_t HD = (int64_t)a.H * a.ldh;
-    __shared__ __align__(128) uint8_t sm[PROD_STAGES][PROD_STAGE];  // [Q hi | Q lo | K hi | K lo]
+    extern __shared__ __align__(128) uint8_t prod_smem[];  // stages of [Q hi | Q lo | K hi | K lo]
     const int warp = threadIdx.x >> 5;
     const int wm = (warp >> 1) * 32, wn = (warp & 1) * 32;
     float acc[2][4][4], tot[2][4][4];
@@ -542,7 +543,7 @@ __global__ void __launch_bounds__(kMmaThreads)
     const int per_head = (a.ldh + TK - 1) / TK;
     const int nst = (h1 - h0) * per_head;
     auto load_stage = [&](int s) {
-        uint8_t* b = sm[s % PROD_STAGES];
+        uint8_t* b = prod_smem + (s % PROD_STAGES) * PROD_STAGE;
         const int h = h0 + s / per_head;
         const int k0 = h * a.ldh + (s % per_head) * TK, ke = (h + 1) * a.ldh;
         load_k_tile(b, a.q_hi, HD, n0, TB, k0, ke);
@@ -560,7 +561,7 @@ __global__ void __launch_bounds__(kMmaThreads)
         __syncthreads();  // stage s landed for every thread; stage s - 1 is no longer read
         if (s + PROD_STAGES - 1 < nst) load_stage(s + PROD_STAGES - 1);
         cp_commit();
-        const uint8_t* b = sm[s % PROD_STAGES];
+        const uint8_t* b = prod_smem + (s % PROD_STAGES) * PROD_STAGE;
 #pragma unroll
         for (int ks = 0; ks < TK; ks += 16) {
             uint32_t ah[2][4], al[2][4], bh[4][2], bl[4][2];
