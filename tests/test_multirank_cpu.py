@@ -64,7 +64,31 @@ def test_single_rank_is_identity():
     assert bench.whole_job_rate(100, 1, 2.0) == 50.0
 
 
-@pytest.mark.parametrize("workload", ["llama7b-16k", "attn-llama7b-16k", "lmhead-llama7b-16k"])
+ALL_WORKLOADS = ["small-1k", "llama7b-8k", "llama7b-16k", "varlen-10k", "llama13b-32k",
+                 "lmhead-llama7b-16k", "attn-llama7b-16k", "predict-llama13b-32k",
+                 "mlp-llama7b-16k"]
+
+
+def test_every_workload_has_its_definition_and_stored_thresholds():
+    """Each bench workload names a generator configuration; the layer
+    workloads also have their oracle-only stored thresholds."""
+    import os
+
+    import bench
+    from contextual_token_sparsity_b200 import synth
+    here = os.path.dirname(os.path.abspath(__file__))
+    for w in ALL_WORKLOADS:
+        if w in synth.WORKLOADS:
+            if w != "small-1k":  # small enough to score in the tests themselves
+                assert os.path.exists(os.path.join(here, "golden", f"{w}.json")), w
+                assert bench.thresholds(w, synth.WORKLOADS[w].layers) is not None, w
+        elif w.startswith("lmhead-"):
+            assert w in synth.LM_HEAD_WORKLOADS, w
+        else:  # extension workloads run on a layer workload's shapes
+            assert w.split("-", 1)[1] in synth.WORKLOADS, w
+
+
+@pytest.mark.parametrize("workload", ALL_WORKLOADS)
 def test_reference_arm_other_ranks_exit_without_work(workload, monkeypatch, capsys):
     """Under torchrun the reference arm runs on rank 0 only: any other rank
     prints nothing and returns at once (no oracle work, no collective)."""
