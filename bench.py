@@ -130,25 +130,34 @@ def score_source_digest() -> str:
 
 
 def profiled_traffic(workload: str):
-    """DRAM bytes per scorer launch from the committed ncu summary
-    (profiles/score_tiles_llama7b.md), if it was taken on the current scorer source
-    (else None)."""
-    path = os.path.join(ROOT, "profiles", "score_tiles_llama7b.md")
-    if workload != "llama7b-16k" or not os.path.exists(path):
-        return None
-    rec = {}
-    with open(path) as f:
-        for line in f:
-            line = line.strip()
-            if " = " in line:
-                k, v = line.split(" = ", 1)
-                rec[k.strip()] = v.strip()
-    if rec.get("source_digest") != score_source_digest():
+    """DRAM bytes per scorer launch from the committed ncu record
+    (profiles/score_tiles_traffic.json), if it was taken on this workload and
+    on the current scorer source (else None)."""
+    path = os.path.join(ROOT, "profiles", "score_tiles_traffic.json")
+    if not os.path.exists(path):
         return None
     try:
+        with open(path) as f:
+            rec = json.load(f)
+        if rec.get("workload") != workload or rec.get("source_digest") != score_source_digest():
+            return None
         return int(rec["dram_bytes_per_launch"])
-    except (KeyError, ValueError):
+    except (KeyError, ValueError, TypeError):
         return None
+
+
+def headline_config(key: str, w, kept, thetas, theta_src: str, world: int) -> dict:
+    """The `config` object of a headline-workload line; both arms print the
+    same one."""
+    nl = w.layers
+    return {"workload": f"{key}: {w.name}", "layers": nl,
+            "seq_lens": list(w.lengths), "heads": w.H, "head_dim": w.dh,
+            "block": w.block, "d": w.d, "keep": list(w.keep), "kept_tokens": list(kept),
+            "thresholds": thetas, "threshold_source": theta_src, "pad_to": PAD_TO,
+            "l2": "not flushed; each step streams "
+                  f"{(nl * (2 * w.total_L * w.H * w.dh * 2) + 3 * w.total_L * w.d * 2) / 1e9:.2f}"
+                  " GB of Q/K/residual rows (> 126 MB L2)",
+            "parallelism": f"{world} independent replica(s), no collective"}
 
 
 def thresholds(key: str, layers: int):
@@ -423,14 +432,7 @@ def run_lemo(args):
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(step_s * 1e3, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": f"{args.workload}: {w.name}", "layers": nl,
-                   "seq_lens": list(w.lengths), "heads": w.H, "head_dim": w.dh,
-                   "block": w.block, "d": w.d, "keep": list(w.keep), "kept_tokens": kept,
-                   "thresholds": thetas, "threshold_source": theta_src, "pad_to": PAD_TO,
-                   "l2": "not flushed; each step streams "
-                         f"{(nl * (2 * w.total_L * w.H * w.dh * 2) + 3 * w.total_L * w.d * 2) / 1e9:.2f}"
-                         " GB of Q/K/residual rows (> 126 MB L2)",
-                   "parallelism": f"{world} independent replica(s), no collective"},
+        "config": headline_config(args.workload, w, kept, thetas, theta_src, world),
         "roofline": roofline,
         "path_roofline": {"frac": round(t_roof / step_s, 4),
                           "roofline_ms_per_step": round(t_roof * 1e3, 4),
@@ -444,6 +446,11 @@ def run_lemo(args):
         "gpu_launches": LAUNCHES_PER_LAYER * nl * args.steps,
         "clocks": clk,
     }
+
+    # the naive token movement beside the fused one (outside the timed region)
+    fused_us = [1e3 * statistics.fmean(ev[i][l][2].elapsed_time(ev[i][l][4])
+                                       for i in range(args.steps)) for l in range(nl)]
+    out["naive_movement"] = naive_movement(x, y_out, layers, kept, fused_us)
 
     # end to end through the C ABI with host buffers: H2D of each layer's
     # Q/K/sublayer output and of the residual, the path, D2H of the residual
@@ -460,6 +467,68 @@ def run_lemo(args):
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(out), flush=True)
+
+
+def naive_movement(x, y_out, layers, kept, fused_us, reps: int = 10):
+    """Time the naive token movement that permutation-free movement replaces
+    (Jenga summary, section 4.2.3, and Fig. 18 of section 6.2) beside the
+    fused gather + scatter of each layer, outside the timed region:
+
+        eliminate      xk = x.index_select(0, kept)          (compact copy of the kept rows)
+        re-permute     o = zeros_like(x); o.index_copy_(0, kept, y[:K])   (zero-padded,
+                       original token order)
+        residual add   x.add_(o)                              (over all L rows)
+
+    (PyTorch ops, a comparator only; the sublayer between them is not
+    timed).  Also checks on a copy of x that both give the same bits."""
+    import torch
+    stream = torch.cuda.current_stream(x.device)
+    res = {"naive_us_per_layer": [], "fused_us_per_layer": [round(v, 2) for v in fused_us],
+           "naive_ops": "torch index_select; zeros_like + index_copy_; full-length add_",
+           "fused_ops": "lemo_gather_pad + lemo_scatter_residual (kept rows only)",
+           "pages": "10x to over 50x, growing with sequence length (Jenga Fig. 18; hardware "
+                    "and naive implementation not stated)", "matches_fused": True}
+    for l, L_ in enumerate(layers):
+        K = kept[l]
+        idx = L_.kept_idx[:K].long()
+        yk = y_out[l][:K]
+        xw = x.clone()
+
+        def naive():
+            xk = xw.index_select(0, idx)
+            o = torch.zeros_like(xw)
+            o.index_copy_(0, idx, yk)
+            xw.add_(o)
+            return xk
+
+        for _ in range(2):
+            naive()
+        ts = []
+        for _ in range(reps):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            naive()
+            b.record(stream)
+            b.synchronize()
+            ts.append(1e3 * a.elapsed_time(b))
+        res["naive_us_per_layer"].append(round(statistics.median(ts), 2))
+        # same bits: the naive path and the fused path on one copy of x each
+        xa, xb = x.clone(), x.clone()
+        torch.cuda.synchronize()
+        xk = xa.index_select(0, idx)
+        o = torch.zeros_like(xa)
+        o.index_copy_(0, idx, yk)
+        xa.add_(o)
+        g = L_.gather(xb)
+        L_.scatter(xb, y_out[l])
+        torch.cuda.synchronize()
+        same = bool(torch.equal(xa.view(torch.int16), xb.view(torch.int16))) and \
+            bool(torch.equal(xk.view(torch.int16), g[:K].view(torch.int16)))
+        res["matches_fused"] = res["matches_fused"] and same
+    res["speedup_per_layer"] = [round(n / f, 2) for n, f in
+                                zip(res["naive_us_per_layer"], res["fused_us_per_layer"])]
+    return res
 
 
 def run_e2e(args, host, layers, thetas, dev, world, local, tokens_per_step):
@@ -1103,26 +1172,30 @@ class OracleSample:
         t = time.perf_counter() - t0
         return t * self.all_pairs / pairs, rows, pairs, t
 
-    def time_rest(self):
-        """select + compact + gather + scatter of the layer, in full."""
-        if self.t_rest is None:
-            o, w, inp = self.oracle, self.w, self.inp
-            gpath = os.path.join(ROOT, "tests", "golden", f"{self.key}.json")
-            if os.path.exists(gpath):
-                with open(gpath) as f:
-                    g = json.load(f)["layers"][self.layer]
-                sc = np.array([float(v) for v in g["scores"]])
-                theta = float(g["theta"])
-            else:
-                sc = np.linspace(1.0, 0.0, sum(-(-Ls // w.block) for Ls in w.lengths))
-                theta = 0.5
-            t1 = time.perf_counter()
-            mask = o.keep_mask(sc, theta)
-            idx, _, _ = o.compact(mask, inp["cu_seqlens"], w.block)
-            o.gather_pad(inp["x"], idx, PAD_TO)
-            o.scatter_residual(inp["x"], inp["y_out"], idx)
-            self.t_rest = time.perf_counter() - t1
+    def run_rest(self):
+        """select + compact + gather + scatter of the layer, in full; returns
+        its time."""
+        o, w, inp = self.oracle, self.w, self.inp
+        gpath = os.path.join(ROOT, "tests", "golden", f"{self.key}.json")
+        if os.path.exists(gpath):
+            with open(gpath) as f:
+                g = json.load(f)["layers"][self.layer]
+            sc = np.array([float(v) for v in g["scores"]])
+            theta = float(g["theta"])
+        else:
+            sc = np.linspace(1.0, 0.0, sum(-(-Ls // w.block) for Ls in w.lengths))
+            theta = 0.5
+        t1 = time.perf_counter()
+        mask = o.keep_mask(sc, theta)
+        idx, _, _ = o.compact(mask, inp["cu_seqlens"], w.block)
+        o.gather_pad(inp["x"], idx, PAD_TO)
+        o.scatter_residual(inp["x"], inp["y_out"], idx)
+        self.t_rest = time.perf_counter() - t1
         return self.t_rest
+
+    def time_rest(self):
+        """select + compact + gather + scatter of the layer, in full (timed once)."""
+        return self.t_rest if self.t_rest is not None else self.run_rest()
 
     def describe(self, rows, pairs, t_rows):
         return (f"layer {self.layer} of {self.key}: {rows} of {self.nb} query-block rows "
@@ -1261,32 +1334,67 @@ def run_reference_ext(args):
     print(json.dumps(out), flush=True)
 
 
+def golden_kept(key: str, w, thetas):
+    """Kept tokens per layer from the stored oracle scores and thresholds."""
+    import oracle
+    with open(os.path.join(ROOT, "tests", "golden", f"{key}.json")) as f:
+        g = json.load(f)
+    cu = np.zeros(len(w.lengths) + 1, dtype=np.int64)
+    cu[1:] = np.cumsum(w.lengths)
+    kept = []
+    for l in range(w.layers):
+        sc = np.array([float(v) for v in g["layers"][l]["scores"]])
+        _, _, K = oracle.compact(oracle.keep_mask(sc, thetas[l]), cu, w.block)
+        kept.append(int(K))
+    return kept
+
+
 def run_reference(args):
+    """The reference arm: the CPU oracle, as it stands, on a bounded sample of
+    the workload per step.  A step scores a random set of query-block rows of
+    layer 0 for a fixed time budget and runs threshold, compaction, gather and
+    scatter of that layer in full; ms_per_step is the measured time of that
+    sampled work.  `value` scales the sample to a whole layer by block pairs
+    (a row's cost is proportional to its key blocks) and is reported in the
+    headline's unit, with the scale factor beside it."""
     world, rank, local = dist_env()
     if rank != 0:
         return  # the reference arm runs on rank 0 only
+    from contextual_token_sparsity_b200 import synth
+    w = synth.WORKLOADS[args.workload]
+    thetas = thresholds(args.workload, w.layers)
     smp = OracleSample(args.workload, 0)
-    w = smp.w
-    t_rest = smp.time_rest()
-    per_step = max(0.3, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
-    vals, desc = [], ""
+    per_step = max(0.3, min(20.0, 90.0 / max(1, args.steps + args.warmup)))
+    measured, layer_est, fracs, desc = [], [], [], ""
     for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
         t_score, rows, pairs, t_rows = smp.time_rows(per_step, seed=i)
+        t_rest = smp.run_rest()
+        t_step = time.perf_counter() - t0
         if i >= args.warmup:
-            vals.append(t_score + t_rest)
+            measured.append(t_step)
+            layer_est.append(t_score + t_rest)
+            fracs.append(pairs / smp.all_pairs)
             desc = smp.describe(rows, pairs, t_rows)
-    t_layer = statistics.fmean(vals)
+    t_layer = statistics.fmean(layer_est)
     value = w.total_L / t_layer
+    if thetas is not None:
+        kept, theta_src = golden_kept(args.workload, w, thetas), "oracle scores (tests/golden)"
+    else:
+        kept, theta_src = [], "none stored"
     out = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(t_layer * w.layers * 1e3, 1), "higher_is_better": True,
+        "ms_per_step": round(1e3 * statistics.fmean(measured), 1), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "impl": "reference",
-        "config": {"workload": f"{args.workload}: {w.name}", "layers": w.layers,
-                   "seq_lens": list(w.lengths), "heads": w.H, "head_dim": w.dh,
-                   "block": w.block, "d": w.d, "keep": list(w.keep),
-                   "parallelism": "CPU oracle, rank 0 only"},
+        "config": headline_config(args.workload, w, kept, thetas, theta_src, world),
+        "reference_arm": "CPU oracle on rank 0 only (the other ranks exit without work); "
+                         "each step is a bounded sample of layer 0",
+        "sample": {"block_pair_fraction_per_step": round(statistics.fmean(fracs), 4),
+                   "measured_s_per_step": round(statistics.fmean(measured), 2),
+                   "extrapolated_s_per_layer": round(t_layer, 2),
+                   "extrapolated_ms_per_full_step": round(1e3 * t_layer * w.layers, 1)},
         "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": blas_threads(),
                          "kind": "oracle", "sample": f"per step: {desc}"},
         "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,

@@ -500,8 +500,10 @@ lemo_status lemo_select(const lemo_shape* shape, const float* block_scores, floa
 // lemo_select with its scratch in a device array owned by the library (for
 // callers that cannot allocate).  The array is reserved in every GPU's memory
 // when the library is loaded.  Host code must not pass the symbol itself to a
-// kernel - on the host it names a host-side stand-in - so its device address
-// is looked up once per device (with that device current) and cached.
+// kernel - on the host it names a host-side stand-in - so every call looks up
+// its device address on the current device (a host-side query that
+// allocates nothing); nothing is cached, so a device that was reset and
+// re-initialised gets the array's new address.
 // ---------------------------------------------------------------------------
 }  // extern "C"
 
@@ -509,7 +511,6 @@ namespace {
 constexpr int32_t kStaticMaxBatch = 4096;
 constexpr int32_t kStaticMaxTokens = 1 << 24;
 constexpr size_t kStaticScratchBytes = 160 * 1024;
-char* g_static_scratch_dev[kMaxDevices];  // device address of the array, per device
 }  // namespace
 
 static __device__ __align__(256) char g_select_scratch[kStaticScratchBytes];
@@ -530,21 +531,12 @@ lemo_status lemo_select_static_ws(const lemo_shape* shape, const float* block_sc
         return LEMO_ERR_CAPACITY;
     const lemo::WsLayout lay = layout_of(shape);
     if (lay.mblk > kStaticScratchBytes) return LEMO_ERR_CAPACITY;  // selection stops before M
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LEMO_ERR_CUDA;
-    char* w = nullptr;
-    {
-        std::lock_guard<std::mutex> lk(g_mu);
-        if (!g_static_scratch_dev[dev]) {
-            void* p = nullptr;
-            if (cudaGetSymbolAddress(&p, g_select_scratch) != cudaSuccess || !p) {
-                cudaGetLastError();
-                return LEMO_ERR_CUDA;
-            }
-            g_static_scratch_dev[dev] = static_cast<char*>(p);
-        }
-        w = g_static_scratch_dev[dev];
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_select_scratch) != cudaSuccess || !p) {
+        cudaGetLastError();
+        return LEMO_ERR_CUDA;
     }
+    char* w = static_cast<char*>(p);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     // The plan kernel re-initialises the look-back descriptors, the ticket and
     // kept_total at the start of every call.
@@ -565,7 +557,7 @@ lemo_status lemo_select_static_ws(const lemo_shape* shape, const float* block_sc
     a.lay = lay;
     a.skip_publish_tile = g_skip_publish_tile;
     a.spin_limit_ns = (uint64_t)g_spin_ns;
-    lemo::select_kernel<<<(unsigned)lay.n_lookback, lemo::kSelectThreads, 0, st>>>(a);
+    launch(lemo::select_kernel, (unsigned)lay.n_lookback, lemo::kSelectThreads, 0, st, a);
     return launch_status();
 }
 

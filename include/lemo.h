@@ -178,8 +178,10 @@ LEMO_API lemo_status lemo_select(const lemo_shape* shape, const float* block_sco
  *
  * Limits: batch <= 4096 and total_L <= 16777216; a larger shape returns
  * LEMO_ERR_CAPACITY and enqueues nothing.
- * The first call on a device looks up the array's device address with that
- * device current; make that first call before any stream capture.
+ * Every call looks up the array's device address on the current device (a
+ * host-side query that allocates nothing).  The first call on a device may
+ * also load the library's device code there; make that first call before
+ * any stream capture.
  * Every call on a device uses the same array and re-initialises what must
  * start at zero at its beginning, so calls that can overlap on the GPU (for
  * example on two streams with no ordering between them) race and corrupt each

@@ -119,22 +119,31 @@ def test_clock_summary_reports_load_clocks_and_reasons():
 
 
 def test_scorer_traffic_record_is_tied_to_the_scorer_source(tmp_path, monkeypatch):
-    """roofline.traffic comes from the committed ncu summary only while that
-    summary was taken on the current scorer source; any other workload, a
-    stale digest or a missing file give null."""
+    """roofline.traffic comes from the committed ncu record only while that
+    record was taken on the current scorer source and on the bench workload;
+    any other workload, a stale digest, a malformed or a missing file give
+    null."""
+    import json
+
     import bench
     prof = tmp_path / "profiles"
     prof.mkdir()
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    assert bench.profiled_traffic("llama7b-16k") is None            # no summary
+    assert bench.profiled_traffic("llama7b-16k") is None            # no record
     src = tmp_path / "contextual_token_sparsity_b200" / "csrc"
     src.mkdir(parents=True)
     for name in bench.SCORE_SOURCES:
         (src / name).write_text("// " + name)
     digest = bench.score_source_digest()
-    (prof / "score_tiles_llama7b.md").write_text(
-        f"text\n\n    source_digest = {digest}\n    dram_bytes_per_launch = 476498261\n")
+    rec = prof / "score_tiles_traffic.json"
+    rec.write_text(json.dumps({"workload": "llama7b-16k", "source_digest": digest,
+                               "dram_bytes_per_launch": 476498261}))
     assert bench.profiled_traffic("llama7b-16k") == 476498261
     assert bench.profiled_traffic("llama7b-8k") is None              # other workload
+    rec.write_text("{not json")
+    assert bench.profiled_traffic("llama7b-16k") is None            # malformed
+    rec.write_text(json.dumps({"workload": "llama7b-16k", "source_digest": digest,
+                               "dram_bytes_per_launch": 476498261}))
     (src / bench.SCORE_SOURCES[0]).write_text("// changed")
     assert bench.profiled_traffic("llama7b-16k") is None            # source changed since
+

@@ -84,3 +84,66 @@ def test_static_workspace_select_rejects_shapes_over_its_limit():
             lemo.lemo_select_static_ws(shape, scores, 0.0, mask, out, out, out)
         assert e.value.status == lemo.LEMO_ERR_CAPACITY
     assert lemo.lemo_get_error() == lemo.LEMO_OK  # nothing was enqueued
+
+
+def _random_scores_layer(lengths, seed):
+    """A Layer for `lengths` (block size 64) with seeded random block scores on
+    the device; selection needs nothing else."""
+    import torch
+    from contextual_token_sparsity_b200.pipeline import Layer
+    layer = Layer(lengths, 1, 64, 64, d=8)
+    rng = np.random.default_rng(seed)
+    s = rng.standard_normal(max(layer.total_blocks, 1)).astype(np.float32)
+    layer.block_scores.copy_(torch.from_numpy(s))
+    return layer, s[: layer.total_blocks].astype(np.float64)
+
+
+def _compare_calls(layer, theta):
+    batch = len(layer.lengths)
+    ref = _outputs(layer, layer.total_blocks, layer.total_L, batch)
+    got = _outputs(layer, layer.total_blocks, layer.total_L, batch)
+    lemo.lemo_select(layer.shape, layer.block_scores, theta, ref["mask"], ref["kept_idx"],
+                     ref["cu_kept"], ref["kept_total"], layer.ws)
+    lemo.lemo_select_static_ws(layer.shape, layer.block_scores, theta, got["mask"],
+                               got["kept_idx"], got["cu_kept"], got["kept_total"])
+    assert lemo.lemo_get_error() == lemo.LEMO_OK
+    m_ref, K_ref, i_ref, c_ref = _host(ref, layer.total_blocks)
+    m_got, K_got, i_got, c_got = _host(got, layer.total_blocks)
+    assert K_got == K_ref > 0
+    assert np.array_equal(m_got, m_ref)
+    assert np.array_equal(i_got, i_ref)
+    assert np.array_equal(c_got, c_ref)
+
+
+def test_static_workspace_select_at_its_documented_limits():
+    """batch = 4096 sequences (some empty) holding exactly 2^24 tokens: the
+    largest shape the fixed array is documented to hold (plan arrays of 4097
+    entries and 8192 look-back descriptors)."""
+    rng = np.random.default_rng(41)
+    lengths = rng.integers(1, 8192, 4096)
+    lengths[rng.choice(4096, 300, replace=False)] = 0
+    lengths = np.floor(lengths * ((1 << 24) / lengths.sum())).astype(np.int64)
+    lengths[np.argmax(lengths)] += (1 << 24) - int(lengths.sum())
+    assert lengths.sum() == 1 << 24 and (lengths == 0).sum() >= 300
+    layer, s = _random_scores_layer(lengths.tolist(), seed=42)
+    for theta in (float(np.median(s)), float(np.quantile(s, 0.9))):  # two calls in a row
+        _compare_calls(layer, theta)
+
+
+def test_static_workspace_select_times_out_and_recovers():
+    """A compaction tile withholds its look-back descriptor (test hook): the
+    tiles after it give up after the shortened bounded wait, the call reports
+    LEMO_ERR_TIMEOUT and leaves K = 0.  The next call on the same shared array
+    matches lemo_select, so each call re-initialises the look-back state."""
+    import torch
+    layer, s = _random_scores_layer([9000, 5000], seed=43)
+    kept_total = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    try:
+        lemo.lemo_set_test_hooks(select_skip_publish_tile=1, spin_limit_ns=50_000_000)
+        lemo.lemo_select_static_ws(layer.shape, layer.block_scores, float(np.min(s)),
+                                   layer.mask, layer.kept_idx, layer.cu_kept, kept_total)
+        assert lemo.lemo_get_error() == lemo.LEMO_ERR_TIMEOUT
+        assert int(kept_total.item()) == 0
+    finally:
+        lemo.lemo_set_test_hooks(-1, 0)
+    _compare_calls(layer, float(np.median(s)))
