@@ -679,13 +679,13 @@ def run_segloss(args):
                    "vocab": V, "segment_rows": S, "segments": -(-T // S),
                    "l2": "not flushed; each step streams the 262 MB lm-head weight 48 times",
                    "parallelism": f"{world} independent replica(s), no collective"},
-        "roofline": {"bound": "tensor", "kernel": "whole call (3 cuBLAS GEMMs + row kernel per "
+        "roofline": {"bound": "tensor", "kernel": "whole call (3 tcgen05 GEMMs + row kernel per "
                      "segment)", "achieved": round(ach, 1), "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": round(ach / peak_tf, 4), "traffic": None,
                      "algorithmic_flops_per_call": flops},
         "peak_memory": {"workspace_bytes": ws.numel(), "unsegmented_workspace_bytes": full_ws},
         "loss": float(loss.item()),
-        "gpu_launches": (2 + -(-T // S)) * args.steps,
+        "gpu_launches": (2 + 4 * -(-T // S)) * args.steps,
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

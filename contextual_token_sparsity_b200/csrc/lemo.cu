@@ -2,11 +2,9 @@
 // tensor-map encoding and launches.  The kernels live in the included .cuh
 // files; everything is one translation unit so that the device error word is
 // a single symbol per device.
-#include <cublas_v2.h>  // types only: cuBLAS itself is opened with dlopen on first use
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
-#include <dlfcn.h>
 
 #include <climits>
 #include <mutex>
@@ -15,6 +13,7 @@
 #include "lemo.h"
 #include "attn.cuh"
 #include "common.cuh"
+#include "gemm.cuh"
 #include "mlp.cuh"
 #include "move.cuh"
 #include "predict.cuh"
@@ -121,9 +120,9 @@ lemo_status check_ws(const lemo_shape* s, const void* ws, size_t ws_bytes) {
 }
 
 void launch_plan(const lemo_shape* s, char* ws, const lemo::WsLayout& lay, int32_t* zero_word,
-                 cudaStream_t st, float* zero_blocks = nullptr) {
+                 cudaStream_t st, float* zero_blocks = nullptr, int shard = 0, int nshards = 1) {
     launch(lemo::plan_kernel, 1, 1024, 0, st, s->cu_seqlens, s->batch, s->total_L, s->max_seqlen,
-           s->block, ws, lay, zero_word, zero_blocks);
+           s->block, ws, lay, zero_word, zero_blocks, shard, nshards);
 }
 
 // 3-D view of a [rows, H*dh] bf16 matrix as (64 elements, rows, H*dh/64
@@ -231,69 +230,71 @@ lemo_status check_move(const void* x, int64_t ld_x, int64_t x_rows, int32_t d, c
 // region holds the block products P) followed by the predictor buffers.
 struct PredictLayout {
     lemo::WsLayout base;
-    // byte offsets: block-mean planes, padded weight planes, split-K
-    // partials, hidden-activation planes, Qhat / Khat planes, partial products
-    size_t xb_hi, xb_lo, w1p[2], w2p[2], part, hid_hi, hid_lo, q_hi, q_lo, k_hi, k_lo, ppart, total;
-    int ldr;         // rank padded to a multiple of 8
-    int ldh;         // head dimension padded to a multiple of 8
+    // byte offsets: block-mean images, split-K partials, hidden-activation
+    // images, Qhat / Khat images, head-group partial products, barrier words
+    size_t xb, part, hid, qk, ppart, sync, total;
     int64_t tb;      // upper bound of the number of token blocks
-    int splits;      // split-K factor of the first predictor GEMM
-    int k_chunk;     // K range of one split
-    int hpg;         // heads per group of the block products
-    int groups;      // head groups (partial planes when > 1)
-    int64_t ptiles;  // lower-triangular 64 x 64 tiles of block pairs
+    int rt, tba;     // row tiles of 128 token blocks
+    int kc, kc2;     // 64-column chunks of d and of the rank
+    int ldr, nj, nt; // rank padded to 32, n tiles of the first GEMM and their width
+    int zk, cps;     // K splits of the first GEMM, chunks per split
+    int dhp, dc;     // head dimension padded to 64, its chunks
+    int np, nj2;     // H * dhp and its 256-column tiles
+    int pt, groups, hpg;
+    bool fits;       // every unit count fits in 32 bits
 };
 
 // The launch shapes depend only on the shape (not on the device), so the
 // workspace size query and the call agree.  The first GEMM is split along K
-// until about four CTAs per SM of a B200 (148 SMs) are busy, with at least
-// four K stages each: its loop is latency-bound, so shorter loops on more
-// SMs finish sooner.  The block products aim at two CTAs per SM.
+// so that about one unit per SM of a B200 (148 SMs) is busy; the block
+// products take one head group per unit, as many groups as keep the SMs busy.
 PredictLayout predict_layout(const lemo_shape* s, int d, int rank) {
     namespace pr = lemo::predict;
-    constexpr int64_t kGemmCtas = 592, kTargetCtas = 296;
+    constexpr int64_t kTarget = 148;
     PredictLayout p;
     p.base = layout_of(s);
     p.tb = ((int64_t)s->total_L + (int64_t)s->batch * (s->block - 1)) / s->block;
     if (p.tb < 1) p.tb = 1;
-    p.ldr = (rank + 7) / 8 * 8;
-    p.ldh = (s->dh + 7) / 8 * 8;
-    const int64_t hdp = (int64_t)s->H * p.ldh;
-    const int64_t mt = (p.tb + pr::TM - 1) / pr::TM;
-    const int64_t tiles = 2 * ((p.ldr + pr::TN - 1) / pr::TN) * mt;
-    const int64_t kst = (d + pr::TK - 1) / pr::TK;        // K stages of the first GEMM
-    int64_t splits = (kGemmCtas + tiles - 1) / tiles;
-    const int64_t max_splits = (kst + 3) / 4;              // at least 4 stages per split
-    if (splits > max_splits) splits = max_splits;
-    if (splits < 1) splits = 1;
-    p.k_chunk = (int)((kst + splits - 1) / splits * pr::TK);
-    p.splits = (int)((d + p.k_chunk - 1) / p.k_chunk);
-    p.ptiles = mt * (mt + 1) / 2;
-    int64_t groups = (kTargetCtas + p.ptiles - 1) / p.ptiles;
+    const int64_t rt = (p.tb + pr::TILE - 1) / pr::TILE;
+    p.rt = (int)rt;
+    p.tba = (int)(rt * pr::TILE);
+    p.kc = (d + pr::KCH - 1) / pr::KCH;
+    p.kc2 = (rank + pr::KCH - 1) / pr::KCH;
+    p.ldr = (rank + 31) / 32 * 32;
+    p.nj = (p.ldr + pr::MAX_NT - 1) / pr::MAX_NT;
+    p.nt = ((p.ldr + p.nj - 1) / p.nj + 31) / 32 * 32;
+    const int64_t base_units = 2 * rt * p.nj;
+    int64_t cps = (p.kc * base_units + kTarget - 1) / kTarget;
+    if (cps < 1) cps = 1;
+    p.cps = (int)cps;
+    p.zk = (int)((p.kc + cps - 1) / cps);
+    p.dhp = (s->dh + pr::KCH - 1) / pr::KCH * pr::KCH;
+    p.dc = p.dhp / pr::KCH;
+    p.np = s->H * p.dhp;
+    p.nj2 = (p.np + pr::MAX_NT - 1) / pr::MAX_NT;
+    const int64_t pt = rt * (rt + 1) / 2;
+    p.pt = (int)(pt < INT_MAX ? pt : INT_MAX);
+    int64_t groups = (kTarget + pt - 1) / pt;
     if (groups > s->H) groups = s->H;
-    while (groups > 1 && groups * p.tb * p.tb * 4 > ((int64_t)64 << 20)) --groups;
+    while (groups > 1 && groups * (int64_t)p.tba * p.tba * 4 > ((int64_t)64 << 20)) --groups;
     if (groups < 1) groups = 1;
     p.hpg = (int)((s->H + groups - 1) / groups);
     p.groups = (s->H + p.hpg - 1) / p.hpg;
+    p.fits = base_units * p.zk < INT_MAX && 2 * rt * p.nj2 < INT_MAX &&
+             pt * p.groups < INT_MAX && (int64_t)p.tba * p.tba < ((int64_t)1 << 40);
     size_t off = p.base.total;
     auto take = [&](size_t bytes) {
         const size_t o = off;
         off = lemo::align_up(off + bytes, 256);
         return o;
     };
-    p.xb_hi = take(2 * (size_t)p.tb * d);
-    p.xb_lo = take(2 * (size_t)p.tb * d);
-    for (int i = 0; i < 2; ++i) p.w1p[i] = take(2 * (size_t)d * p.ldr);
-    for (int i = 0; i < 2; ++i) p.w2p[i] = take(2 * (size_t)p.ldr * hdp);
-    p.part = take(4 * (size_t)2 * p.splits * p.tb * p.ldr);
-    p.hid_hi = take(2 * (size_t)2 * p.tb * p.ldr);
-    p.hid_lo = take(2 * (size_t)2 * p.tb * p.ldr);
-    p.q_hi = take(2 * (size_t)p.tb * hdp);
-    p.q_lo = take(2 * (size_t)p.tb * hdp);
-    p.k_hi = take(2 * (size_t)p.tb * hdp);
-    p.k_lo = take(2 * (size_t)p.tb * hdp);
+    p.sync = take(4 * pr::kSyncWords);
+    p.xb = take((size_t)rt * p.kc * 2 * pr::IMG);
+    p.part = take(4 * (size_t)2 * p.zk * p.tba * p.ldr);
+    p.hid = take((size_t)2 * rt * p.kc2 * 2 * pr::IMG);
+    p.qk = take((size_t)2 * rt * s->H * p.dc * 2 * pr::IMG);
     p.ppart = off;
-    if (p.groups > 1) off = lemo::align_up(off + 4 * (size_t)p.groups * p.tb * p.tb, 256);
+    if (p.groups > 1) off = lemo::align_up(off + 4 * (size_t)p.groups * p.tba * p.tba, 256);
     p.total = off;
     return p;
 }
@@ -308,50 +309,9 @@ lemo_status check_predict(const lemo_shape* s, int d, int rank) {
     return LEMO_OK;
 }
 
-// ---------------------------------------------------------------------------
-// cuBLAS for the plain GEMMs of the segmented loss, opened on first use so
-// that the rest of the library does not depend on it.
-// ---------------------------------------------------------------------------
-struct Blas {
-    using Create = cublasStatus_t (*)(cublasHandle_t*);
-    using SetStream = cublasStatus_t (*)(cublasHandle_t, cudaStream_t);
-    using SetWorkspace = cublasStatus_t (*)(cublasHandle_t, void*, size_t);
-    using GemmEx = cublasStatus_t (*)(cublasHandle_t, cublasOperation_t, cublasOperation_t, int, int,
-                                      int, const void*, const void*, cudaDataType, int, const void*,
-                                      cudaDataType, int, const void*, void*, cudaDataType, int,
-                                      cublasComputeType_t, cublasGemmAlgo_t);
-    bool tried = false;
-    Create create = nullptr;
-    SetStream set_stream = nullptr;
-    SetWorkspace set_workspace = nullptr;
-    GemmEx gemm = nullptr;
-    cublasHandle_t handle[kMaxDevices] = {};
-};
-Blas g_blas;
-constexpr size_t kBlasWorkspace = 32u << 20;
-
-// Handle of device `dev` (created on first use), or nullptr if cuBLAS is
-// unavailable.  Caller holds g_mu.
-cublasHandle_t blas_handle(int dev) {
-    Blas& b = g_blas;
-    if (!b.tried) {
-        b.tried = true;
-        void* lib = dlopen("libcublas.so.12", RTLD_NOW | RTLD_GLOBAL);
-        if (lib) {
-            b.create = reinterpret_cast<Blas::Create>(dlsym(lib, "cublasCreate_v2"));
-            b.set_stream = reinterpret_cast<Blas::SetStream>(dlsym(lib, "cublasSetStream_v2"));
-            b.set_workspace = reinterpret_cast<Blas::SetWorkspace>(dlsym(lib, "cublasSetWorkspace_v2"));
-            b.gemm = reinterpret_cast<Blas::GemmEx>(dlsym(lib, "cublasGemmEx"));
-        }
-    }
-    if (!b.create || !b.set_stream || !b.set_workspace || !b.gemm) return nullptr;
-    if (!b.handle[dev] && b.create(&b.handle[dev]) != CUBLAS_STATUS_SUCCESS) b.handle[dev] = nullptr;
-    return b.handle[dev];
-}
-
 // Workspace of lemo_segment_loss.
 struct SegLayout {
-    size_t n_valid, token_loss, blas, z, g, total;
+    size_t n_valid, token_loss, z, g, total;
     int64_t ld;    // row stride of the segment's logits and gradient
     int64_t rows;  // rows of one segment buffer
 };
@@ -363,7 +323,6 @@ SegLayout seg_layout(int64_t T, int V, int seg_rows) {
     size_t off = 0;
     l.n_valid = off; off = lemo::align_up(off + 4, 256);
     l.token_loss = off; off = lemo::align_up(off + 4 * (size_t)(T > 0 ? T : 1), 256);
-    l.blas = off; off = lemo::align_up(off + kBlasWorkspace, 256);
     l.z = off; off = lemo::align_up(off + 4 * (size_t)l.rows * l.ld, 256);
     l.g = off; off = lemo::align_up(off + 2 * (size_t)l.rows * l.ld, 256);
     l.total = off;
@@ -372,6 +331,92 @@ SegLayout seg_layout(int64_t T, int V, int seg_rows) {
 
 bool seg_args_ok(int64_t T, int V, int seg_rows) {
     return T >= 0 && T <= INT_MAX && V >= 1 && seg_rows >= 1 && (int64_t)V + 7 <= INT_MAX;
+}
+
+// 2-D tensor map of a bf16 matrix [rows, cols] with row stride ld elements,
+// 128-byte swizzle: K-major operands (cols = K) take boxes of 64 x 128,
+// MN-major operands (rows = K, cols = M or N) boxes of 64 x 64.
+bool encode_operand(CUtensorMap* tm, const uint16_t* base, int64_t rows, int64_t cols, int64_t ld,
+                    bool mn_major) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
+    const cuuint32_t box[2] = {(cuuint32_t)lemo::gemm::KB,
+                               (cuuint32_t)(mn_major ? lemo::gemm::KB : lemo::gemm::ROWS)};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(base), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+// CTA pairs of the GEMM kernel that fit at once (sets its shared-memory
+// limit on first use).
+int g_gemm_pairs[kMaxDevices];
+
+int gemm_pairs(int dev, int sms) {
+    namespace gm = lemo::gemm;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_gemm_pairs[dev] == 0) {
+        if (cudaFuncSetAttribute(gm::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 gm::SMEM_BYTES) != cudaSuccess)
+            return 0;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
+        cfg.blockDim = dim3(gm::THREADS, 1, 1);
+        cfg.dynamicSmemBytes = gm::SMEM_BYTES;
+        cudaLaunchAttribute attr;
+        attr.id = cudaLaunchAttributeClusterDimension;
+        attr.val.clusterDim.x = 2;
+        attr.val.clusterDim.y = 1;
+        attr.val.clusterDim.z = 1;
+        cfg.attrs = &attr;
+        cfg.numAttrs = 1;
+        int clusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&clusters, gm::gemm_kernel, &cfg) != cudaSuccess ||
+            clusters < 1) {
+            cudaGetLastError();
+            clusters = sms / 2;
+        }
+        g_gemm_pairs[dev] = clusters < sms / 2 ? clusters : sms / 2;
+    }
+    return g_gemm_pairs[dev];
+}
+
+// C[M, N] (=, or += for kAddF32) A[M, K] B[K, N] on the tensor cores.
+// a_mn / b_mn: the operand's M / N index is the contiguous one in memory.
+lemo_status run_gemm(int dev, int sms, cudaStream_t st, const uint16_t* A, int64_t lda, bool a_mn,
+                     const uint16_t* B, int64_t ldb, bool b_mn, int M, int N, int K, int epi,
+                     void* out, int64_t ld_out, bool m_fastest) {
+    namespace gm = lemo::gemm;
+    if (M <= 0 || N <= 0) return LEMO_OK;
+    CUtensorMap ta, tb;
+    if (!encode_operand(&ta, A, a_mn ? K : M, a_mn ? M : K, lda, a_mn) ||
+        !encode_operand(&tb, B, b_mn ? K : N, b_mn ? N : K, ldb, b_mn))
+        return LEMO_ERR_CUDA;
+    const int pairs = gemm_pairs(dev, sms);
+    if (pairs <= 0) return LEMO_ERR_CUDA;
+    gm::Args a;
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.a_mn = a_mn ? 1 : 0;
+    a.b_mn = b_mn ? 1 : 0;
+    a.epi = epi;
+    a.out = out;
+    a.ld_out = ld_out;
+    a.tiles_m = (M + gm::TM - 1) / gm::TM;
+    a.tiles_n = (N + gm::TN - 1) / gm::TN;
+    a.m_fastest = m_fastest ? 1 : 0;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        a.spin_limit_ns = (uint64_t)g_spin_ns;
+    }
+    const int64_t tiles = (int64_t)a.tiles_m * a.tiles_n;
+    const int64_t use = tiles < pairs ? tiles : pairs;
+    launch(gm::gemm_kernel, (unsigned)(2 * use), gm::THREADS, gm::SMEM_BYTES, st, ta, tb, a);
+    return launch_status();
 }
 
 }  // namespace
@@ -406,9 +451,13 @@ int64_t lemo_block_max_elems(int32_t batch, const int32_t* lengths_host, int32_t
     return n;
 }
 
-lemo_status lemo_score_blocks(const lemo_shape* shape, const uint16_t* q, const uint16_t* k,
-                              float scale, float* block_max, float* block_scores, void* ws,
-                              size_t ws_bytes, lemo_stream stream) {
+}  // extern "C"
+
+namespace {
+
+lemo_status score_blocks(const lemo_shape* shape, const uint16_t* q, const uint16_t* k, float scale,
+                         int shard, int nshards, float* block_max, float* block_scores, void* ws,
+                         size_t ws_bytes, lemo_stream stream) {
     lemo_status e = check_shape(shape, true);
     if (e != LEMO_OK) return e;
     if (!q || !k || !block_scores) return LEMO_ERR_INVALID_ARG;
@@ -416,6 +465,7 @@ lemo_status lemo_score_blocks(const lemo_shape* shape, const uint16_t* q, const 
         (block_max && !aligned(block_max, 4)))
         return LEMO_ERR_INVALID_ARG;
     if (!(scale > 0.f) || scale == __builtin_inff()) return LEMO_ERR_INVALID_ARG;
+    if (nshards < 1 || nshards > 4096 || shard < 0 || shard >= nshards) return LEMO_ERR_INVALID_ARG;
     if ((e = check_ws(shape, ws, ws_bytes)) != LEMO_OK) return e;
     int dev = 0;
     const int sms = device_sms(&dev);
@@ -425,7 +475,7 @@ lemo_status lemo_score_blocks(const lemo_shape* shape, const uint16_t* q, const 
     char* w = static_cast<char*>(ws);
     float* mblk = block_max ? block_max : reinterpret_cast<float*>(w + lay.mblk);
 
-    launch_plan(shape, w, lay, nullptr, st);
+    launch_plan(shape, w, lay, nullptr, st, nullptr, shard, nshards);
     if ((e = launch_status()) != LEMO_OK) return e;
     if (shape->total_L > 0) {
         namespace sc = lemo::score;
@@ -447,6 +497,8 @@ lemo_status lemo_score_blocks(const lemo_shape* shape, const uint16_t* q, const 
         a.ws = w;
         a.lay = lay;
         a.spin_limit_ns = (uint64_t)g_spin_ns;
+        a.shard = shard;
+        a.nshards = nshards;
         launch(sc::score_tiles_kernel, 2 * pairs, sc::THREADS, sc::SMEM_BYTES, st, tm_q, tm_k, a);
         if ((e = launch_status()) != LEMO_OK) return e;
         // one warp per token block; the host knows an upper bound of their number
@@ -455,10 +507,28 @@ lemo_status lemo_score_blocks(const lemo_shape* shape, const uint16_t* q, const 
         const int64_t cs_ctas = (nb_bound + 7) / 8;
         const int cs_grid = (int)(cs_ctas < (int64_t)sms * 8 ? (cs_ctas > 0 ? cs_ctas : 1) : sms * 8);
         launch(sc::column_sum_kernel, cs_grid, 256, 0, st, mblk, w, lay, shape->batch,
-               block_scores);
+               block_scores, shape->block, shard, nshards);
         if ((e = launch_status()) != LEMO_OK) return e;
     }
     return LEMO_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+lemo_status lemo_score_blocks(const lemo_shape* shape, const uint16_t* q, const uint16_t* k,
+                              float scale, float* block_max, float* block_scores, void* ws,
+                              size_t ws_bytes, lemo_stream stream) {
+    return score_blocks(shape, q, k, scale, 0, 1, block_max, block_scores, ws, ws_bytes, stream);
+}
+
+lemo_status lemo_score_blocks_shard(const lemo_shape* shape, const uint16_t* q, const uint16_t* k,
+                                    float scale, int32_t shard, int32_t nshards, float* block_max,
+                                    float* block_scores, void* ws, size_t ws_bytes,
+                                    lemo_stream stream) {
+    return score_blocks(shape, q, k, scale, shard, nshards, block_max, block_scores, ws, ws_bytes,
+                        stream);
 }
 
 lemo_status lemo_select(const lemo_shape* shape, const float* block_scores, float threshold,
@@ -696,6 +766,7 @@ lemo_status lemo_predict_scores(const lemo_shape* shape, int32_t d, const uint16
         !aligned(w1k, 2) || !aligned(w2k, 2) || !aligned(block_scores, 4) || !aligned(ws, 256))
         return LEMO_ERR_INVALID_ARG;
     const PredictLayout p = predict_layout(shape, d, rank);
+    if (!p.fits) return LEMO_ERR_UNSUPPORTED;
     if (ws_bytes < p.total) return LEMO_ERR_INVALID_ARG;
     int dev = 0;
     const int sms = device_sms(&dev);
@@ -703,140 +774,81 @@ lemo_status lemo_predict_scores(const lemo_shape* shape, int32_t d, const uint16
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     char* w = static_cast<char*>(ws);
     const lemo::WsLayout& lay = p.base;
-    const lemo::PlanHeader* hdr = reinterpret_cast<const lemo::PlanHeader*>(w + lay.hdr);
-    float* part = reinterpret_cast<float*>(w + p.part);
-    float* P = reinterpret_cast<float*>(w + lay.mblk);
-    auto plane = [&](size_t off) { return reinterpret_cast<uint16_t*>(w + off); };
-    const int hdp = shape->H * p.ldh;  // columns of the Qhat / Khat planes (heads padded)
+    uint32_t* sync = reinterpret_cast<uint32_t*>(w + p.sync);
 
     launch_plan(shape, w, lay, nullptr, st);
     if ((e = launch_status()) != LEMO_OK) return e;
     if (shape->total_L == 0) return LEMO_OK;
-    // weights whose rows are not 16-byte aligned: padded copies
-    const bool w1_vec16 = rank % 8 == 0 && aligned(w1q, 16) && aligned(w1k, 16);
-    const bool w1_vec4 = !w1_vec16 && rank % 2 == 0 && aligned(w1q, 4) && aligned(w1k, 4);
-    const bool pad_w1 = !w1_vec16 && !w1_vec4;
-    const bool pad_w2 = shape->dh % 8 != 0 || !aligned(w2q, 16) || !aligned(w2k, 16);
-    if (pad_w1) {
-        pr::PadArgs pa1 = {};
-        pa1.src[0] = w1q;
-        pa1.src[1] = w1k;
-        pa1.dst[0] = plane(p.w1p[0]);
-        pa1.dst[1] = plane(p.w1p[1]);
-        pa1.rows = pa1.rows_out = d;
-        pa1.cols = pa1.run = rank;
-        pa1.run_ld = p.ldr;
-        pa1.ld_out = p.ldr;
-        launch(pr::pad_kernel, dim3((unsigned)((d + 7) / 8), 2u), 256, 0, st, pa1);
-    }
-    if (pad_w2) {
-        pr::PadArgs pa2 = {};
-        pa2.src[0] = w2q;
-        pa2.src[1] = w2k;
-        pa2.dst[0] = plane(p.w2p[0]);
-        pa2.dst[1] = plane(p.w2p[1]);
-        pa2.rows = pa2.rows_out = rank;
-        pa2.cols = shape->H * shape->dh;
-        pa2.run = shape->dh;
-        pa2.run_ld = p.ldh;
-        pa2.ld_out = hdp;
-        launch(pr::pad_kernel, dim3((unsigned)((rank + 7) / 8), 2u), 256, 0, st, pa2);
-    }
-    const uint16_t* w1s[2] = {pad_w1 ? plane(p.w1p[0]) : w1q, pad_w1 ? plane(p.w1p[1]) : w1k};
-    const uint16_t* w2s[2] = {pad_w2 ? plane(p.w2p[0]) : w2q, pad_w2 ? plane(p.w2p[1]) : w2k};
-    // block means, as hi / lo planes
-    launch(pr::pool_kernel,
-           dim3((unsigned)p.tb, (unsigned)((d + pr::kPoolCols - 1) / pr::kPoolCols)),
-           pr::kPoolThreads, 0, st, x, ld_x, d, shape->cu_seqlens, shape->batch, shape->block, w,
-           lay, plane(p.xb_hi), plane(p.xb_lo));
-    if ((e = launch_status()) != LEMO_OK) return e;
-    const unsigned mtiles = (unsigned)((p.tb + pr::TM - 1) / pr::TM);
-    // hidden layers of both predictors: split-K partials, then relu of their sum
-    pr::GemmArgs g1 = {};
-    g1.a_hi[0] = g1.a_hi[1] = plane(p.xb_hi);
-    g1.a_lo[0] = g1.a_lo[1] = plane(p.xb_lo);
-    g1.lda = d;
-    g1.w[0] = w1s[0];
-    g1.w[1] = w1s[1];
-    g1.ldw = pad_w1 ? p.ldr : rank;
-    g1.c[0] = part;
-    g1.c[1] = part + (int64_t)p.splits * p.tb * p.ldr;
-    g1.ldc = p.ldr;
-    g1.c_split = p.tb * p.ldr;
-    g1.hdr = hdr;
-    g1.N = p.ldr;
-    g1.K = d;
-    g1.w_rows = d;
-    g1.w_cols = pad_w1 ? p.ldr : rank;
-    g1.w_vec4 = w1_vec4;
-    g1.k_chunk = p.k_chunk;
-    g1.splits = p.splits;
-    launch(pr::gemm_kernel<false>,
-           dim3((unsigned)((p.ldr + pr::TN - 1) / pr::TN), mtiles, 2u * p.splits), pr::kMmaThreads,
-           0, st, g1);
-    launch(pr::reduce_kernel, dim3((unsigned)sms, 2u), 256, 0, st, part,
-           (int64_t)p.splits * p.tb * p.ldr, p.tb * p.ldr, p.splits, hdr, p.ldr, plane(p.hid_hi),
-           plane(p.hid_lo), p.tb * p.ldr);
-    // block embeddings of both predictors, as hi / lo planes
-    pr::GemmArgs g2 = {};
-    g2.a_hi[0] = plane(p.hid_hi);
-    g2.a_hi[1] = plane(p.hid_hi) + p.tb * p.ldr;
-    g2.a_lo[0] = plane(p.hid_lo);
-    g2.a_lo[1] = plane(p.hid_lo) + p.tb * p.ldr;
-    g2.lda = p.ldr;
-    g2.w[0] = w2s[0];
-    g2.w[1] = w2s[1];
-    g2.ldw = hdp;
-    g2.c_hi[0] = plane(p.q_hi);
-    g2.c_lo[0] = plane(p.q_lo);
-    g2.c_hi[1] = plane(p.k_hi);
-    g2.c_lo[1] = plane(p.k_lo);
-    g2.ldc = hdp;
-    g2.c_split = 0;
-    g2.hdr = hdr;
-    g2.N = hdp;
-    g2.K = p.ldr;
-    g2.w_rows = rank;
-    g2.w_cols = hdp;
-    g2.w_vec4 = false;
-    g2.k_chunk = (p.ldr + pr::TK - 1) / pr::TK * pr::TK;
-    g2.splits = 1;
-    launch(pr::gemm_kernel<true>, dim3((unsigned)((hdp + pr::TN - 1) / pr::TN), mtiles, 2u),
-           pr::kMmaThreads, 0, st, g2);
-    if ((e = launch_status()) != LEMO_OK) return e;
-    // block products, mean over heads of the positive parts
-    pr::ProductsArgs pa;
-    pa.q_hi = plane(p.q_hi);
-    pa.q_lo = plane(p.q_lo);
-    pa.k_hi = plane(p.k_hi);
-    pa.k_lo = plane(p.k_lo);
-    pa.H = shape->H;
-    pa.ldh = p.ldh;
-    pa.hpg = p.hpg;
-    pa.groups = p.groups;
-    pa.batch = shape->batch;
-    pa.tb_cap = p.tb;
-    pa.inv_h = 1.f / (float)shape->H;
-    pa.part = reinterpret_cast<float*>(w + p.ppart);
-    pa.P = P;
     {
         std::lock_guard<std::mutex> lk(g_mu);
         if (!g_prod_smem_set[dev]) {
-            if (cudaFuncSetAttribute(pr::products_kernel,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     pr::PROD_SMEM) != cudaSuccess)
+            if (cudaFuncSetAttribute(pr::predict_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     pr::SMEM_BYTES) != cudaSuccess)
+                return LEMO_ERR_CUDA;
+            int per_sm = 0;
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, pr::predict_kernel,
+                                                              pr::THREADS, pr::SMEM_BYTES) !=
+                    cudaSuccess ||
+                per_sm < 1)
                 return LEMO_ERR_CUDA;
             g_prod_smem_set[dev] = true;
         }
     }
-    launch(pr::products_kernel, dim3((unsigned)p.ptiles, (unsigned)p.groups), pr::kMmaThreads,
-           pr::PROD_SMEM, st, pa, w, lay);
+    // block means, as hi / lo operand images (and the barrier words cleared)
+    launch(pr::pool_kernel,
+           dim3((unsigned)p.tba, (unsigned)((p.kc * pr::KCH + pr::kPoolCols - 1) / pr::kPoolCols)),
+           pr::kPoolThreads, 0, st, x, ld_x, d, p.kc, shape->cu_seqlens, shape->batch,
+           shape->block, w, lay, reinterpret_cast<uint8_t*>(w + p.xb), sync);
     if ((e = launch_status()) != LEMO_OK) return e;
-    if (p.groups > 1) launch(pr::products_reduce_kernel, sms * 2, 256, 0, st, pa, w, lay);
-    const int64_t cs_ctas = (p.tb + 7) / 8;
-    const int cs_grid = (int)(cs_ctas < (int64_t)sms * 8 ? cs_ctas : sms * 8);
-    launch(lemo::score::column_sum_kernel, cs_grid, 256, 0, st, P, w, lay, shape->batch,
-           block_scores);
+    pr::Args a;
+    a.ws = w;
+    a.lay = lay;
+    a.batch = shape->batch;
+    a.d = d;
+    a.rank = rank;
+    a.H = shape->H;
+    a.dh = shape->dh;
+    a.dhp = p.dhp;
+    a.dc = p.dc;
+    a.rt = p.rt;
+    a.tba = p.tba;
+    a.kc = p.kc;
+    a.kc2 = p.kc2;
+    a.ldr = p.ldr;
+    a.nj = p.nj;
+    a.nt = p.nt;
+    a.zk = p.zk;
+    a.cps = p.cps;
+    a.np = p.np;
+    a.nj2 = p.nj2;
+    a.pt = p.pt;
+    a.groups = p.groups;
+    a.hpg = p.hpg;
+    a.inv_h = 1.f / (float)shape->H;
+    a.w1[0] = w1q;
+    a.w1[1] = w1k;
+    a.w2[0] = w2q;
+    a.w2[1] = w2k;
+    a.w1_mode = (rank % 8 == 0 && aligned(w1q, 16) && aligned(w1k, 16))  ? pr::kW16
+                : (rank % 2 == 0 && aligned(w1q, 4) && aligned(w1k, 4)) ? pr::kW4
+                                                                         : pr::kW2;
+    a.w2_mode = (shape->dh % 8 == 0 && aligned(w2q, 16) && aligned(w2k, 16))  ? pr::kW16
+                : (shape->dh % 2 == 0 && aligned(w2q, 4) && aligned(w2k, 4)) ? pr::kW4
+                                                                              : pr::kW2;
+    a.xb = reinterpret_cast<const uint8_t*>(w + p.xb);
+    a.part = reinterpret_cast<float*>(w + p.part);
+    a.hid = reinterpret_cast<uint8_t*>(w + p.hid);
+    a.qk = reinterpret_cast<uint8_t*>(w + p.qk);
+    a.ppart = reinterpret_cast<float*>(w + p.ppart);
+    a.P = reinterpret_cast<float*>(w + lay.mblk);
+    a.sync = sync;
+    a.scores = block_scores;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        a.spin_limit_ns = (uint64_t)g_spin_ns;
+    }
+    // one persistent CTA per SM (the grid barriers need every CTA resident)
+    launch(pr::predict_kernel, (unsigned)sms, pr::THREADS, pr::SMEM_BYTES, st, a);
     return launch_status();
 }
 
@@ -938,7 +950,8 @@ lemo_status lemo_segment_loss(const uint16_t* h, int64_t ld_h, int64_t T, int32_
     const SegLayout l = seg_layout(T, V, seg_rows);
     if (ws_bytes < l.total) return LEMO_ERR_INVALID_ARG;
     int dev = 0;
-    if (device_sms(&dev) <= 0) return LEMO_ERR_CUDA;
+    const int sms = device_sms(&dev);
+    if (sms <= 0) return LEMO_ERR_CUDA;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     char* wsp = static_cast<char*>(ws);
     int32_t* n_valid = reinterpret_cast<int32_t*>(wsp + l.n_valid);
@@ -946,29 +959,17 @@ lemo_status lemo_segment_loss(const uint16_t* h, int64_t ld_h, int64_t T, int32_
     float* z = reinterpret_cast<float*>(wsp + l.z);
     uint16_t* g = reinterpret_cast<uint16_t*>(wsp + l.g);
 
-    // The handle's stream and workspace are per call: hold the lock until
-    // every GEMM of this call is enqueued.
-    std::lock_guard<std::mutex> lk(g_mu);
-    cublasHandle_t hb = nullptr;
-    if (T > 0) {
-        hb = blas_handle(dev);
-        if (!hb) return LEMO_ERR_UNSUPPORTED;
-        if (g_blas.set_stream(hb, st) != CUBLAS_STATUS_SUCCESS ||
-            g_blas.set_workspace(hb, wsp + l.blas, kBlasWorkspace) != CUBLAS_STATUS_SUCCESS)
-            return LEMO_ERR_CUDA;
-    }
     launch(sl::count_kernel, 1, sl::kCountThreads, 0, st, targets, T, V, ignore_index, n_valid);
     lemo_status e = launch_status();
     if (e != LEMO_OK) return e;
-    const float one = 1.f, zero = 0.f;
+    namespace gm = lemo::gemm;
     for (int64_t s0 = 0; s0 < T; s0 += seg_rows) {
         const int S = (int)(T - s0 < seg_rows ? T - s0 : seg_rows);
         const uint16_t* hs = h + s0 * ld_h;
-        // z^T [V, S] = W [V, d] . h_seg^T   (column-major view of row-major z [S, ld])
-        if (g_blas.gemm(hb, CUBLAS_OP_T, CUBLAS_OP_N, V, S, d, &one, w, CUDA_R_16BF, (int)ld_w, hs,
-                        CUDA_R_16BF, (int)ld_h, &zero, z, CUDA_R_32F, (int)l.ld, CUBLAS_COMPUTE_32F,
-                        CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS)
-            return LEMO_ERR_CUDA;
+        // z [S, V] = h_seg [S, d] . W [V, d]^T  (fp32, row stride l.ld)
+        if ((e = run_gemm(dev, sms, st, hs, ld_h, false, w, ld_w, false, S, V, d, gm::kStoreF32, z,
+                          l.ld, true)) != LEMO_OK)
+            return e;
         sl::RowArgs a;
         a.z = z;
         a.ldz = l.ld;
@@ -981,17 +982,14 @@ lemo_status lemo_segment_loss(const uint16_t* h, int64_t ld_h, int64_t T, int32_
         a.ignore = ignore_index;
         launch(sl::row_kernel, S, sl::kRowThreads, 0, st, a);
         if ((e = launch_status()) != LEMO_OK) return e;
-        // dh_seg^T [d, S] = W^T [d, V] . dz^T [V, S]
-        if (dh && g_blas.gemm(hb, CUBLAS_OP_N, CUBLAS_OP_N, d, S, V, &one, w, CUDA_R_16BF, (int)ld_w,
-                              g, CUDA_R_16BF, (int)l.ld, &zero, dh + s0 * ld_dh, CUDA_R_16BF,
-                              (int)ld_dh, CUBLAS_COMPUTE_32F,
-                              CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS)
-            return LEMO_ERR_CUDA;
-        // dW^T [d, V] += h_seg^T [d, S] . dz [S, V]
-        if (dw && g_blas.gemm(hb, CUBLAS_OP_N, CUBLAS_OP_T, d, V, S, &one, hs, CUDA_R_16BF, (int)ld_h,
-                              g, CUDA_R_16BF, (int)l.ld, &one, dw, CUDA_R_32F, (int)ld_dw,
-                              CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS)
-            return LEMO_ERR_CUDA;
+        // dh_seg [S, d] = dz [S, V] . W [V, d]  (W read N-contiguous: MN-major B)
+        if (dh && (e = run_gemm(dev, sms, st, g, l.ld, false, w, ld_w, true, S, d, V,
+                                gm::kStoreBF16, dh + s0 * ld_dh, ld_dh, true)) != LEMO_OK)
+            return e;
+        // dW [V, d] += dz^T [V, S] . h_seg [S, d]  (both read MN-major)
+        if (dw && (e = run_gemm(dev, sms, st, g, l.ld, true, hs, ld_h, true, V, d, S,
+                                gm::kAddF32, dw, ld_dw, false)) != LEMO_OK)
+            return e;
     }
     launch(sl::loss_kernel, 1, sl::kCountThreads, 0, st, tl, T, n_valid, loss);
     return launch_status();

@@ -6,37 +6,105 @@
 //   P[n][m]  = (1/H) sum_h max(Qhat_n^h . Khat_m^h, 0),  n >= m          (block products)
 //   score[m] = sum_{n >= m} P[n][m]                                      (column sum)
 //
-// The pooling pass streams X once and is bound by HBM bandwidth.  The
-// predictor GEMMs and the block products are small (about 2 GFLOP at 32K
-// tokens, one representative per block) and bound by latency, so they run
-// as register-tiled warp-level tensor-core MMAs (m16n8k16, bf16 operands,
-// fp32 accumulation) rather than as TMEM tiles sized for large problems.
-// fp32 values are split into two bf16 parts, v = hi + lo with
-// hi = bf16(v) and lo = bf16(v - hi); a product a.b is taken as
-// a_hi b_hi + a_lo b_hi + a_hi b_lo (the weights are bf16 already, so for
-// the GEMMs only a_hi b + a_lo b is needed).  The dropped term is below
-// 2^-16 of each product, so a score's error is about 2^-16 of the sum of
-// the magnitudes of its products: near fp32 accuracy, except where a block
-// pair's dot products cancel (then it stays small against the scores'
-// scale, not against that one score).
+// Two kernels after the per-call plan:
 //
-// Every fp32 intermediate (block means, hidden activations, Qhat, Khat) is
-// split once, by the kernel that produces it, and stored as two bf16 planes
-// whose rows are padded to a multiple of 8 elements.  Every operand of every
-// MMA kernel is read with cp.async (16-byte chunks; 4-byte ones for weight
-// rows that are only 4-byte aligned; weights with odd row lengths are first
-// copied into padded planes) through a shared-memory pipeline, zero-filled
-// outside the matrix, and taken into registers with ldmatrix.  Split-K partial sums and
-// per-head-group partial products are reduced in a fixed order: results
-// are the same bits on every run.
+//   pool_kernel     streams X once (bound by HBM bandwidth) and writes the
+//                   block means as bf16 hi / lo planes already laid out as
+//                   tensor-core operand tiles;
+//   predict_kernel  one persistent CTA per SM runs everything else as
+//                   phases separated by grid-wide barriers:
+//                     A  split-K partial products xbar W1 (both predictors)
+//                     B  sum of the split-K partials, ReLU, hi / lo split
+//                     C  the hidden activations times W2 -> Qhat, Khat tiles
+//                     D  Eq. 3 block products, positive part per head
+//                     E  sum over head groups (when there are several), then
+//                        the column sums.
+//
+// Every contraction runs on the tensor cores: tcgen05.mma (cta_group::1,
+// M = 128, kind::f16, bf16 operands from shared memory, fp32 accumulators in
+// tensor memory, read back with tcgen05.ld).  fp32 operands are split into
+// two bf16 parts, v = hi + lo with hi = bf16(v) and lo = bf16(v - hi), and a
+// product a.b is taken as a_hi b_hi + a_lo b_hi + a_hi b_lo in one fp32
+// accumulator (a_hi b + a_lo b when b is a bf16 weight).  The dropped term is
+// below 2^-16 of each product, so scores keep about fp32 accuracy.
+//
+// Operand tiles ("images") are [128 rows x 64] bf16 K-major blocks of 16 KB
+// in the layout a 128-byte-swizzled TMA box would have: 8-row groups of 1024
+// bytes, row r at 128 (r % 8), its 16-byte chunk j at (j ^ (r % 8)) * 16.
+// Every intermediate is written by its producer directly in that layout, so
+// a consumer fetches a whole tile with one bulk copy (cp.async.bulk, no
+// tensor map).  The weights are read with plain loads (any 2-byte alignment)
+// into MN-major swizzled tiles: 64 rows of K, 64-column groups 8 KB apart.
+//
+// Per CTA: warp 0 issues the bulk copies into a 3-stage ring of 64 KB,
+// warp 1 issues the MMAs into two 256-column accumulators, warps 2-9 load
+// the weight tiles, run the epilogues and the reductions.  Sums are taken
+// in a fixed order everywhere (split-K partials, head groups, columns):
+// results are the same bits on every run.  Every wait - mbarriers and the
+// grid barriers - is bounded in time; a wait that runs out records
+// LEMO_ERR_TIMEOUT, raises a flag that makes every CTA skip the rest, and
+// each CTA drains what it issued and frees its tensor memory before it
+// returns.
 #pragma once
 
 #include <cuda_bf16.h>
 
 #include "common.cuh"
+#include "score.cuh"
 
 namespace lemo {
 namespace predict {
+
+using score::mbar_arrive;
+using score::mbar_arrive_expect_tx;
+using score::mbar_init;
+using score::mbar_try_wait;
+using score::smem_u32;
+using score::tc_fence_after;
+using score::tc_fence_before;
+using score::tmem_ld16;
+using score::tmem_wait_ld;
+
+constexpr int TILE = 128;                 // rows of a row tile (MMA M, TMEM lanes)
+constexpr int KCH = 64;                   // K elements of one image (one 128-byte row)
+constexpr int IMG = TILE * KCH * 2;       // 16 KB
+constexpr int STAGES = 3;
+constexpr int STAGE_BYTES = 4 * IMG;      // A hi | A lo | B (hi) | B lo
+constexpr int LOAD_WARPS = 8;             // weight loaders + epilogue (warps 2..9)
+constexpr int THREADS = 32 * (2 + LOAD_WARPS);
+constexpr int ACC_COLS = 256;
+constexpr int TMEM_COLS = 2 * ACC_COLS;
+constexpr int MAX_NT = 256;               // widest MMA N
+constexpr int kPoolThreads = 128;
+constexpr int kPoolCols = kPoolThreads * 8;  // columns of X per pooling CTA
+
+// Grid-barrier words (in the workspace; zeroed by the pooling pass).
+constexpr int kSyncA = 0, kSyncB = 1, kSyncC = 2, kSyncD = 3, kSyncE = 4, kSyncAbort = 7;
+constexpr int kSyncWords = 8;
+
+struct Smem {
+    uint64_t full[STAGES];      // bulk bytes landed + every loader warp stored its part
+    uint64_t empty[STAGES];     // the MMAs reading the stage completed
+    uint64_t acc_full[2];       // accumulator holds a finished product
+    uint64_t acc_empty[2];      // the epilogue warps read the accumulator
+    uint64_t done;              // every MMA of this CTA completed
+    uint32_t tmem_base;
+    int abort_flag;
+};
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align slack*/ + (int)sizeof(Smem);
+static_assert(SMEM_BYTES <= 232448, "exceeds the 227 KB of shared memory per CTA");
+
+// Byte offset of element e (0..63) of row r (0..127) inside an image.
+__host__ __device__ __forceinline__ uint32_t img_off(int r, int e) {
+    return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((((e >> 3) ^ (r & 7)) & 7) << 4) +
+                      ((e & 7) << 1));
+}
+
+// Byte offset of the 16-byte chunk (row k, columns 8 j8 .. 8 j8 + 7 of 64-column
+// group grp) of an MN-major weight tile (64 rows of K, groups 8 KB apart).
+__device__ __forceinline__ uint32_t mn_off(int k, int grp, int j8) {
+    return (uint32_t)(grp * 8192 + (k >> 3) * 1024 + (k & 7) * 128 + (((j8 ^ (k & 7)) & 7) << 4));
+}
 
 __device__ __forceinline__ void split2(float v, uint16_t& hi, uint16_t& lo) {
     const __nv_bfloat16 h = __float2bfloat16_rn(v);
@@ -45,68 +113,25 @@ __device__ __forceinline__ void split2(float v, uint16_t& hi, uint16_t& lo) {
     lo = *reinterpret_cast<const uint16_t*>(&l);
 }
 
-// Split 8 fp32 values and store them as 8 bf16 in each plane (16 bytes).
-__device__ __forceinline__ void store_split8(const float* v, uint16_t* hi, uint16_t* lo) {
+// Split 8 fp32 values into two 16-byte chunks (8 bf16 each).
+__device__ __forceinline__ void split8(const float* v, uint4& a, uint4& b) {
     uint16_t h[8], l[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) split2(v[i], h[i], l[i]);
-    uint4 a, b;
     a.x = h[0] | ((uint32_t)h[1] << 16);  b.x = l[0] | ((uint32_t)l[1] << 16);
     a.y = h[2] | ((uint32_t)h[3] << 16);  b.y = l[2] | ((uint32_t)l[3] << 16);
     a.z = h[4] | ((uint32_t)h[5] << 16);  b.z = l[4] | ((uint32_t)l[5] << 16);
     a.w = h[6] | ((uint32_t)h[7] << 16);  b.w = l[6] | ((uint32_t)l[7] << 16);
-    *reinterpret_cast<uint4*>(hi) = a;
-    *reinterpret_cast<uint4*>(lo) = b;
 }
 
 // ---------------------------------------------------------------------------
-// Weight planes.  pad_kernel copies a bf16 matrix [rows][cols] (any
-// alignment) into a plane [rows_out][ld] whose rows are 16-byte aligned:
-// columns are grouped in runs of `run` (the head dimension of W2, or all
-// columns of W1), each run padded to `run_ld` (a multiple of 8); padding and
-// rows >= rows are zero.  blockIdx.y selects one of up to four matrices;
-// CTA x copies rows [8 x, 8 x + 8), 32 threads per row.
+// Pooling pass.  CTA (row g, column chunk y): block means of token block g
+// over columns [y*1024, +1024), each thread 8 consecutive columns (16-byte
+// loads, eight rows in flight, added in row order).  The means are written
+// as hi / lo images [row tile][64-column chunk][plane]; rows g >= TB and
+// columns >= d of the last tile / chunk are written as zeros.  CTA (0, 0)
+// also clears the grid-barrier words of predict_kernel.
 // ---------------------------------------------------------------------------
-struct PadArgs {
-    const uint16_t* src[4];
-    uint16_t* dst[4];
-    int rows, rows_out, cols, run, run_ld;
-    int64_t ld_out;
-};
-
-__global__ void __launch_bounds__(256) pad_kernel(const PadArgs a) {
-    pdl_entry();
-    const int y = blockIdx.y;
-    const uint16_t* src = y == 0 ? a.src[0] : y == 1 ? a.src[1] : y == 2 ? a.src[2] : a.src[3];
-    uint16_t* dst = y == 0 ? a.dst[0] : y == 1 ? a.dst[1] : y == 2 ? a.dst[2] : a.dst[3];
-    const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
-    if (row >= a.rows_out) return;
-    const int runs = a.cols / a.run, chunks_per_run = a.run_ld / 8;
-    for (int c = threadIdx.x & 31; c < runs * chunks_per_run; c += 32) {
-        const int r = c / chunks_per_run, c0 = (c % chunks_per_run) * 8;
-        uint16_t v[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-            v[e] = (row < a.rows && c0 + e < a.run)
-                       ? src[(int64_t)row * a.cols + (int64_t)r * a.run + c0 + e]
-                       : (uint16_t)0;
-        uint4 o;
-        o.x = v[0] | ((uint32_t)v[1] << 16);
-        o.y = v[2] | ((uint32_t)v[3] << 16);
-        o.z = v[4] | ((uint32_t)v[5] << 16);
-        o.w = v[6] | ((uint32_t)v[7] << 16);
-        *reinterpret_cast<uint4*>(dst + (int64_t)row * a.ld_out + (int64_t)r * a.run_ld + c0) = o;
-    }
-}
-
-// ---------------------------------------------------------------------------
-// Pooling pass.  CTA (g, c): block means of token block g, columns
-// [c*2048, +2048), each thread 8 consecutive columns (16-byte loads, four
-// rows in flight, added in row order), written as hi / lo planes [TB][d].
-// ---------------------------------------------------------------------------
-constexpr int kPoolThreads = 256;
-constexpr int kPoolCols = kPoolThreads * 8;
-
 __device__ __forceinline__ void add_row(float* acc, const uint4 v) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -117,528 +142,778 @@ __device__ __forceinline__ void add_row(float* acc, const uint4 v) {
 }
 
 __global__ void __launch_bounds__(kPoolThreads)
-    pool_kernel(const uint16_t* __restrict__ x, int64_t ld_x, int d, const int32_t* __restrict__ cu,
+    pool_kernel(const uint16_t* __restrict__ x, int64_t ld_x, int d, int kc, const int32_t* __restrict__ cu,
                 int batch, int block, const char* __restrict__ ws, WsLayout lay,
-                uint16_t* __restrict__ xb_hi, uint16_t* __restrict__ xb_lo) {
+                uint8_t* __restrict__ xb, uint32_t* __restrict__ sync) {
     pdl_entry();
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x < kSyncWords) sync[threadIdx.x] = 0u;
     const PlanHeader* hdr = reinterpret_cast<const PlanHeader*>(ws + lay.hdr);
     if (!hdr->valid) return;
     const int g = blockIdx.x;
-    if (g >= hdr->total_blocks) return;
-    const int32_t* blk_prefix = reinterpret_cast<const int32_t*>(ws + lay.blk_prefix);
-    const int s = last_le(blk_prefix, batch + 1, g);
-    const int m = g - blk_prefix[s];
-    const int64_t r0 = (int64_t)cu[s] + (int64_t)m * block;
-    const int64_t r1 = min((int64_t)cu[s + 1], r0 + block);
-    const int c = blockIdx.y * kPoolCols + threadIdx.x * 8;
-    if (c >= d) return;
+    const int c0 = blockIdx.y * kPoolCols + threadIdx.x * 8;
+    if (c0 >= kc * KCH) return;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    const uint16_t* p = x + r0 * ld_x + c;
-    int64_t r = r0;
-    for (; r + 4 <= r1; r += 4, p += 4 * ld_x) {
-        uint4 v[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) v[u] = *reinterpret_cast<const uint4*>(p + u * ld_x);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) add_row(acc, v[u]);
-    }
-    for (; r < r1; ++r, p += ld_x) add_row(acc, *reinterpret_cast<const uint4*>(p));
-    const float inv = 1.f / (float)(r1 - r0);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] *= inv;
-    store_split8(acc, xb_hi + (int64_t)g * d + c, xb_lo + (int64_t)g * d + c);
-}
-
-// ---------------------------------------------------------------------------
-// Warp-level tensor-core tiles.  A CTA of 4 warps computes a 64 x 64 tile of
-// C = A B: A is a pair of bf16 planes [M][lda] (hi, lo) and B either a bf16
-// plane [K][ldb] (weights, N contiguous) or a pair of bf16 planes [N][ldb]
-// (Khat, K contiguous).  K advances in stages of 32 through a ring of
-// shared-memory buffers filled by cp.async (16-byte chunks; chunks outside
-// the matrix are zero-filled), so the loads of the next stages are in
-// flight while the current one is multiplied.  Each warp owns a 32 x 32
-// sub-tile (2 x 4 MMAs of 16 x 8) and takes its fragments with ldmatrix
-// (.trans for the N-contiguous weights).  Row pitches of 80 and 144 bytes
-// keep every ldmatrix phase on distinct banks.
-// ---------------------------------------------------------------------------
-constexpr int TM = 64, TN = 64, TK = 32;
-constexpr int kMmaThreads = 128;
-constexpr int A_PITCH = 80;                 // bytes per row of a [64][32] bf16 tile
-constexpr int A_PLANE = TM * A_PITCH;       // 5120 bytes
-constexpr int B_PITCH = 144;                // bytes per row of a [32][64] bf16 tile
-constexpr int B_PLANE = TK * B_PITCH;       // 4608 bytes
-constexpr int GEMM_STAGES = 3;
-constexpr int GEMM_STAGE = 2 * A_PLANE + B_PLANE;
-constexpr int PROD_STAGES = 3;
-constexpr int PROD_STAGE = 4 * A_PLANE;
-constexpr int PROD_SMEM = PROD_STAGES * PROD_STAGE;  // dynamic shared memory (60 KB)
-
-__device__ __forceinline__ uint32_t smem_addr(const void* p) {
-    return (uint32_t)__cvta_generic_to_shared(p);
-}
-
-// 16 bytes global -> shared; `valid` false writes 16 zero bytes (nothing is read).
-__device__ __forceinline__ void cp16(uint32_t dst, const void* src, bool valid) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
-                 "r"(valid ? 16u : 0u)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
-__device__ __forceinline__ void ldsm4(uint32_t addr, uint32_t* r) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(addr));
-}
-__device__ __forceinline__ void ldsm4t(uint32_t addr, uint32_t* r) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(addr));
-}
-
-__device__ __forceinline__ void mma16816(float* c, const uint32_t* a, const uint32_t* b) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-        "{%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
-}
-
-// A [64][32] bf16 tile of a K-contiguous plane (rows r0.., columns k0..)
-// into shared memory (pitch A_PITCH): 256 chunks, two per thread.  Chunks of
-// rows >= rows or at columns >= kend are zero (kend is a multiple of 8).
-__device__ __forceinline__ void load_k_tile(uint8_t* dst, const uint16_t* __restrict__ src,
-                                            int64_t ld, int r0, int rows, int k0, int kend) {
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        const int c = threadIdx.x + kMmaThreads * i;
-        const int r = c >> 2, kc = (c & 3) * 8;
-        const bool ok = r0 + r < rows && k0 + kc < kend;
-        cp16(smem_addr(dst + r * A_PITCH + kc * 2), ok ? src + (int64_t)(r0 + r) * ld + k0 + kc : src,
-             ok);
-    }
-}
-
-// 4 bytes global -> shared (same zero fill).
-__device__ __forceinline__ void cp4(uint32_t dst, const void* src, bool valid) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src),
-                 "r"(valid ? 4u : 0u)
-                 : "memory");
-}
-
-// A [32][64] bf16 tile of an N-contiguous matrix [K][ld] (rows k0.., columns
-// n0..) into shared memory (pitch B_PITCH); rows >= kend, columns >= ncols
-// are zero.  VEC16: rows 16-byte aligned, ncols a multiple of 8 (two
-// 16-byte chunks per thread); otherwise rows 4-byte aligned, ncols even
-// (eight 4-byte copies per thread).
-template <bool VEC16>
-__device__ __forceinline__ void load_n_tile(uint8_t* dst, const uint16_t* __restrict__ src,
-                                            int64_t ld, int k0, int kend, int n0, int ncols) {
-    if (VEC16) {
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const int c = threadIdx.x + kMmaThreads * i;
-            const int k = c >> 3, nc = (c & 7) * 8;
-            const bool ok = k0 + k < kend && n0 + nc < ncols;
-            cp16(smem_addr(dst + k * B_PITCH + nc * 2),
-                 ok ? src + (int64_t)(k0 + k) * ld + n0 + nc : src, ok);
-        }
-    } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int c = threadIdx.x + kMmaThreads * i;
-            const int k = c >> 5, nc = (c & 31) * 2;
-            const bool ok = k0 + k < kend && n0 + nc < ncols;
-            cp4(smem_addr(dst + k * B_PITCH + nc * 2),
-                ok ? src + (int64_t)(k0 + k) * ld + n0 + nc : src, ok);
-        }
-    }
-}
-
-// A fragments (rows wm + 16 mi ..) of one plane at K offset ks.
-__device__ __forceinline__ void frag_a(const uint8_t* tile, int wm, int ks, uint32_t (*a)[4]) {
-    const int lane = threadIdx.x & 31;
-#pragma unroll
-    for (int mi = 0; mi < 2; ++mi)
-        ldsm4(smem_addr(tile + (wm + mi * 16 + (lane & 15)) * A_PITCH + (ks + (lane >> 4) * 8) * 2),
-              a[mi]);
-}
-
-// B fragments of the 4 n8 blocks (columns wn ..) at K offset ks, from an
-// N-contiguous [32][64] tile (transposing loads) ...
-__device__ __forceinline__ void frag_b_n(const uint8_t* tile, int wn, int ks, uint32_t (*b)[2]) {
-    const int lane = threadIdx.x & 31, mtx = lane >> 3, r8 = lane & 7;
-#pragma unroll
-    for (int p = 0; p < 2; ++p) {
-        uint32_t r[4];
-        ldsm4t(smem_addr(tile + (ks + (mtx & 1) * 8 + r8) * B_PITCH + (wn + 16 * p + (mtx >> 1) * 8) * 2),
-               r);
-        b[2 * p][0] = r[0];
-        b[2 * p][1] = r[1];
-        b[2 * p + 1][0] = r[2];
-        b[2 * p + 1][1] = r[3];
-    }
-}
-
-// ... or from a K-contiguous [64][32] tile.
-__device__ __forceinline__ void frag_b_k(const uint8_t* tile, int wn, int ks, uint32_t (*b)[2]) {
-    const int lane = threadIdx.x & 31, mtx = lane >> 3, r8 = lane & 7;
-#pragma unroll
-    for (int p = 0; p < 2; ++p) {
-        uint32_t r[4];
-        ldsm4(smem_addr(tile + (wn + 16 * p + (mtx >> 1) * 8 + r8) * A_PITCH + (ks + (mtx & 1) * 8) * 2),
-              r);
-        b[2 * p][0] = r[0];
-        b[2 * p][1] = r[1];
-        b[2 * p + 1][0] = r[2];
-        b[2 * p + 1][1] = r[3];
-    }
-}
-
-__device__ __forceinline__ void zero_acc(float (*acc)[4][4]) {
-#pragma unroll
-    for (int mi = 0; mi < 2; ++mi)
-#pragma unroll
-        for (int ni = 0; ni < 4; ++ni)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) acc[mi][ni][i] = 0.f;
-}
-
-// Visit the accumulator elements with their tile coordinates (row, column).
-template <typename F>
-__device__ __forceinline__ void for_acc(const float (*acc)[4][4], F f) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int g = lane >> 2, t = lane & 3;
-    const int wm = (warp >> 1) * 32, wn = (warp & 1) * 32;
-#pragma unroll
-    for (int mi = 0; mi < 2; ++mi)
-#pragma unroll
-        for (int ni = 0; ni < 4; ++ni)
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                f(wm + mi * 16 + g + (i >> 1) * 8, wn + ni * 8 + 2 * t + (i & 1), acc[mi][ni][i]);
-}
-
-// ---------------------------------------------------------------------------
-// Predictor GEMM, both predictors in one launch: for side s (0 = query,
-// 1 = key) and K split z (blockIdx.z = s * splits + z),
-//   C[s] (+ z * c_split)[m][n] = sum_{k in split z} A[s][m][k] W[s][k][n]
-// with A = hi + lo bf16 planes [M][lda] (M = number of token blocks, read
-// on the device) and W bf16 [K][ldw] with w_cols columns (columns w_cols ..
-// N - 1 read as zero).  SPLIT_OUT: C is written as hi / lo planes (c, c_lo)
-// for the block products, else as fp32 (split-K partial sums).
-// ---------------------------------------------------------------------------
-struct GemmArgs {
-    const uint16_t* a_hi[2];
-    const uint16_t* a_lo[2];
-    int64_t lda;
-    const uint16_t* w[2];
-    int64_t ldw;
-    float* c[2];         // fp32 output
-    uint16_t* c_hi[2];   // split output
-    uint16_t* c_lo[2];
-    int64_t ldc;
-    int64_t c_split;     // elements between the split-K partial planes
-    const PlanHeader* hdr;
-    int N, K;
-    int w_rows;          // rows of W that exist (rows past it read as zero)
-    int w_cols;          // columns of W that exist (a multiple of 8, or even with w_vec4)
-    bool w_vec4;         // W rows only 4-byte aligned: 4-byte copies
-    int k_chunk;         // K range of one split (a multiple of TK)
-    int splits;
-};
-
-template <bool SPLIT_OUT>
-__global__ void __launch_bounds__(kMmaThreads) gemm_kernel(const GemmArgs p) {
-    pdl_entry();
-    const int M = p.hdr->total_blocks;
-    const int m0 = blockIdx.y * TM, n0 = blockIdx.x * TN;
-    if (!p.hdr->valid || m0 >= M) return;
-    const int side = blockIdx.z / p.splits, z = blockIdx.z % p.splits;
-    const int kb = z * p.k_chunk, ke = min(p.K, kb + p.k_chunk);
-    if (kb >= ke) return;
-    __shared__ __align__(128) uint8_t sm[GEMM_STAGES][GEMM_STAGE];  // [A hi | A lo | B]
-    const uint16_t* Ah = side ? p.a_hi[1] : p.a_hi[0];  // (selects: no local copy of the arrays)
-    const uint16_t* Al = side ? p.a_lo[1] : p.a_lo[0];
-    const uint16_t* W = side ? p.w[1] : p.w[0];
-    const int warp = threadIdx.x >> 5;
-    const int wm = (warp >> 1) * 32, wn = (warp & 1) * 32;
-    float acc[2][4][4];
-    zero_acc(acc);
-    const int nst = (ke - kb + TK - 1) / TK;
-    auto load_stage = [&](int s) {
-        uint8_t* b = sm[s % GEMM_STAGES];
-        const int k0 = kb + s * TK;
-        load_k_tile(b, Ah, p.lda, m0, M, k0, ke);
-        load_k_tile(b + A_PLANE, Al, p.lda, m0, M, k0, ke);
-        if (p.w_vec4)
-            load_n_tile<false>(b + 2 * A_PLANE, W, p.ldw, k0, min(ke, p.w_rows), n0, p.w_cols);
-        else
-            load_n_tile<true>(b + 2 * A_PLANE, W, p.ldw, k0, min(ke, p.w_rows), n0, p.w_cols);
-    };
-#pragma unroll
-    for (int s = 0; s < GEMM_STAGES - 1; ++s) {
-        if (s < nst) load_stage(s);
-        cp_commit();
-    }
-    for (int s = 0; s < nst; ++s) {
-        cp_wait<GEMM_STAGES - 2>();
-        __syncthreads();  // stage s landed for every thread; stage s - 1 is no longer read
-        if (s + GEMM_STAGES - 1 < nst) load_stage(s + GEMM_STAGES - 1);
-        cp_commit();
-        const uint8_t* b = sm[s % GEMM_STAGES];
-#pragma unroll
-        for (int ks = 0; ks < TK; ks += 16) {
-            uint32_t ah[2][4], al[2][4], bf[4][2];
-            frag_a(b, wm, ks, ah);
-            frag_a(b + A_PLANE, wm, ks, al);
-            frag_b_n(b + 2 * A_PLANE, wn, ks, bf);
-#pragma unroll
-            for (int ni = 0; ni < 4; ++ni)
-#pragma unroll
-                for (int mi = 0; mi < 2; ++mi) {
-                    mma16816(acc[mi][ni], ah[mi], bf[ni]);
-                    mma16816(acc[mi][ni], al[mi], bf[ni]);
-                }
-        }
-    }
-    if (SPLIT_OUT) {
-        // hi / lo tiles [64][64] staged in shared memory (pitch B_PITCH),
-        // then written as 16-byte row chunks
-        uint16_t* Ch = side ? p.c_hi[1] : p.c_hi[0];
-        uint16_t* Cl = side ? p.c_lo[1] : p.c_lo[0];
-        cp_wait<0>();
-        __syncthreads();  // every warp is done with the operand buffers
-        uint8_t* th = &sm[0][0];  // 2 x 64 rows of B_PITCH: spans the first two stages
-        uint8_t* tl = th + TM * B_PITCH;
-        static_assert(2 * TM * B_PITCH <= GEMM_STAGES * GEMM_STAGE, "staging exceeds the ring");
-        for_acc(acc, [&](int r, int c, float v) {
-            uint16_t h, l;
-            split2(v, h, l);
-            *reinterpret_cast<uint16_t*>(th + r * B_PITCH + c * 2) = h;
-            *reinterpret_cast<uint16_t*>(tl + r * B_PITCH + c * 2) = l;
-        });
-        __syncthreads();
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int e = threadIdx.x + kMmaThreads * i;  // 512 chunks of 8 per plane
-            const int r = e >> 3, c = (e & 7) * 8;
-            if (m0 + r < M && n0 + c < p.N) {
-                const int64_t o = (int64_t)(m0 + r) * p.ldc + n0 + c;
-                *reinterpret_cast<uint4*>(Ch + o) = *reinterpret_cast<const uint4*>(th + r * B_PITCH + c * 2);
-                *reinterpret_cast<uint4*>(Cl + o) = *reinterpret_cast<const uint4*>(tl + r * B_PITCH + c * 2);
-            }
-        }
-    } else {
-        float* C = (side ? p.c[1] : p.c[0]) + (int64_t)z * p.c_split;
-        for_acc(acc, [&](int r, int c, float v) {
-            if (m0 + r < M && n0 + c < p.N) C[(int64_t)(m0 + r) * p.ldc + n0 + c] = v;
-        });
-    }
-}
-
-// hid[s][m][n] = relu(sum_z part[s][z][m][n]), z in increasing order, for
-// both sides (blockIdx.y = side), written as hi / lo planes.  Partial
-// planes are `plane` elements apart, rows N apart (N a multiple of 8); each
-// thread takes 4 consecutive elements and keeps the loads of 8 splits in
-// flight at a time.
-__global__ void __launch_bounds__(256)
-    reduce_kernel(const float* __restrict__ part, int64_t side_stride, int64_t plane, int splits,
-                  const PlanHeader* __restrict__ hdr, int N, uint16_t* __restrict__ hid_hi,
-                  uint16_t* __restrict__ hid_lo, int64_t hid_side_stride) {
-    pdl_entry();
-    if (!hdr->valid) return;
-    const int64_t total = (int64_t)hdr->total_blocks * N / 4;
-    const float* src = part + blockIdx.y * side_stride;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        int z = 0;
-        for (; z + 8 <= splits; z += 8) {
-            float4 t[8];
+    if (g < hdr->total_blocks && c0 < d) {
+        const int32_t* blk_prefix = reinterpret_cast<const int32_t*>(ws + lay.blk_prefix);
+        const int s = last_le(blk_prefix, batch + 1, g);
+        const int m = g - blk_prefix[s];
+        const int64_t r0 = (int64_t)cu[s] + (int64_t)m * block;
+        const int64_t r1 = min((int64_t)cu[s + 1], r0 + block);
+        const uint16_t* p = x + r0 * ld_x + c0;
+        int64_t r = r0;
+        for (; r + 8 <= r1; r += 8, p += 8 * ld_x) {
+            uint4 v[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u)
-                t[u] = *reinterpret_cast<const float4*>(src + (int64_t)(z + u) * plane + i * 4);
+                v[u] = __ldg(reinterpret_cast<const uint4*>(p + u * ld_x));
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                v.x += t[u].x; v.y += t[u].y; v.z += t[u].z; v.w += t[u].w;
-            }
+            for (int u = 0; u < 8; ++u) add_row(acc, v[u]);
         }
-        for (; z < splits; ++z) {
-            const float4 t = *reinterpret_cast<const float4*>(src + (int64_t)z * plane + i * 4);
-            v.x += t.x; v.y += t.y; v.z += t.z; v.w += t.w;
-        }
-        const float r[4] = {fmaxf(v.x, 0.f), fmaxf(v.y, 0.f), fmaxf(v.z, 0.f), fmaxf(v.w, 0.f)};
-        uint16_t h[4], l[4];
+        for (; r < r1; ++r, p += ld_x) add_row(acc, __ldg(reinterpret_cast<const uint4*>(p)));
+        const float inv = 1.f / (float)(r1 - r0);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) split2(r[e], h[e], l[e]);
-        const int64_t o = blockIdx.y * hid_side_stride + i * 4;
-        *reinterpret_cast<uint2*>(hid_hi + o) =
-            make_uint2(h[0] | ((uint32_t)h[1] << 16), h[2] | ((uint32_t)h[3] << 16));
-        *reinterpret_cast<uint2*>(hid_lo + o) =
-            make_uint2(l[0] | ((uint32_t)l[1] << 16), l[2] | ((uint32_t)l[3] << 16));
+        for (int i = 0; i < 8; ++i) acc[i] *= inv;
     }
+    uint4 hi, lo;
+    split8(acc, hi, lo);
+    const int R = g / TILE, r = g % TILE, c = c0 / KCH;
+    uint8_t* im = xb + ((size_t)(R * kc + c) * 2) * IMG + img_off(r, c0 % KCH);
+    *reinterpret_cast<uint4*>(im) = hi;
+    *reinterpret_cast<uint4*>(im + IMG) = lo;
 }
 
 // ---------------------------------------------------------------------------
-// Block products.  CTA (tile, head group): the 64 x 64 tile of block pairs
-// (n, m) number `tile` of the lower triangle (tile rows tn >= tile columns
-// tm), heads [g * hpg, (g + 1) * hpg).  For each head the tile's dot
-// products Qhat_n^h . Khat_m^h are accumulated over its ldh columns (dh
-// values and zero padding), then their positive parts are added up.  With
-// one head group the CTA writes P[n][m] = inv_h * sum directly (per-sequence
-// [N_b, N_b] layout, pairs of one sequence with n >= m only); otherwise it
-// writes its partial sums to plane g of `part` ([groups][tb_cap][tb_cap])
-// for products_reduce_kernel.
+// predict_kernel
 // ---------------------------------------------------------------------------
-struct ProductsArgs {
-    const uint16_t* q_hi;   // [TB][H * ldh]
-    const uint16_t* q_lo;
-    const uint16_t* k_hi;
-    const uint16_t* k_lo;
-    int H, ldh, hpg, groups, batch;
-    int64_t tb_cap;    // row stride of the partial planes
+enum WeightLoad : int { kW16 = 0, kW4 = 1, kW2 = 2 };  // 16-, 4- or 2-byte loads
+
+struct Args {
+    const char* ws;
+    WsLayout lay;
+    int batch;
+    // shapes
+    int d, rank, H, dh, dhp, dc;   // dhp: dh padded to 64; dc = dhp / 64
+    int rt;                        // row tiles of 128 token blocks
+    int tba;                       // rt * 128
+    int kc;                        // 64-column chunks of d
+    int kc2;                       // 64-column chunks of rank
+    int ldr;                       // rank padded to 32 (columns of the split-K partials)
+    int nj, nt;                    // n tiles of the first GEMM and their width
+    int zk, cps;                   // K splits of the first GEMM and chunks per split
+    int np, nj2;                   // H * dhp and its 256-column tiles
+    int pt, groups, hpg;           // block-product tiles, head groups, heads per group
     float inv_h;
-    float* part;       // [groups][tb_cap][tb_cap] (groups > 1)
-    float* P;          // per-sequence block-product matrices
+    // inputs
+    const uint16_t* w1[2];
+    const uint16_t* w2[2];
+    int w1_mode, w2_mode;
+    // workspace
+    const uint8_t* xb;    // [rt][kc][2] images
+    float* part;          // [2][zk][tba][ldr]
+    uint8_t* hid;         // [2][rt][kc2][2] images
+    uint8_t* qk;          // [2][rt][H][dc][2] images
+    float* ppart;         // [groups][tba][tba] (groups > 1)
+    float* P;             // per-sequence block-product matrices
+    uint32_t* sync;
+    float* scores;
+    uint64_t spin_limit_ns;
 };
 
-__device__ __forceinline__ void store_pair(const ProductsArgs& a, const int32_t* blk_prefix,
-                                           const int64_t* m_prefix, int s, int n, int m,
-                                           float v) {
-    const int b0 = blk_prefix[s];
-    if (m < b0 || m > n) return;  // other sequence, or above the diagonal
-    const int nb = blk_prefix[s + 1] - b0;
-    a.P[m_prefix[s] + (int64_t)(n - b0) * nb + (m - b0)] = v * a.inv_h;
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo) {
+    uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)(1024u >> 4) << 32;
+    d |= (uint64_t)1u << 46;
+    d |= (uint64_t)2u << 61;
+    return d;
 }
 
-__global__ void __launch_bounds__(kMmaThreads)
-    products_kernel(const ProductsArgs a, const char* __restrict__ ws, WsLayout lay) {
-    pdl_entry();
-    const PlanHeader* hdr = reinterpret_cast<const PlanHeader*>(ws + lay.hdr);
-    if (!hdr->valid) return;
-    const int32_t* blk_prefix = reinterpret_cast<const int32_t*>(ws + lay.blk_prefix);
-    const int64_t* m_prefix = reinterpret_cast<const int64_t*>(ws + lay.m_prefix);
-    const int TB = hdr->total_blocks;
-    // lower-triangular tile number -> (tn, tm), tm <= tn
-    const int idx = blockIdx.x;
-    int tn = (int)((sqrtf(8.f * (float)idx + 1.f) - 1.f) * 0.5f);
-    while ((tn + 1) * (tn + 2) / 2 <= idx) ++tn;
-    while (tn * (tn + 1) / 2 > idx) --tn;
-    const int tm = idx - tn * (tn + 1) / 2;
-    const int n0 = tn * TM, mb0 = tm * TN;
-    if (n0 >= TB) return;
-    const int64_t HD = (int64_t)a.H * a.ldh;
-    extern __shared__ __align__(128) uint8_t prod_smem[];  // stages of [Q hi | Q lo | K hi | K lo]
-    const int warp = threadIdx.x >> 5;
-    const int wm = (warp >> 1) * 32, wn = (warp & 1) * 32;
-    float acc[2][4][4], tot[2][4][4];
-    zero_acc(tot);
-    zero_acc(acc);
-    const int h0 = blockIdx.y * a.hpg, h1 = min(a.H, h0 + a.hpg);
-    const int per_head = (a.ldh + TK - 1) / TK;
-    const int nst = (h1 - h0) * per_head;
-    auto load_stage = [&](int s) {
-        uint8_t* b = prod_smem + (s % PROD_STAGES) * PROD_STAGE;
-        const int h = h0 + s / per_head;
-        const int k0 = h * a.ldh + (s % per_head) * TK, ke = (h + 1) * a.ldh;
-        load_k_tile(b, a.q_hi, HD, n0, TB, k0, ke);
-        load_k_tile(b + A_PLANE, a.q_lo, HD, n0, TB, k0, ke);
-        load_k_tile(b + 2 * A_PLANE, a.k_hi, HD, mb0, TB, k0, ke);
-        load_k_tile(b + 3 * A_PLANE, a.k_lo, HD, mb0, TB, k0, ke);
-    };
-#pragma unroll
-    for (int s = 0; s < PROD_STAGES - 1; ++s) {
-        if (s < nst) load_stage(s);
-        cp_commit();
-    }
-    for (int s = 0; s < nst; ++s) {
-        cp_wait<PROD_STAGES - 2>();
-        __syncthreads();  // stage s landed for every thread; stage s - 1 is no longer read
-        if (s + PROD_STAGES - 1 < nst) load_stage(s + PROD_STAGES - 1);
-        cp_commit();
-        const uint8_t* b = prod_smem + (s % PROD_STAGES) * PROD_STAGE;
-#pragma unroll
-        for (int ks = 0; ks < TK; ks += 16) {
-            uint32_t ah[2][4], al[2][4], bh[4][2], bl[4][2];
-            frag_a(b, wm, ks, ah);
-            frag_a(b + A_PLANE, wm, ks, al);
-            frag_b_k(b + 2 * A_PLANE, wn, ks, bh);
-            frag_b_k(b + 3 * A_PLANE, wn, ks, bl);
-#pragma unroll
-            for (int ni = 0; ni < 4; ++ni) {
-#pragma unroll
-                for (int mi = 0; mi < 2; ++mi) {
-                    mma16816(acc[mi][ni], ah[mi], bh[ni]);
-                    mma16816(acc[mi][ni], al[mi], bh[ni]);
-                }
-#pragma unroll
-                for (int mi = 0; mi < 2; ++mi) mma16816(acc[mi][ni], ah[mi], bl[ni]);
+// Instruction descriptor of tcgen05.mma kind::f16: D fp32, A and B bf16,
+// A K-major, B K-major or MN-major (bit 16), M = 128, N = n.
+__device__ __forceinline__ uint32_t idesc(int n, bool b_mn_major) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | (b_mn_major ? (1u << 16) : 0u) |
+           ((uint32_t)(n >> 3) << 17) | ((uint32_t)(TILE >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t id,
+                                     uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %3, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %4, p;\n\t}\n" ::"r"(tmem_d),
+        "l"(da), "l"(db), "r"(accumulate), "r"(id));
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            dst),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// `count` arrivals on a CTA-local mbarrier.
+__device__ __forceinline__ void mbar_arrive_cnt(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__device__ __forceinline__ bool aborted(const Smem* sm) {
+    return *reinterpret_cast<const volatile int*>(&sm->abort_flag) != 0;
+}
+
+__device__ __forceinline__ void give_up(Smem* sm, uint32_t* sync) {
+    *reinterpret_cast<volatile int*>(&sm->abort_flag) = 1;
+    atomicExch(&sync[kSyncAbort], 1u);
+}
+
+__device__ __noinline__ bool wait_slow(uint64_t* bar, uint32_t parity, Smem* sm, uint32_t* sync,
+                                       uint64_t limit_ns) {
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t n = 1;; ++n) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((n & 63) == 0) {
+            if (aborted(sm)) return false;
+            if (globaltimer_ns() - t0 > limit_ns) {
+                raise_error(LEMO_ERR_TIMEOUT);
+                give_up(sm, sync);
+                return false;
             }
         }
-        if ((s + 1) % per_head == 0) {  // head complete: keep its positive part
-#pragma unroll
-            for (int mi = 0; mi < 2; ++mi)
-#pragma unroll
-                for (int ni = 0; ni < 4; ++ni)
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        tot[mi][ni][i] += fmaxf(acc[mi][ni][i], 0.f);
-                        acc[mi][ni][i] = 0.f;
-                    }
-        }
-    }
-    if (a.groups == 1) {
-        for_acc(tot, [&](int r, int c, float v) {
-            const int n = n0 + r, m = mb0 + c;
-            if (n >= TB || m >= TB) return;
-            store_pair(a, blk_prefix, m_prefix, last_le(blk_prefix, a.batch + 1, n), n, m, v);
-        });
-    } else {
-        float* plane = a.part + (int64_t)blockIdx.y * a.tb_cap * a.tb_cap;
-        for_acc(tot, [&](int r, int c, float v) {
-            const int n = n0 + r, m = mb0 + c;
-            if (n < TB && m < TB && m <= n) plane[(int64_t)n * a.tb_cap + m] = v;
-        });
     }
 }
 
-// P[n][m] = inv_h * sum_g part[g][n][m], g in increasing order, for the
-// pairs of one sequence with n >= m (head groups > 1).  Threads run along
-// m, so the partial planes are read with coalesced loads.
-__global__ void __launch_bounds__(256)
-    products_reduce_kernel(const ProductsArgs a, const char* __restrict__ ws, WsLayout lay) {
-    pdl_entry();
-    const PlanHeader* hdr = reinterpret_cast<const PlanHeader*>(ws + lay.hdr);
-    if (!hdr->valid) return;
-    const int32_t* blk_prefix = reinterpret_cast<const int32_t*>(ws + lay.blk_prefix);
-    const int64_t* m_prefix = reinterpret_cast<const int64_t*>(ws + lay.m_prefix);
-    const int TB = hdr->total_blocks;
-    const int64_t total = (int64_t)TB * TB;
-    const int64_t plane = a.tb_cap * a.tb_cap;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        const int n = (int)(i / TB), m = (int)(i % TB);
-        if (m > n) continue;
-        const int s = last_le(blk_prefix, a.batch + 1, n);
-        if (m < blk_prefix[s]) continue;
-        const int64_t o = (int64_t)n * a.tb_cap + m;
-        // loads in batches of 8 (in flight together), added in g order
-        float v = 0.f;
-        int g = 0;
-        for (; g + 8 <= a.groups; g += 8) {
-            float t[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) t[u] = a.part[(g + u) * plane + o];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) v += t[u];
+// Wait for the phase of the given parity (false: this CTA gave up).
+__device__ __forceinline__ bool wait(uint64_t* bar, uint32_t parity, Smem* sm, uint32_t* sync,
+                                     uint64_t limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return wait_slow(bar, parity, sm, sync, limit_ns);
+}
+
+// wait() by every lane of a warp with a warp-uniform result, so that the
+// warp runs its collective instructions (tcgen05.ld) together or not at all.
+__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, Smem* sm, uint32_t* sync,
+                                          uint64_t limit_ns) {
+    const bool ok = wait(bar, parity, sm, sync, limit_ns);
+    return __all_sync(0xffffffffu, ok);
+}
+
+// Bounded wait for work already issued (copies, MMAs), ignoring the abort
+// flag: used before the CTA exits.
+__device__ __noinline__ void wait_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > limit_ns) {
+            raise_error(LEMO_ERR_TIMEOUT);
+            return;
         }
-        for (; g < a.groups; ++g) v += a.part[g * plane + o];
-        store_pair(a, blk_prefix, m_prefix, s, n, m, v);
+    }
+}
+
+// Grid-wide barrier on counter `word` (every CTA of the grid is resident: one
+// per SM).  Every thread of the CTA calls it, after every phase, whether or
+// not the CTA has given up (a CTA that gave up passes straight through);
+// returns false once this CTA or any other gave up.
+__device__ __noinline__ bool grid_sync(const Args& a, Smem* sm, int word) {
+    __syncthreads();
+    if (threadIdx.x == 0 && !aborted(sm)) {
+        uint32_t* ctr = a.sync + word;
+        const volatile uint32_t* abort_word = a.sync + kSyncAbort;
+        fence_proxy_global();  // this CTA's stores -> later bulk copies of other CTAs
+        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
+        const uint64_t t0 = globaltimer_ns();
+        for (uint32_t n = 1;; ++n) {
+            uint32_t v;
+            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+            if (v >= gridDim.x) break;
+            if ((n & 15) == 0) {
+                if (*abort_word) {
+                    *reinterpret_cast<volatile int*>(&sm->abort_flag) = 1;
+                    break;
+                }
+                if (globaltimer_ns() - t0 > a.spin_limit_ns) {
+                    raise_error(LEMO_ERR_TIMEOUT);
+                    give_up(sm, a.sync);
+                    break;
+                }
+            }
+        }
+        fence_proxy_global();  // other CTAs' stores -> this CTA's bulk copies
+    }
+    __syncthreads();
+    return !aborted(sm);
+}
+
+// ------------------------------------------------------------ phase geometry
+// Every role walks the same sequence of units and chunks; these describe it.
+struct UnitA {  // split-K partial of the first GEMM
+    int p, R, j, z, c0, nc, n0, nt;
+};
+__device__ __forceinline__ UnitA unit_a(const Args& a, int u) {
+    UnitA t;
+    t.z = u % a.zk;
+    int v = u / a.zk;
+    t.j = v % a.nj;
+    v /= a.nj;
+    t.R = v % a.rt;
+    t.p = v / a.rt;
+    t.c0 = t.z * a.cps;
+    t.nc = min(a.kc, t.c0 + a.cps) - t.c0;
+    t.n0 = t.j * a.nt;
+    t.nt = min(a.nt, a.ldr - t.n0);
+    return t;
+}
+struct UnitC {  // one 256-column tile of the second GEMM
+    int p, R, j, n0, nt;
+};
+__device__ __forceinline__ UnitC unit_c(const Args& a, int u) {
+    UnitC t;
+    t.j = u % a.nj2;
+    const int v = u / a.nj2;
+    t.R = v % a.rt;
+    t.p = v / a.rt;
+    t.n0 = t.j * MAX_NT;
+    t.nt = min(MAX_NT, a.np - t.n0);
+    return t;
+}
+struct UnitD {  // lower-triangle tile (tn >= tm) of block pairs, one head group
+    int tn, tm, g, h0, nh;
+};
+__device__ __forceinline__ UnitD unit_d(const Args& a, int u) {
+    UnitD t;
+    t.g = u % a.groups;
+    const int idx = u / a.groups;
+    int tn = 0;
+    while ((tn + 1) * (tn + 2) / 2 <= idx) ++tn;
+    t.tn = tn;
+    t.tm = idx - tn * (tn + 1) / 2;
+    t.h0 = t.g * a.hpg;
+    t.nh = min(a.H, t.h0 + a.hpg) - t.h0;
+    return t;
+}
+
+__device__ __forceinline__ const uint8_t* xb_img(const Args& a, int R, int c, int plane) {
+    return a.xb + ((size_t)(R * a.kc + c) * 2 + plane) * IMG;
+}
+__device__ __forceinline__ uint8_t* hid_img(const Args& a, int p, int R, int c, int plane) {
+    return a.hid + ((size_t)((p * a.rt + R) * a.kc2 + c) * 2 + plane) * IMG;
+}
+__device__ __forceinline__ uint8_t* qk_img(const Args& a, int p, int R, int h, int c, int plane) {
+    return a.qk + ((size_t)(((p * a.rt + R) * a.H + h) * a.dc + c) * 2 + plane) * IMG;
+}
+
+// 8 consecutive bf16 of a weight row into a 16-byte chunk; elements whose
+// column is at or past `valid` are zero.  MODE picks the load width.
+template <int MODE>
+__device__ __forceinline__ uint4 load8(const uint16_t* src, int valid) {
+    uint4 o = make_uint4(0u, 0u, 0u, 0u);
+    if (valid <= 0) return o;
+    if (valid >= 8 && MODE == kW16) return __ldg(reinterpret_cast<const uint4*>(src));
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    if (valid >= 8 && MODE == kW4) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) w[i] = __ldg(reinterpret_cast<const uint32_t*>(src) + i);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (i < valid) w[i >> 1] |= (uint32_t)__ldg(src + i) << ((i & 1) * 16);
+    }
+    o.x = w[0]; o.y = w[1]; o.z = w[2]; o.w = w[3];
+    return o;
+}
+
+// W1[p] rows [64 c, +64) x columns [n0, n0 + nt) into an MN-major tile
+// (groups of 64 columns; columns past nt, rows past d, columns past rank: 0).
+template <int MODE>
+__device__ __forceinline__ void load_w1(const Args& a, uint8_t* dst, int p, int c, int n0, int nt,
+                                        int ltid) {
+    const uint16_t* w = p ? a.w1[1] : a.w1[0];
+    const int groups = (nt + 63) >> 6;
+    const int chunks = 64 * groups * 8;
+    for (int q = ltid; q < chunks; q += 32 * LOAD_WARPS) {
+        const int j8 = q & 7, grp = (q >> 3) % groups, k = (q >> 3) / groups;
+        const int kk = c * KCH + k, n = n0 + grp * 64 + j8 * 8;
+        int valid = min(a.rank - n, nt - (grp * 64 + j8 * 8));
+        if (kk >= a.d) valid = 0;
+        const uint4 v = load8<MODE>(w + (size_t)kk * a.rank + n, valid);
+        *reinterpret_cast<uint4*>(dst + mn_off(k, grp, j8)) = v;
+    }
+}
+
+// W2[p] rows [64 c, +64) (rank index) x padded columns [n0, n0 + nt) of
+// H * dhp (column h * dhp + e is W2 column h * dh + e for e < dh, else 0).
+template <int MODE>
+__device__ __forceinline__ void load_w2(const Args& a, uint8_t* dst, int p, int c, int n0, int nt,
+                                        int ltid) {
+    const uint16_t* w = p ? a.w2[1] : a.w2[0];
+    const int groups = nt >> 6;
+    const int chunks = 64 * groups * 8;
+    const int64_t ldw = (int64_t)a.H * a.dh;
+    for (int q = ltid; q < chunks; q += 32 * LOAD_WARPS) {
+        const int j8 = q & 7, grp = (q >> 3) % groups, k = (q >> 3) / groups;
+        const int kk = c * KCH + k, n = n0 + grp * 64 + j8 * 8;
+        const int h = n / a.dhp, e = n - h * a.dhp;
+        const int valid = kk < a.rank ? a.dh - e : 0;
+        const uint4 v = load8<MODE>(w + (size_t)kk * ldw + (int64_t)h * a.dh + e, valid);
+        *reinterpret_cast<uint4*>(dst + mn_off(k, grp, j8)) = v;
+    }
+}
+
+__global__ void __launch_bounds__(THREADS, 1) predict_kernel(const Args a) {
+    pdl_entry();
+    fence_proxy_global();  // the pooling pass's stores -> this kernel's bulk copies
+    const PlanHeader* hdr = reinterpret_cast<const PlanHeader*>(a.ws + a.lay.hdr);
+    if (!hdr->valid) return;  // every CTA leaves here, before any barrier
+    const int TB = hdr->total_blocks;
+    const int32_t* blk_prefix = reinterpret_cast<const int32_t*>(a.ws + a.lay.blk_prefix);
+    const int64_t* m_prefix = reinterpret_cast<const int64_t*>(a.ws + a.lay.m_prefix);
+
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* tiles = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    Smem* sm = reinterpret_cast<Smem*>(tiles + STAGES * STAGE_BYTES);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint64_t lim = a.spin_limit_ns;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&sm->full[s], 1 + LOAD_WARPS);
+            mbar_init(&sm->empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm->acc_full[b], 1);
+            mbar_init(&sm->acc_empty[b], LOAD_WARPS);
+        }
+        mbar_init(&sm->done, 1);
+        sm->abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(&sm->tmem_base)),
+                     "r"(TMEM_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm->tmem_base;
+
+    // Role state, carried across phases (every role counts the same chunks
+    // and accumulations).
+    uint32_t it = 0;      // stage uses
+    uint32_t acc_it = 0;  // accumulations
+    const uint32_t ring = smem_u32(tiles);
+    const int ltid = threadIdx.x - 64;  // loader / epilogue thread id (warps 2..9)
+    const int q4 = warp & 3;            // TMEM lane quadrant of an epilogue warp
+    const int hf = (warp - 2) >> 2;     // which half of the accumulator's columns
+    const int erow = q4 * 32 + lane;    // row of the tile (TMEM lane) of this thread
+    bool ok = true;
+
+    // ================================================================ phase A
+    {
+        const int nunits = 2 * a.rt * a.nj * a.zk;
+        if (warp == 0 && lane == 0) {
+            for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
+                const UnitA t = unit_a(a, u);
+                for (int ci = 0; ci < t.nc && ok; ++ci, ++it) {
+                    const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
+                    if (!(ok = wait(&sm->empty[s], ph ^ 1, sm, a.sync, lim))) break;
+                    mbar_arrive_expect_tx(&sm->full[s], 2 * IMG);
+                    bulk_load(ring + s * STAGE_BYTES, xb_img(a, t.R, t.c0 + ci, 0), IMG, &sm->full[s]);
+                    bulk_load(ring + s * STAGE_BYTES + IMG, xb_img(a, t.R, t.c0 + ci, 1), IMG, &sm->full[s]);
+                }
+            }
+        } else if (warp == 1 && lane == 0) {
+            for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
+                const UnitA t = unit_a(a, u);
+                const uint32_t b = acc_it & 1;
+                if (!(ok = wait(&sm->acc_empty[b], ((acc_it >> 1) & 1) ^ 1, sm, a.sync, lim))) break;
+                const uint32_t id = idesc(t.nt, true);
+                for (int ci = 0; ci < t.nc && ok; ++ci, ++it) {
+                    const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
+                    if (!(ok = wait(&sm->full[s], ph, sm, a.sync, lim))) break;
+                    tc_fence_after();
+                    const uint32_t st = ring + s * STAGE_BYTES;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint64_t bd = sdesc(st + 2 * IMG + k * 2048, 8192);
+                        umma(tmem + b * ACC_COLS, sdesc(st + k * 32, 16), bd, id, (ci > 0 || k > 0) ? 1u : 0u);
+                        umma(tmem + b * ACC_COLS, sdesc(st + IMG + k * 32, 16), bd, id, 1u);
+                    }
+                    umma_commit(&sm->empty[s]);
+                }
+                if (!ok) break;
+                umma_commit(&sm->acc_full[b]);
+                ++acc_it;
+            }
+        } else if (warp >= 2) {
+            for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
+                const UnitA t = unit_a(a, u);
+                for (int ci = 0; ci < t.nc && ok; ++ci, ++it) {
+                    const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
+                    if (!(ok = wait_warp(&sm->empty[s], ph ^ 1, sm, a.sync, lim))) break;
+                    uint8_t* dst = tiles + s * STAGE_BYTES + 2 * IMG;
+                    if (a.w1_mode == kW16) load_w1<kW16>(a, dst, t.p, t.c0 + ci, t.n0, t.nt, ltid);
+                    else if (a.w1_mode == kW4) load_w1<kW4>(a, dst, t.p, t.c0 + ci, t.n0, t.nt, ltid);
+                    else load_w1<kW2>(a, dst, t.p, t.c0 + ci, t.n0, t.nt, ltid);
+                    fence_proxy_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sm->full[s]);
+                }
+                if (!ok) break;
+                // epilogue: the fp32 partial of rows [128 R, +128), columns [n0, n0 + nt)
+                const uint32_t b = acc_it & 1;
+                if (!(ok = wait_warp(&sm->acc_full[b], (acc_it >> 1) & 1, sm, a.sync, lim))) break;
+                tc_fence_after();
+                const int half = t.nt >> 1;
+                const uint32_t taddr = tmem + b * ACC_COLS + ((uint32_t)(q4 * 32) << 16) + hf * half;
+                float* dst = a.part + ((size_t)(t.p * a.zk + t.z) * a.tba + t.R * TILE + erow) * a.ldr +
+                             t.n0 + hf * half;
+                for (int c = 0; c < half; c += 16) {
+                    uint32_t r[16];
+                    tmem_ld16(taddr + c, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 16; i += 4)
+                        *reinterpret_cast<uint4*>(dst + c + i) = make_uint4(r[i], r[i + 1], r[i + 2], r[i + 3]);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm->acc_empty[b]);
+                ++acc_it;
+            }
+        }
+    }
+    ok = grid_sync(a, sm, kSyncA);
+
+    // ================================================================ phase B
+    // hid[p][row][col] = relu(sum_z part[p][z][row][col]) (z in order), as
+    // hi / lo images; rows >= TB and columns >= rank are zero.
+    if (ok) {
+        const int chunks_per_row = a.kc2 * 8;
+        const int64_t items = 2LL * a.tba * chunks_per_row;
+        for (int64_t i = blockIdx.x * (int64_t)THREADS + threadIdx.x; i < items;
+             i += (int64_t)gridDim.x * THREADS) {
+            const int cj = (int)(i % chunks_per_row);
+            const int row = (int)((i / chunks_per_row) % a.tba);
+            const int p = (int)(i / ((int64_t)chunks_per_row * a.tba));
+            const int col0 = cj * 8;
+            float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            if (row < TB && col0 < a.rank) {
+                const float* src = a.part + ((size_t)p * a.zk * a.tba + row) * a.ldr + col0;
+                const size_t plane = (size_t)a.tba * a.ldr;
+                int z = 0;
+                for (; z + 4 <= a.zk; z += 4) {
+                    float4 t[8];
+#pragma unroll
+                    for (int uu = 0; uu < 4; ++uu) {
+                        t[2 * uu] = *reinterpret_cast<const float4*>(src + (z + uu) * plane);
+                        t[2 * uu + 1] = *reinterpret_cast<const float4*>(src + (z + uu) * plane + 4);
+                    }
+#pragma unroll
+                    for (int uu = 0; uu < 4; ++uu) {
+                        v[0] += t[2 * uu].x; v[1] += t[2 * uu].y; v[2] += t[2 * uu].z; v[3] += t[2 * uu].w;
+                        v[4] += t[2 * uu + 1].x; v[5] += t[2 * uu + 1].y; v[6] += t[2 * uu + 1].z; v[7] += t[2 * uu + 1].w;
+                    }
+                }
+                for (; z < a.zk; ++z) {
+                    const float4 t0 = *reinterpret_cast<const float4*>(src + z * plane);
+                    const float4 t1 = *reinterpret_cast<const float4*>(src + z * plane + 4);
+                    v[0] += t0.x; v[1] += t0.y; v[2] += t0.z; v[3] += t0.w;
+                    v[4] += t1.x; v[5] += t1.y; v[6] += t1.z; v[7] += t1.w;
+                }
+#pragma unroll
+                for (int e = 0; e < 8; ++e) v[e] = (col0 + e < a.rank) ? fmaxf(v[e], 0.f) : 0.f;
+            }
+            uint4 hi, lo;
+            split8(v, hi, lo);
+            uint8_t* im = hid_img(a, p, row / TILE, col0 / KCH, 0) + img_off(row % TILE, col0 % KCH);
+            *reinterpret_cast<uint4*>(im) = hi;
+            *reinterpret_cast<uint4*>(im + IMG) = lo;
+        }
+    }
+    ok = grid_sync(a, sm, kSyncB);
+
+    // ================================================================ phase C
+    // Qhat / Khat tiles: hid[p] (hi, lo) x W2[p], written as hi / lo images
+    // per (row tile, head, 64-column chunk of dhp).
+    if (ok) {
+        const int nunits = 2 * a.rt * a.nj2;
+        if (warp == 0 && lane == 0) {
+            for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
+                const UnitC t = unit_c(a, u);
+                for (int c = 0; c < a.kc2 && ok; ++c, ++it) {
+                    const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
+                    if (!(ok = wait(&sm->empty[s], ph ^ 1, sm, a.sync, lim))) break;
+                    mbar_arrive_expect_tx(&sm->full[s], 2 * IMG);
+                    bulk_load(ring + s * STAGE_BYTES, hid_img(a, t.p, t.R, c, 0), IMG, &sm->full[s]);
+                    bulk_load(ring + s * STAGE_BYTES + IMG, hid_img(a, t.p, t.R, c, 1), IMG, &sm->full[s]);
+                }
+            }
+        } else if (warp == 1 && lane == 0) {
+            for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
+                const UnitC t = unit_c(a, u);
+                const uint32_t b = acc_it & 1;
+                if (!(ok = wait(&sm->acc_empty[b], ((acc_it >> 1) & 1) ^ 1, sm, a.sync, lim))) break;
+                const uint32_t id = idesc(t.nt, true);
+                for (int c = 0; c < a.kc2 && ok; ++c, ++it) {
+                    const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
+                    if (!(ok = wait(&sm->full[s], ph, sm, a.sync, lim))) break;
+                    tc_fence_after();
+                    const uint32_t st = ring + s * STAGE_BYTES;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint64_t bd = sdesc(st + 2 * IMG + k * 2048, 8192);
+                        umma(tmem + b * ACC_COLS, sdesc(st + k * 32, 16), bd, id, (c > 0 || k > 0) ? 1u : 0u);
+                        umma(tmem + b * ACC_COLS, sdesc(st + IMG + k * 32, 16), bd, id, 1u);
+                    }
+                    umma_commit(&sm->empty[s]);
+                }
+                if (!ok) break;
+                umma_commit(&sm->acc_full[b]);
+                ++acc_it;
+            }
+        } else if (warp >= 2) {
+            for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
+                const UnitC t = unit_c(a, u);
+                for (int c = 0; c < a.kc2 && ok; ++c, ++it) {
+                    const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
+                    if (!(ok = wait_warp(&sm->empty[s], ph ^ 1, sm, a.sync, lim))) break;
+                    uint8_t* dst = tiles + s * STAGE_BYTES + 2 * IMG;
+                    if (a.w2_mode == kW16) load_w2<kW16>(a, dst, t.p, c, t.n0, t.nt, ltid);
+                    else if (a.w2_mode == kW4) load_w2<kW4>(a, dst, t.p, c, t.n0, t.nt, ltid);
+                    else load_w2<kW2>(a, dst, t.p, c, t.n0, t.nt, ltid);
+                    fence_proxy_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sm->full[s]);
+                }
+                if (!ok) break;
+                const uint32_t b = acc_it & 1;
+                if (!(ok = wait_warp(&sm->acc_full[b], (acc_it >> 1) & 1, sm, a.sync, lim))) break;
+                tc_fence_after();
+                const int half = t.nt >> 1;
+                const uint32_t taddr = tmem + b * ACC_COLS + ((uint32_t)(q4 * 32) << 16) + hf * half;
+                for (int c = 0; c < half; c += 16) {
+                    uint32_t r[16];
+                    tmem_ld16(taddr + c, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 16; i += 8) {
+                        const int n = t.n0 + hf * half + c + i;  // padded column (multiple of 8)
+                        const int h = n / a.dhp, e = n - h * a.dhp;
+                        float v[8];
+#pragma unroll
+                        for (int e8 = 0; e8 < 8; ++e8) v[e8] = __uint_as_float(r[i + e8]);
+                        uint4 hi, lo;
+                        split8(v, hi, lo);
+                        uint8_t* im = qk_img(a, t.p, t.R, h, e / KCH, 0) + img_off(erow, e % KCH);
+                        *reinterpret_cast<uint4*>(im) = hi;
+                        *reinterpret_cast<uint4*>(im + IMG) = lo;
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm->acc_empty[b]);
+                ++acc_it;
+            }
+        }
+    }
+    ok = grid_sync(a, sm, kSyncC);
+
+    // ================================================================ phase D
+    // Block products of one lower-triangle tile (query row tile tn, key row
+    // tile tm) for the heads of one group: per head 3 MMAs per K step (hi hi,
+    // lo hi, hi lo), then the positive part is added into 64 running sums per
+    // thread.
+    if (ok) {
+        const int nunits = a.pt * a.groups;
+        if (warp == 0 && lane == 0) {
+            for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
+                const UnitD t = unit_d(a, u);
+                for (int hh = 0; hh < t.nh && ok; ++hh)
+                    for (int c = 0; c < a.dc && ok; ++c, ++it) {
+                        const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
+                        if (!(ok = wait(&sm->empty[s], ph ^ 1, sm, a.sync, lim))) break;
+                        const int h = t.h0 + hh;
+                        const uint32_t st = ring + s * STAGE_BYTES;
+                        // the loader warps have nothing to load in this phase:
+                        // their arrivals are made here
+                        mbar_arrive_expect_tx(&sm->full[s], 4 * IMG);
+                        mbar_arrive_cnt(&sm->full[s], LOAD_WARPS);
+                        bulk_load(st, qk_img(a, 0, t.tn, h, c, 0), IMG, &sm->full[s]);
+                        bulk_load(st + IMG, qk_img(a, 0, t.tn, h, c, 1), IMG, &sm->full[s]);
+                        bulk_load(st + 2 * IMG, qk_img(a, 1, t.tm, h, c, 0), IMG, &sm->full[s]);
+                        bulk_load(st + 3 * IMG, qk_img(a, 1, t.tm, h, c, 1), IMG, &sm->full[s]);
+                    }
+            }
+        } else if (warp == 1 && lane == 0) {
+            const uint32_t id = idesc(TILE, false);
+            for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
+                const UnitD t = unit_d(a, u);
+                for (int hh = 0; hh < t.nh && ok; ++hh) {
+                    const uint32_t b = acc_it & 1;
+                    if (!(ok = wait(&sm->acc_empty[b], ((acc_it >> 1) & 1) ^ 1, sm, a.sync, lim))) break;
+                    for (int c = 0; c < a.dc && ok; ++c, ++it) {
+                        const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
+                        if (!(ok = wait(&sm->full[s], ph, sm, a.sync, lim))) break;
+                        tc_fence_after();
+                        const uint32_t st = ring + s * STAGE_BYTES;
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const uint64_t ah = sdesc(st + k * 32, 16), al = sdesc(st + IMG + k * 32, 16);
+                            const uint64_t bh = sdesc(st + 2 * IMG + k * 32, 16);
+                            const uint64_t bl = sdesc(st + 3 * IMG + k * 32, 16);
+                            umma(tmem + b * ACC_COLS, ah, bh, id, (c > 0 || k > 0) ? 1u : 0u);
+                            umma(tmem + b * ACC_COLS, al, bh, id, 1u);
+                            umma(tmem + b * ACC_COLS, ah, bl, id, 1u);
+                        }
+                        umma_commit(&sm->empty[s]);
+                    }
+                    if (!ok) break;
+                    umma_commit(&sm->acc_full[b]);
+                    ++acc_it;
+                }
+            }
+        } else if (warp >= 2) {
+            // epilogue: the accumulations the MMA thread commits, one per head
+            for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
+                const UnitD t = unit_d(a, u);
+                float tot[64];
+#pragma unroll
+                for (int i = 0; i < 64; ++i) tot[i] = 0.f;
+                for (int hh = 0; hh < t.nh; ++hh) {
+                    const uint32_t b = acc_it & 1;
+                    if (!(ok = wait_warp(&sm->acc_full[b], (acc_it >> 1) & 1, sm, a.sync, lim))) break;
+                    tc_fence_after();
+                    const uint32_t taddr = tmem + b * ACC_COLS + ((uint32_t)(q4 * 32) << 16) + hf * 64;
+#pragma unroll
+                    for (int c = 0; c < 64; c += 16) {
+                        uint32_t r[16];
+                        tmem_ld16(taddr + c, r);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) tot[c + i] += fmaxf(__uint_as_float(r[i]), 0.f);
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sm->acc_empty[b]);
+                    ++acc_it;
+                }
+                if (!ok) break;
+                const int n = t.tn * TILE + erow;
+                const int mb = t.tm * TILE + hf * 64;
+                if (a.groups == 1) {
+                    if (n < TB) {
+                        const int s = last_le(blk_prefix, a.batch + 1, n);
+                        const int b0 = blk_prefix[s], nb = blk_prefix[s + 1] - b0;
+                        float* row = a.P + m_prefix[s] + (int64_t)(n - b0) * nb - b0;
+#pragma unroll
+                        for (int i = 0; i < 64; ++i) {
+                            const int m = mb + i;
+                            if (m >= b0 && m <= n) row[m] = tot[i] * a.inv_h;
+                        }
+                    }
+                } else {
+                    float* row = a.ppart + ((size_t)t.g * a.tba + n) * a.tba + mb;
+#pragma unroll
+                    for (int i = 0; i < 64; i += 4)
+                        *reinterpret_cast<float4*>(row + i) = make_float4(tot[i], tot[i + 1], tot[i + 2], tot[i + 3]);
+                }
+            }
+        }
+    }
+    ok = grid_sync(a, sm, kSyncD);
+
+    // ================================================================ phase E
+    // P[n][m] = inv_h * sum_g ppart[g][n][m] (g in order) for the pairs of one
+    // sequence with n >= m, when the heads were split into groups ...
+    if (a.groups > 1) {
+      if (ok) {
+        const int64_t total = (int64_t)TB * TB;
+        const size_t plane = (size_t)a.tba * a.tba;
+        for (int64_t i = blockIdx.x * (int64_t)THREADS + threadIdx.x; i < total;
+             i += (int64_t)gridDim.x * THREADS) {
+            const int n = (int)(i / TB), m = (int)(i % TB);
+            if (m > n) continue;
+            const int s = last_le(blk_prefix, a.batch + 1, n);
+            const int b0 = blk_prefix[s];
+            if (m < b0) continue;
+            const float* src = a.ppart + (size_t)n * a.tba + m;
+            float v = 0.f;
+            int g = 0;
+            for (; g + 8 <= a.groups; g += 8) {
+                float t[8];
+#pragma unroll
+                for (int uu = 0; uu < 8; ++uu) t[uu] = src[(g + uu) * plane];
+#pragma unroll
+                for (int uu = 0; uu < 8; ++uu) v += t[uu];
+            }
+            for (; g < a.groups; ++g) v += src[g * plane];
+            const int nb = blk_prefix[s + 1] - b0;
+            a.P[m_prefix[s] + (int64_t)(n - b0) * nb + (m - b0)] = v * a.inv_h;
+        }
+      }
+      ok = grid_sync(a, sm, kSyncE);
+    }
+    // ... then score[g] = sum_{n = m}^{N_b - 1} P[n][m] for the token block
+    // g = (seq, m): one warp per block, lane l adds rows m + l, m + l + 32, ...
+    // in increasing order, then a fixed butterfly.
+    if (ok) {
+        const int nwarps = gridDim.x * (THREADS / 32);
+        for (int g = blockIdx.x * (THREADS / 32) + warp; g < TB; g += nwarps) {
+            const int s = last_le(blk_prefix, a.batch + 1, g);
+            const int m = g - blk_prefix[s];
+            const int nb = blk_prefix[s + 1] - blk_prefix[s];
+            const float* col = a.P + m_prefix[s] + m;
+            float sum = 0.f;
+            int n = m + lane;
+            for (; n + 96 < nb; n += 128) {
+                float t[4];
+#pragma unroll
+                for (int uu = 0; uu < 4; ++uu) t[uu] = col[(int64_t)(n + 32 * uu) * nb];
+#pragma unroll
+                for (int uu = 0; uu < 4; ++uu) sum += t[uu];
+            }
+            for (; n < nb; n += 32) sum += col[(int64_t)n * nb];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+            if (lane == 0) a.scores[g] = sum;
+        }
+    }
+
+    // ---------------------------------------------------------------- teardown
+    // Every MMA this CTA issued completes before its tensor memory is freed;
+    // every bulk copy completes before the CTA exits.
+    if (warp == 1 && lane == 0) {
+        umma_commit(&sm->done);
+        wait_drain(&sm->done, 0, lim);
+    }
+    if (warp == 0 && lane == 0 && aborted(sm)) {
+        const uint32_t first = it > STAGES ? it - STAGES : 0;
+        for (uint32_t j = first; j < it; ++j) wait_drain(&sm->full[j % STAGES], (j / STAGES) & 1, lim);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                     "r"(TMEM_COLS));
     }
 }
 

@@ -110,6 +110,7 @@ struct Args {
     const char* ws;
     WsLayout lay;
     uint64_t spin_limit_ns;
+    int shard, nshards;  // key-tile shard of every sequence computed here (1 shard: all)
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -314,7 +315,10 @@ __device__ __forceinline__ TileCoord tile_coord(const Args& a, const int64_t* ti
     c.seq = last_le(tile_prefix, a.batch + 1, t);
     c.seq_start = a.cu[c.seq];
     c.L = a.cu[c.seq + 1] - c.seq_start;
-    lemo_plan::decode_tile(c.L, t - tile_prefix[c.seq], &c.qi, &c.kj);
+    if (a.nshards > 1)
+        lemo_plan::decode_tile_shard(c.L, t - tile_prefix[c.seq], a.shard, a.nshards, &c.qi, &c.kj);
+    else
+        lemo_plan::decode_tile(c.L, t - tile_prefix[c.seq], &c.qi, &c.kj);
     return c;
 }
 
@@ -573,10 +577,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 // score[g] = sum_{n = m}^{N_b - 1} M[n][m] for the token block g = (seq, m).
 // One warp per token block: lane l adds rows n = m + l, m + l + 32, ... in
 // increasing order, then a fixed butterfly combines the 32 partial sums, so
-// the result is the same bits on every run (no float atomics).
+// the result is the same bits on every run (no float atomics).  With key-tile
+// shards, blocks whose key tile belongs to another shard get 0.
 __global__ void __launch_bounds__(256) column_sum_kernel(const float* __restrict__ mblk,
                                                          const char* __restrict__ ws, WsLayout lay,
-                                                         int batch, float* __restrict__ scores) {
+                                                         int batch, float* __restrict__ scores,
+                                                         int block, int shard, int nshards) {
     pdl_entry();
     const PlanHeader* hdr = reinterpret_cast<const PlanHeader*>(ws + lay.hdr);
     if (!hdr->valid) return;
@@ -589,6 +595,10 @@ __global__ void __launch_bounds__(256) column_sum_kernel(const float* __restrict
         const int s = last_le(blk_prefix, batch + 1, g);
         const int m = g - blk_prefix[s];
         const int nb = blk_prefix[s + 1] - blk_prefix[s];
+        if (nshards > 1 && !lemo_plan::owns_key_tile((int64_t)m * block / TN, shard, nshards)) {
+            if (lane == 0) scores[g] = 0.f;
+            continue;
+        }
         const float* col = mblk + m_prefix[s] + m;
         // rows in batches of 4 per lane (loads in flight together), added in n order
         float sum = 0.f;

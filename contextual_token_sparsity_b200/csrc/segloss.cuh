@@ -4,10 +4,10 @@
 // The tokens are processed in segments of S rows.  For one segment the host
 // runs, in stream order:
 //
-//   z   = h_seg W^T                      fp32 [S, V]   (library GEMM)
+//   z   = h_seg W^T                      fp32 [S, V]   (gemm_kernel)
 //   dz  = (softmax(z) - onehot(y)) / n   bf16 [S, V]   (row_kernel, here)
-//   dh_seg  = dz W                       bf16 [S, d]   (library GEMM)
-//   dW     += dz^T h_seg                 fp32 [V, d]   (library GEMM)
+//   dh_seg  = dz W                       bf16 [S, d]   (gemm_kernel)
+//   dW     += dz^T h_seg                 fp32 [V, d]   (gemm_kernel)
 //
 // so only one segment's logits exist at a time: the activation peak of the
 // loss is S/T of the unsegmented one.  n is the number of valid tokens of

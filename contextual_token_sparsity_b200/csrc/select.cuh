@@ -41,6 +41,8 @@ __device__ __forceinline__ T block_scan_incl(T v, T* warp_sums, T* total) {
 // ---------------------------------------------------------------------------
 // Plan: per-sequence prefix arrays of a packed batch, device-side checks of
 // cu_seqlens, and a reset of the compaction look-back state.  One CTA.
+// The score-tile prefix counts the tiles of key-tile shard `shard` of
+// `nshards` (1 shard: every tile).
 // `zero_word` (optional) is set to 0 first, so that a compaction that gives
 // up leaves K = 0 behind rather than a stale count.  `zero_blocks` (optional)
 // gets its first total_blocks entries cleared (the host only knows an upper
@@ -49,7 +51,8 @@ __device__ __forceinline__ T block_scan_incl(T v, T* warp_sums, T* total) {
 __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ cu, int batch,
                                                     int total_L, int max_seqlen, int block,
                                                     char* __restrict__ ws, WsLayout lay,
-                                                    int32_t* zero_word, float* zero_blocks) {
+                                                    int32_t* zero_word, float* zero_blocks,
+                                                    int shard, int nshards) {
     pdl_entry();
     PlanHeader* hdr = reinterpret_cast<PlanHeader*>(ws + lay.hdr);
     int64_t* tile_prefix = reinterpret_cast<int64_t*>(ws + lay.tile_prefix);
@@ -81,7 +84,8 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
             } else {
                 b_s = (L + block - 1) / block;
                 m_s = (int64_t)b_s * b_s;
-                t_s = lemo_plan::seq_tiles(L);
+                t_s = nshards > 1 ? lemo_plan::shard_seq_tiles(L, shard, nshards)
+                                  : lemo_plan::seq_tiles(L);
             }
         }
         int64_t tot_t, tot_m;

@@ -51,6 +51,8 @@ _SIGS = {
     "lemo_block_max_elems": (_I64, [_I32, _P, _I32]),
     "lemo_score_blocks": (ctypes.c_int, [ctypes.POINTER(lemo_shape), _P, _P, ctypes.c_float, _P,
                                          _P, _P, ctypes.c_size_t, _P]),
+    "lemo_score_blocks_shard": (ctypes.c_int, [ctypes.POINTER(lemo_shape), _P, _P, ctypes.c_float,
+                                               _I32, _I32, _P, _P, _P, ctypes.c_size_t, _P]),
     "lemo_select": (ctypes.c_int, [ctypes.POINTER(lemo_shape), _P, ctypes.c_float, _P, _P, _P,
                                    _P, _P, ctypes.c_size_t, _P]),
     "lemo_select_static_ws": (ctypes.c_int, [ctypes.POINTER(lemo_shape), _P, ctypes.c_float, _P,
@@ -136,6 +138,15 @@ def lemo_score_blocks(shape, q, k, scale, block_max, block_scores, ws, stream=No
                                     _ptr(block_max), _ptr(block_scores), _ptr(ws),
                                     ws.numel() * ws.element_size(), _stream(stream)),
            "lemo_score_blocks")
+
+
+def lemo_score_blocks_shard(shape, q, k, scale, shard, nshards, block_max, block_scores, ws,
+                            stream=None):
+    _check(load().lemo_score_blocks_shard(ctypes.byref(shape), _ptr(q), _ptr(k), float(scale),
+                                          int(shard), int(nshards), _ptr(block_max),
+                                          _ptr(block_scores), _ptr(ws),
+                                          ws.numel() * ws.element_size(), _stream(stream)),
+           "lemo_score_blocks_shard")
 
 
 def lemo_select(shape, block_scores, threshold, block_mask, kept_idx, cu_kept, kept_total, ws,

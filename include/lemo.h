@@ -131,6 +131,33 @@ LEMO_API lemo_status lemo_score_blocks(const lemo_shape* shape, const uint16_t* 
                               void* ws, size_t ws_bytes, lemo_stream stream);
 
 /*
+ * Block scores of one key-tile shard of each sequence (steps a1-a3 split
+ * over several GPUs for one long sequence).
+ *
+ * Jenga summary, section 6.4 "Scalability Analysis": the method scales over
+ * GPUs without extra communication on its data path.  For a sequence too
+ * long for one GPU's share of the work, the block scoring is divided by key
+ * columns: the key tiles of 256 tokens of every sequence are dealt to
+ * `nshards` shards in snake order (round i of nshards consecutive tiles gives
+ * tile i*nshards + p to shard p when i is even, to shard nshards-1-p when i
+ * is odd), so the long early columns are spread evenly.  Shard `shard`
+ * computes every score tile of its key tiles - the same tiles, with the same
+ * arithmetic, as lemo_score_blocks - so the column sums of its key blocks are
+ * complete; it writes 0 for every other block.  The sum over all shards of
+ * block_scores is therefore exactly (bit for bit) lemo_score_blocks' result:
+ * one all-reduce (sum) of total_blocks floats combines the shards.
+ *
+ * Arguments as lemo_score_blocks, plus 0 <= shard < nshards <= 4096.
+ * block_max, when given, receives only the entries of the shard's key tiles.
+ * With nshards = 1 the call is lemo_score_blocks.
+ */
+LEMO_API lemo_status lemo_score_blocks_shard(const lemo_shape* shape, const uint16_t* q,
+                                             const uint16_t* k, float scale, int32_t shard,
+                                             int32_t nshards, float* block_max,
+                                             float* block_scores, void* ws, size_t ws_bytes,
+                                             lemo_stream stream);
+
+/*
  * Threshold comparison and compaction of kept token ids (steps a4-a5).
  *
  * Jenga summary, section 4.2.1, "Layer-specific Threshold": the score of each
@@ -293,11 +320,12 @@ LEMO_API lemo_status lemo_mlp_block_scores(const lemo_shape* shape, int32_t d_ff
 
 /*
  * Workspace bytes of lemo_predict_scores for `shape`, residual width d and
- * predictor rank (the plan arrays; the block means, hidden activations and
- * predicted Q/K block embeddings, each as a pair of bf16 planes hi + lo; row-
- * padded copies of the weights for shapes whose rows are not aligned; the
- * split-K partial sums and the block-product matrices).  Returns 0 for
- * invalid arguments.  HOST-only computation.
+ * predictor rank: the plan arrays; the block means, hidden activations and
+ * predicted Q/K block embeddings, each as a pair of bf16 planes hi + lo laid
+ * out as tensor-core operand tiles; the split-K partial sums of the first
+ * predictor GEMM; the head-group partial block products and the block-product
+ * matrices; a few barrier words.  Returns 0 for invalid arguments.
+ * HOST-only computation.
  */
 LEMO_API size_t lemo_predict_workspace_size(const lemo_shape* shape, int32_t d, int32_t rank);
 
@@ -324,12 +352,18 @@ LEMO_API size_t lemo_predict_workspace_size(const lemo_shape* shape, int32_t d, 
  * block_scores DEVICE fp32 [total_blocks].
  * ws, ws_bytes DEVICE workspace of lemo_predict_workspace_size bytes,
  *              256-byte aligned.
- * fp32 accuracy on the tensor cores: every fp32 operand is split into
- * bf16 hi + lo and a product is taken as hi*b + lo*b (+ hi*lo' when both
- * operands are fp32), with fp32 accumulation; split-K and head-group sums
- * are reduced in a fixed order, so the result is deterministic.  Weights
- * need only 2-byte alignment (rows that are not 16-byte aligned are read
- * with smaller copies or through a padded copy in the workspace).
+ * Three launches: the plan, a pass that streams x once (bound by HBM
+ * bandwidth) and writes the block means, and one persistent kernel (one CTA
+ * per SM, grid-wide barriers between its phases) that runs both predictor
+ * GEMMs, the Eq. 3 block products and the column sums on the tensor cores
+ * (tcgen05, fp32 accumulation in tensor memory).  fp32 accuracy: every fp32
+ * operand is split into bf16 hi + lo and a product is taken as hi*b + lo*b
+ * (+ hi*lo' when both operands are fp32) in one fp32 accumulator; split-K and
+ * head-group sums are reduced in a fixed order, so the result is
+ * deterministic.  Weights need only 2-byte alignment: they are read with
+ * plain loads whose width follows their alignment, with the same arithmetic.
+ * A grid barrier or a tile wait that runs out reports LEMO_ERR_TIMEOUT
+ * through lemo_get_error.
  */
 LEMO_API lemo_status lemo_predict_scores(const lemo_shape* shape, int32_t d, const uint16_t* x,
                                          int64_t ld_x, const uint16_t* w1q, const uint16_t* w2q,
@@ -391,10 +425,10 @@ LEMO_API lemo_status lemo_attention_kept(const lemo_shape* shape, const uint16_t
 /*
  * Workspace bytes of lemo_segment_loss for T tokens, vocabulary V and
  * segments of seg_rows tokens: the valid-token count, the per-token loss
- * terms, 32 MiB for the library GEMMs, and ONE segment's fp32 logits plus
- * their bf16 gradient (2 x min(seg_rows, T) x round_up(V, 8) elements).
- * That last part is the activation peak that segmenting divides by T /
- * seg_rows.  Returns 0 for invalid arguments.  HOST-only computation.
+ * terms and ONE segment's fp32 logits plus their bf16 gradient
+ * (2 x min(seg_rows, T) x round_up(V, 8) elements).  That last part is the
+ * activation peak that segmenting divides by T / seg_rows.  Returns 0 for
+ * invalid arguments.  HOST-only computation.
  */
 LEMO_API size_t lemo_segment_loss_workspace_size(int64_t T, int32_t V, int32_t seg_rows);
 
@@ -433,12 +467,12 @@ LEMO_API size_t lemo_segment_loss_workspace_size(int64_t T, int32_t V, int32_t s
  * matrix 16-byte aligned; d, V, seg_rows and strides below 2^31.  With T = 0,
  * h, w and targets may be NULL (the loss is 0).
  *
- * The three GEMMs of a segment run in cuBLAS (bf16 inputs, fp32
- * accumulation, cuBLAS loaded on first use; LEMO_ERR_UNSUPPORTED if it is not
- * found); the softmax / loss / gradient of each logit row is this library's
- * kernel.  The first call on a device creates a cuBLAS handle; the GEMMs use
- * the caller's workspace.  The loss is the fixed-order sum of the per-token
- * terms (deterministic).  Logits are fp32, dz and dh are rounded to bf16.
+ * The three GEMMs of a segment run on this library's tensor-core kernel
+ * (tcgen05 on CTA pairs, bf16 inputs, fp32 accumulation in tensor memory;
+ * the logits are stored in fp32, dh rounded once to bf16, dW accumulated in
+ * fp32 segment after segment); the softmax / loss / gradient of each logit
+ * row is a separate row kernel.  The loss is the fixed-order sum of the
+ * per-token terms (deterministic); dz is rounded to bf16.
  */
 LEMO_API lemo_status lemo_segment_loss(const uint16_t* h, int64_t ld_h, int64_t T, int32_t d,
                                        const uint16_t* w, int64_t ld_w, int32_t V,
