@@ -16,7 +16,7 @@
 // in its own tensor memory.
 //
 //   warp 0 (both CTAs)  TMA: A and B slices of 64 K-elements per stage
-//                       (128-byte swizzle, no multicast) into a 6-stage ring
+//                       (128-byte swizzle, no multicast) into a 5-stage ring
 //                       of 32 KB; completion is signalled on the leader's
 //                       barrier.  K-major operands come as one box of 64 x 128,
 //                       MN-major ones as two boxes of 64 (MN) x 64 (K) rows.
@@ -24,9 +24,14 @@
 //                       the epilogue of a tile overlaps the MMAs of the next;
 //                       commits are multicast to both CTAs.
 //   warps 2-9           epilogue: tcgen05.ld of 128 rows x 256 columns (two
-//                       warps per TMEM lane quadrant, 128 columns each), then
-//                       a fp32 store, a bf16 store (round to nearest even) or
-//                       a fp32 read-add-write into the output (dW += ...).
+//                       warps per TMEM lane quadrant, 128 columns each); each
+//                       warp stages 32 rows x 128 bytes at a time in its own
+//                       double buffer (128-byte swizzle) and hands it to a TMA
+//                       store (fp32 logits, bf16 dh rounded to nearest even)
+//                       or a TMA reduce-add (dW += ..., the fp32 additions
+//                       done at L2, one per element per launch, so the result
+//                       does not depend on timing).  Rows and columns past the
+//                       output are clipped by the TMA unit.
 //
 // Tiles are taken round-robin by the pairs; consecutive tiles share the
 // operand that is read the most, so it is read from DRAM about once.  Every
@@ -61,7 +66,7 @@ constexpr int TM = 256;              // tile rows per pair (MMA M)
 constexpr int TN = 256;              // tile columns (MMA N)
 constexpr int ROWS = 128;            // A rows / B columns held by one CTA
 constexpr int KB = 64;               // K elements per stage (one 128-byte swizzle row)
-constexpr int STAGES = 6;
+constexpr int STAGES = 5;
 constexpr int A_BYTES = ROWS * KB * 2;   // 16 KB
 constexpr int B_BYTES = ROWS * KB * 2;   // 16 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -70,6 +75,8 @@ constexpr int THREADS = 32 * (2 + EPI_WARPS);
 constexpr int ACC_COLS = TN;
 constexpr int TMEM_COLS = 2 * ACC_COLS;
 constexpr int COLS_PER_THREAD = TN / 2;
+constexpr int STG_BYTES = 32 * 128;          // one staging buffer: 32 rows x 128 bytes
+constexpr int STG_PER_WARP = 2 * STG_BYTES;   // double buffered
 
 enum Epi : int { kStoreF32 = 0, kStoreBF16 = 1, kAddF32 = 2 };
 
@@ -82,15 +89,14 @@ struct Smem {
     uint32_t tmem_base;
     int abort_flag;
 };
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align slack*/ + (int)sizeof(Smem);
+constexpr int SMEM_BYTES =
+    STAGES * STAGE_BYTES + EPI_WARPS * STG_PER_WARP + 1024 /*align slack*/ + (int)sizeof(Smem);
 static_assert(SMEM_BYTES <= 232448, "exceeds the 227 KB of shared memory per CTA");
 
 struct Args {
     int M, N, K;
     int a_mn, b_mn;        // 1: the operand is MN-major (MN contiguous in memory)
-    int epi;               // Epi
-    void* out;             // [M, ld_out] fp32 or bf16
-    int64_t ld_out;
+    int epi;               // Epi (the output itself is the tensor map tm_c)
     int tiles_m, tiles_n;
     int m_fastest;         // 1: consecutive tiles step along M (they share a B tile)
     uint64_t spin_limit_ns;
@@ -186,60 +192,42 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<const uint32_t*>(&r);
 }
 
-// 16 accumulator values of one row, columns col .. col + 15 of the output.
-__device__ __forceinline__ void epi_store16(const Args& a, int64_t row, int col, const uint32_t* r) {
-    if (a.epi == kStoreBF16) {
-        uint16_t* o = static_cast<uint16_t*>(a.out) + row * a.ld_out + col;
-        if (col + 16 <= a.N) {
-            uint4 v0, v1;
-            v0.x = pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1]));
-            v0.y = pack_bf16x2(__uint_as_float(r[2]), __uint_as_float(r[3]));
-            v0.z = pack_bf16x2(__uint_as_float(r[4]), __uint_as_float(r[5]));
-            v0.w = pack_bf16x2(__uint_as_float(r[6]), __uint_as_float(r[7]));
-            v1.x = pack_bf16x2(__uint_as_float(r[8]), __uint_as_float(r[9]));
-            v1.y = pack_bf16x2(__uint_as_float(r[10]), __uint_as_float(r[11]));
-            v1.z = pack_bf16x2(__uint_as_float(r[12]), __uint_as_float(r[13]));
-            v1.w = pack_bf16x2(__uint_as_float(r[14]), __uint_as_float(r[15]));
-            reinterpret_cast<uint4*>(o)[0] = v0;
-            reinterpret_cast<uint4*>(o)[1] = v1;
-        } else {
-            for (int i = 0; i < 16 && col + i < a.N; ++i) {
-                const __nv_bfloat16 b = __float2bfloat16_rn(__uint_as_float(r[i]));
-                o[i] = *reinterpret_cast<const uint16_t*>(&b);
-            }
-        }
-        return;
-    }
-    float* o = static_cast<float*>(a.out) + row * a.ld_out + col;
-    if (col + 16 <= a.N) {
-        float4* o4 = reinterpret_cast<float4*>(o);
-        if (a.epi == kAddF32) {
-            float4 p[4];
+// TMA store / reduce-add of a staged 32-row box at output (x = column, y = row).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* tm, uint32_t src, int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(tm)),
+        "r"(src), "r"(x), "r"(y)
+        : "memory");
+}
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* tm, uint32_t src, int x, int y) {
+    asm volatile(
+        "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(tm)),
+        "r"(src), "r"(x), "r"(y)
+        : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// the staging buffer of the group before the last may be rewritten
+__device__ __forceinline__ void bulk_wait_read1() {
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// One 128-byte row of a staging buffer: eight 16-byte chunks of row `lane`,
+// chunk j at (j ^ (lane % 8)) * 16 (the 128-byte swizzle the tensor map names).
+__device__ __forceinline__ void stage_row(uint32_t buf, int lane, const uint32_t* w) {
+    const uint32_t row = buf + (uint32_t)lane * 128u;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) p[i] = o4[i];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                p[i].x += __uint_as_float(r[4 * i]);
-                p[i].y += __uint_as_float(r[4 * i + 1]);
-                p[i].z += __uint_as_float(r[4 * i + 2]);
-                p[i].w += __uint_as_float(r[4 * i + 3]);
-                o4[i] = p[i];
-            }
-        } else {
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                o4[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
-                                    __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
-        }
-    } else {
-        for (int i = 0; i < 16 && col + i < a.N; ++i)
-            o[i] = a.epi == kAddF32 ? o[i] + __uint_as_float(r[i]) : __uint_as_float(r[i]);
-    }
+    for (int j = 0; j < 8; ++j)
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + (((j ^ lane) & 7) << 4)),
+                     "r"(w[4 * j]), "r"(w[4 * j + 1]), "r"(w[4 * j + 2]), "r"(w[4 * j + 3])
+                     : "memory");
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                const Args a) {
+                const __grid_constant__ CUtensorMap tm_c, const Args a) {
     pdl_entry();
     const int64_t total_tiles = (int64_t)a.tiles_m * a.tiles_n;
     const int64_t pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
@@ -249,7 +237,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* tiles = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    Smem* sm = reinterpret_cast<Smem*>(tiles + STAGES * STAGE_BYTES);
+    uint8_t* stg = tiles + STAGES * STAGE_BYTES;  // epilogue staging buffers
+    Smem* sm = reinterpret_cast<Smem*>(stg + EPI_WARPS * STG_PER_WARP);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cta_rank();
     const bool leader = rank == 0;
@@ -284,6 +273,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         if (lane == 0) {
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_a)) : "memory");
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_b)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_c)) : "memory");
             const uint32_t ring = smem_u32(tiles);
             uint32_t it = 0;
             bool ok = true;
@@ -363,13 +353,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;
         const int colhalf = (warp - 2) >> 2;
-        const int row_in = q * 32 + lane;
         const uint32_t lane_addr =
             tmem_base + ((uint32_t)(q * 32) << 16) + colhalf * COLS_PER_THREAD;
+        const uint32_t my_stg = smem_u32(stg) + (uint32_t)(warp - 2) * STG_PER_WARP;
         uint32_t acc_empty_c[2];
         acc_empty_c[0] = map_to_rank(smem_u32(&sm->acc_empty[0]), 0);
         acc_empty_c[1] = map_to_rank(smem_u32(&sm->acc_empty[1]), 0);
-        uint32_t acc_it = 0;
+        const bool bf16_out = a.epi == kStoreBF16;
+        const int chunk = bf16_out ? 64 : 32;  // columns per staged box (128 bytes a row)
+        uint32_t acc_it = 0, nst = 0;
         bool ok = true;
         for (int64_t t = pair; ok && t < total_tiles; t += npairs, ++acc_it) {
             int tm, tn;
@@ -377,28 +369,48 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             const uint32_t buf = acc_it & 1;
             if (!(ok = wait_warp(&sm->acc_full[buf], (acc_it >> 1) & 1, sm, lim))) break;
             tc_fence_after();
-            const int64_t row = (int64_t)tm * TM + (int)rank * ROWS + row_in;
+            const int row0 = tm * TM + (int)rank * ROWS + q * 32;  // first output row of this warp
             const int col0 = tn * TN + colhalf * COLS_PER_THREAD;
-            const bool live = row < a.M;
             const uint32_t base = lane_addr + buf * ACC_COLS;
 #pragma unroll 1
-            for (int ch = 0; ch < COLS_PER_THREAD; ch += 32) {
-                uint32_t r[32];
+            for (int ch = 0; ch < COLS_PER_THREAD; ch += chunk, ++nst) {
+                uint32_t r[64];
                 tmem_ld16(base + ch, &r[0]);
                 tmem_ld16(base + ch + 16, &r[16]);
+                if (bf16_out) {
+                    tmem_ld16(base + ch + 32, &r[32]);
+                    tmem_ld16(base + ch + 48, &r[48]);
+                }
                 tmem_wait_ld();
-                if (ch + 32 == COLS_PER_THREAD) {
+                if (ch + chunk == COLS_PER_THREAD) {
                     // every read of this accumulator has landed: free it
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive_cluster(acc_empty_c[buf]);
                 }
-                if (live) {
-                    if (col0 + ch < a.N) epi_store16(a, row, col0 + ch, &r[0]);
-                    if (col0 + ch + 16 < a.N) epi_store16(a, row, col0 + ch + 16, &r[16]);
+                if (bf16_out) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        r[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+                }
+                // the staging buffer used two boxes ago has been read by its TMA
+                const uint32_t sb = my_stg + (nst & 1) * STG_BYTES;
+                if (lane == 0 && nst >= 2) bulk_wait_read1();
+                __syncwarp();
+                stage_row(sb, lane, r);
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) {
+                    if (a.epi == kAddF32)
+                        tma_reduce_add_2d(&tm_c, sb, col0 + ch, row0);
+                    else
+                        tma_store_2d(&tm_c, sb, col0 + ch, row0);
+                    bulk_commit();
                 }
             }
         }
+        if (lane == 0) bulk_wait_all();  // every store landed before the CTA exits
+        __syncwarp();
     }
 
     // ---------------------------------------------------------------- teardown

@@ -351,6 +351,23 @@ bool encode_operand(CUtensorMap* tm, const uint16_t* base, int64_t rows, int64_t
            CUDA_SUCCESS;
 }
 
+// 2-D tensor map of a GEMM output [rows, cols] (fp32 or bf16, row stride ld
+// elements), boxes of 32 rows x 128 bytes with 128-byte swizzle, for the
+// epilogue's TMA stores and reduce-adds.
+bool encode_output(CUtensorMap* tm, void* base, int64_t rows, int64_t cols, int64_t ld, bool f32) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return false;
+    const int esz = f32 ? 4 : 2;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)(ld * esz)};
+    const cuuint32_t box[2] = {(cuuint32_t)(128 / esz), 32u};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(tm, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base,
+               dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
 // CTA pairs of the GEMM kernel that fit at once (sets its shared-memory
 // limit on first use).
 int g_gemm_pairs[kMaxDevices];
@@ -391,9 +408,10 @@ lemo_status run_gemm(int dev, int sms, cudaStream_t st, const uint16_t* A, int64
                      void* out, int64_t ld_out, bool m_fastest) {
     namespace gm = lemo::gemm;
     if (M <= 0 || N <= 0) return LEMO_OK;
-    CUtensorMap ta, tb;
+    CUtensorMap ta, tb, tc;
     if (!encode_operand(&ta, A, a_mn ? K : M, a_mn ? M : K, lda, a_mn) ||
-        !encode_operand(&tb, B, b_mn ? K : N, b_mn ? N : K, ldb, b_mn))
+        !encode_operand(&tb, B, b_mn ? K : N, b_mn ? N : K, ldb, b_mn) ||
+        !encode_output(&tc, out, M, N, ld_out, epi != gm::kStoreBF16))
         return LEMO_ERR_CUDA;
     const int pairs = gemm_pairs(dev, sms);
     if (pairs <= 0) return LEMO_ERR_CUDA;
@@ -404,8 +422,6 @@ lemo_status run_gemm(int dev, int sms, cudaStream_t st, const uint16_t* A, int64
     a.a_mn = a_mn ? 1 : 0;
     a.b_mn = b_mn ? 1 : 0;
     a.epi = epi;
-    a.out = out;
-    a.ld_out = ld_out;
     a.tiles_m = (M + gm::TM - 1) / gm::TM;
     a.tiles_n = (N + gm::TN - 1) / gm::TN;
     a.m_fastest = m_fastest ? 1 : 0;
@@ -415,7 +431,7 @@ lemo_status run_gemm(int dev, int sms, cudaStream_t st, const uint16_t* A, int64
     }
     const int64_t tiles = (int64_t)a.tiles_m * a.tiles_n;
     const int64_t use = tiles < pairs ? tiles : pairs;
-    launch(gm::gemm_kernel, (unsigned)(2 * use), gm::THREADS, gm::SMEM_BYTES, st, ta, tb, a);
+    launch(gm::gemm_kernel, (unsigned)(2 * use), gm::THREADS, gm::SMEM_BYTES, st, ta, tb, tc, a);
     return launch_status();
 }
 

@@ -437,12 +437,52 @@ __device__ __forceinline__ uint4 load8(const uint16_t* src, int valid) {
     return o;
 }
 
-// W1[p] rows [64 c, +64) x columns [n0, n0 + nt) into an MN-major tile
-// (groups of 64 columns; columns past nt, rows past d, columns past rank: 0).
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// 8 consecutive bf16 of a weight row (columns at or past `valid` read as
+// zero) into the 16-byte chunk at shared address dst.  kW16 and kW4 issue
+// asynchronous copies (cp.async, zero fill past the source bytes); kW2 loads
+// and stores directly.
 template <int MODE>
-__device__ __forceinline__ void load_w1(const Args& a, uint8_t* dst, int p, int c, int n0, int nt,
-                                        int ltid) {
+__device__ __forceinline__ void copy8(uint32_t dst, uint8_t* dst_ptr, const uint16_t* src,
+                                      const uint16_t* safe, int valid) {
+    if (MODE == kW16) {
+        const int v = valid < 0 ? 0 : (valid > 8 ? 8 : valid);
+        cp_async16(dst, v > 0 ? src : safe, (uint32_t)v * 2u);
+    } else if (MODE == kW4) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int e = 2 * u;
+            const uint32_t bytes = valid >= e + 2 ? 4u : (valid == e + 1 ? 2u : 0u);
+            cp_async4(dst + 4 * u, bytes ? src + e : safe, bytes);
+        }
+    } else {
+        *reinterpret_cast<uint4*>(dst_ptr) = load8<kW2>(src, valid);
+    }
+}
+
+// W1[p] rows [64 c, +64) x columns [n0, n0 + nt) into an MN-major tile
+// (groups of 64 columns; columns past nt, rows past d, columns past rank: 0),
+// issued as asynchronous copies (the caller commits and waits).
+template <int MODE>
+__device__ __forceinline__ void issue_w1(const Args& a, uint8_t* dst, int p, int c, int n0, int nt,
+                                         int ltid) {
     const uint16_t* w = p ? a.w1[1] : a.w1[0];
+    const uint32_t dsa = smem_u32(dst);
     const int groups = (nt + 63) >> 6;
     const int chunks = 64 * groups * 8;
     for (int q = ltid; q < chunks; q += 32 * LOAD_WARPS) {
@@ -450,17 +490,18 @@ __device__ __forceinline__ void load_w1(const Args& a, uint8_t* dst, int p, int 
         const int kk = c * KCH + k, n = n0 + grp * 64 + j8 * 8;
         int valid = min(a.rank - n, nt - (grp * 64 + j8 * 8));
         if (kk >= a.d) valid = 0;
-        const uint4 v = load8<MODE>(w + (size_t)kk * a.rank + n, valid);
-        *reinterpret_cast<uint4*>(dst + mn_off(k, grp, j8)) = v;
+        const uint32_t o = mn_off(k, grp, j8);
+        copy8<MODE>(dsa + o, dst + o, w + (size_t)kk * a.rank + n, w, valid);
     }
 }
 
 // W2[p] rows [64 c, +64) (rank index) x padded columns [n0, n0 + nt) of
 // H * dhp (column h * dhp + e is W2 column h * dh + e for e < dh, else 0).
 template <int MODE>
-__device__ __forceinline__ void load_w2(const Args& a, uint8_t* dst, int p, int c, int n0, int nt,
-                                        int ltid) {
+__device__ __forceinline__ void issue_w2(const Args& a, uint8_t* dst, int p, int c, int n0, int nt,
+                                         int ltid) {
     const uint16_t* w = p ? a.w2[1] : a.w2[0];
+    const uint32_t dsa = smem_u32(dst);
     const int groups = nt >> 6;
     const int chunks = 64 * groups * 8;
     const int64_t ldw = (int64_t)a.H * a.dh;
@@ -469,8 +510,8 @@ __device__ __forceinline__ void load_w2(const Args& a, uint8_t* dst, int p, int 
         const int kk = c * KCH + k, n = n0 + grp * 64 + j8 * 8;
         const int h = n / a.dhp, e = n - h * a.dhp;
         const int valid = kk < a.rank ? a.dh - e : 0;
-        const uint4 v = load8<MODE>(w + (size_t)kk * ldw + (int64_t)h * a.dh + e, valid);
-        *reinterpret_cast<uint4*>(dst + mn_off(k, grp, j8)) = v;
+        const uint32_t o = mn_off(k, grp, j8);
+        copy8<MODE>(dsa + o, dst + o, w + (size_t)kk * ldw + (int64_t)h * a.dh + e, w, valid);
     }
 }
 
@@ -565,18 +606,32 @@ __global__ void __launch_bounds__(THREADS, 1) predict_kernel(const Args a) {
         } else if (warp >= 2) {
             for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
                 const UnitA t = unit_a(a, u);
+                // the copies of chunk ci + 1 are issued before chunk ci is
+                // waited for: two chunks in flight per thread
+                uint32_t prev = 0;
                 for (int ci = 0; ci < t.nc && ok; ++ci, ++it) {
                     const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
                     if (!(ok = wait_warp(&sm->empty[s], ph ^ 1, sm, a.sync, lim))) break;
                     uint8_t* dst = tiles + s * STAGE_BYTES + 2 * IMG;
-                    if (a.w1_mode == kW16) load_w1<kW16>(a, dst, t.p, t.c0 + ci, t.n0, t.nt, ltid);
-                    else if (a.w1_mode == kW4) load_w1<kW4>(a, dst, t.p, t.c0 + ci, t.n0, t.nt, ltid);
-                    else load_w1<kW2>(a, dst, t.p, t.c0 + ci, t.n0, t.nt, ltid);
+                    if (a.w1_mode == kW16) issue_w1<kW16>(a, dst, t.p, t.c0 + ci, t.n0, t.nt, ltid);
+                    else if (a.w1_mode == kW4) issue_w1<kW4>(a, dst, t.p, t.c0 + ci, t.n0, t.nt, ltid);
+                    else issue_w1<kW2>(a, dst, t.p, t.c0 + ci, t.n0, t.nt, ltid);
+                    cp_commit();
+                    if (ci > 0) {
+                        cp_wait<1>();
+                        fence_proxy_smem();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&sm->full[prev]);
+                    }
+                    prev = s;
+                }
+                cp_wait<0>();
+                if (!ok) break;
+                if (t.nc > 0) {
                     fence_proxy_smem();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&sm->full[s]);
+                    if (lane == 0) mbar_arrive(&sm->full[prev]);
                 }
-                if (!ok) break;
                 // epilogue: the fp32 partial of rows [128 R, +128), columns [n0, n0 + nt)
                 const uint32_t b = acc_it & 1;
                 if (!(ok = wait_warp(&sm->acc_full[b], (acc_it >> 1) & 1, sm, a.sync, lim))) break;
@@ -618,25 +673,23 @@ __global__ void __launch_bounds__(THREADS, 1) predict_kernel(const Args a) {
             if (row < TB && col0 < a.rank) {
                 const float* src = a.part + ((size_t)p * a.zk * a.tba + row) * a.ldr + col0;
                 const size_t plane = (size_t)a.tba * a.ldr;
-                int z = 0;
-                for (; z + 4 <= a.zk; z += 4) {
-                    float4 t[8];
+                // z in increasing order, the loads of eight planes in flight
+                for (int z = 0; z < a.zk; z += 8) {
+                    float4 t[16];
 #pragma unroll
-                    for (int uu = 0; uu < 4; ++uu) {
-                        t[2 * uu] = *reinterpret_cast<const float4*>(src + (z + uu) * plane);
-                        t[2 * uu + 1] = *reinterpret_cast<const float4*>(src + (z + uu) * plane + 4);
+                    for (int uu = 0; uu < 8; ++uu) {
+                        if (z + uu < a.zk) {
+                            t[2 * uu] = *reinterpret_cast<const float4*>(src + (z + uu) * plane);
+                            t[2 * uu + 1] = *reinterpret_cast<const float4*>(src + (z + uu) * plane + 4);
+                        }
                     }
 #pragma unroll
-                    for (int uu = 0; uu < 4; ++uu) {
-                        v[0] += t[2 * uu].x; v[1] += t[2 * uu].y; v[2] += t[2 * uu].z; v[3] += t[2 * uu].w;
-                        v[4] += t[2 * uu + 1].x; v[5] += t[2 * uu + 1].y; v[6] += t[2 * uu + 1].z; v[7] += t[2 * uu + 1].w;
+                    for (int uu = 0; uu < 8; ++uu) {
+                        if (z + uu < a.zk) {
+                            v[0] += t[2 * uu].x; v[1] += t[2 * uu].y; v[2] += t[2 * uu].z; v[3] += t[2 * uu].w;
+                            v[4] += t[2 * uu + 1].x; v[5] += t[2 * uu + 1].y; v[6] += t[2 * uu + 1].z; v[7] += t[2 * uu + 1].w;
+                        }
                     }
-                }
-                for (; z < a.zk; ++z) {
-                    const float4 t0 = *reinterpret_cast<const float4*>(src + z * plane);
-                    const float4 t1 = *reinterpret_cast<const float4*>(src + z * plane + 4);
-                    v[0] += t0.x; v[1] += t0.y; v[2] += t0.z; v[3] += t0.w;
-                    v[4] += t1.x; v[5] += t1.y; v[6] += t1.z; v[7] += t1.w;
                 }
 #pragma unroll
                 for (int e = 0; e < 8; ++e) v[e] = (col0 + e < a.rank) ? fmaxf(v[e], 0.f) : 0.f;
@@ -692,18 +745,30 @@ __global__ void __launch_bounds__(THREADS, 1) predict_kernel(const Args a) {
         } else if (warp >= 2) {
             for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
                 const UnitC t = unit_c(a, u);
+                uint32_t prev = 0;
                 for (int c = 0; c < a.kc2 && ok; ++c, ++it) {
                     const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
                     if (!(ok = wait_warp(&sm->empty[s], ph ^ 1, sm, a.sync, lim))) break;
                     uint8_t* dst = tiles + s * STAGE_BYTES + 2 * IMG;
-                    if (a.w2_mode == kW16) load_w2<kW16>(a, dst, t.p, c, t.n0, t.nt, ltid);
-                    else if (a.w2_mode == kW4) load_w2<kW4>(a, dst, t.p, c, t.n0, t.nt, ltid);
-                    else load_w2<kW2>(a, dst, t.p, c, t.n0, t.nt, ltid);
+                    if (a.w2_mode == kW16) issue_w2<kW16>(a, dst, t.p, c, t.n0, t.nt, ltid);
+                    else if (a.w2_mode == kW4) issue_w2<kW4>(a, dst, t.p, c, t.n0, t.nt, ltid);
+                    else issue_w2<kW2>(a, dst, t.p, c, t.n0, t.nt, ltid);
+                    cp_commit();
+                    if (c > 0) {
+                        cp_wait<1>();
+                        fence_proxy_smem();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&sm->full[prev]);
+                    }
+                    prev = s;
+                }
+                cp_wait<0>();
+                if (!ok) break;
+                if (a.kc2 > 0) {
                     fence_proxy_smem();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&sm->full[s]);
+                    if (lane == 0) mbar_arrive(&sm->full[prev]);
                 }
-                if (!ok) break;
                 const uint32_t b = acc_it & 1;
                 if (!(ok = wait_warp(&sm->acc_full[b], (acc_it >> 1) & 1, sm, a.sync, lim))) break;
                 tc_fence_after();
@@ -856,15 +921,16 @@ __global__ void __launch_bounds__(THREADS, 1) predict_kernel(const Args a) {
             if (m < b0) continue;
             const float* src = a.ppart + (size_t)n * a.tba + m;
             float v = 0.f;
-            int g = 0;
-            for (; g + 8 <= a.groups; g += 8) {
-                float t[8];
+            // g in increasing order, sixteen loads in flight
+            for (int g = 0; g < a.groups; g += 16) {
+                float t[16];
 #pragma unroll
-                for (int uu = 0; uu < 8; ++uu) t[uu] = src[(g + uu) * plane];
+                for (int uu = 0; uu < 16; ++uu)
+                    if (g + uu < a.groups) t[uu] = src[(g + uu) * plane];
 #pragma unroll
-                for (int uu = 0; uu < 8; ++uu) v += t[uu];
+                for (int uu = 0; uu < 16; ++uu)
+                    if (g + uu < a.groups) v += t[uu];
             }
-            for (; g < a.groups; ++g) v += src[g * plane];
             const int nb = blk_prefix[s + 1] - b0;
             a.P[m_prefix[s] + (int64_t)(n - b0) * nb + (m - b0)] = v * a.inv_h;
         }

@@ -88,8 +88,9 @@ def kept_offsets(kept_total, world: int, group=None):
 class SplitLayer:
     """One layer of one long sequence on rank `rank` of `world` GPUs: device
     buffers and the steps, in order (score -> combine -> select -> gather ->
-    scatter).  ``x_shard`` / ``y_shard`` passed to gather / scatter are this
-    rank's rows of the residual and of the sublayer output."""
+    scatter).  ``x_shard`` passed to gather / scatter is this rank's rows of
+    the residual; ``y_shard`` the sublayer output of this rank's kept rows, in
+    their (compact) order."""
 
     def __init__(self, L: int, H: int, dh: int, block: int, d: int, rank: int, world: int,
                  pad_to: int = 128, device="cuda", group=None):

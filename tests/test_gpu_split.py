@@ -95,11 +95,12 @@ def test_split_flow_matches_unsharded_layer(world):
         sl.select(theta)
         xs = to_device_bf16(x[sl.lo:sl.hi])
         ys = sl.gather(xs)
-        sl.scatter(xs, to_device_bf16(y_out[sl.lo:sl.hi]))
-        assert lemo.lemo_get_error() == lemo.LEMO_OK
         Kr = int(sl.kept_total.item())
-        idx = sl.kept_idx[:Kr].cpu().numpy() + sl.lo
         off = sum(counts)
+        # the sublayer output of this rank's kept rows, in the global kept order
+        sl.scatter(xs, to_device_bf16(y_out[off:off + max(Kr, 1)]))
+        assert lemo.lemo_get_error() == lemo.LEMO_OK
+        idx = sl.kept_idx[:Kr].cpu().numpy() + sl.lo
         assert np.array_equal(ys[:Kr].view(torch.int16).cpu().numpy(),
                               y_ref[off:off + Kr].view(torch.int16).cpu().numpy())
         assert np.array_equal(xs.view(torch.int16).cpu().numpy(),
