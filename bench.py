@@ -461,12 +461,57 @@ def run_lemo(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(args.workload, budget_s=args.cpu_seconds)
 
+    if world == 1 and not args.no_extensions:
+        del q, k, y_out, x0, x, layers
+        out["extensions"] = run_extensions(args)
+
     if world > 1:
         import torch.distributed as dist
         dist.barrier(device_ids=[local])
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(out), flush=True)
+
+
+EXTENSIONS = ("predict-llama13b-32k", "lmhead-llama7b-16k", "attn-llama7b-16k", "mlp-llama7b-16k")
+
+
+def run_extensions(args):
+    """Each extension workload, briefly, in the same run (one GPU): the
+    summary of its own line - throughput, time per step, the roofline of its
+    dominant kernel, per-kernel times and the clocks - so that every row is
+    measured by the default benchmark run.  The full line (with e2e and the
+    CPU oracle) comes from `bench.py --workload W`."""
+    import copy
+
+    import torch
+    global _COLLECT
+    res = {}
+    for wl in EXTENSIONS:
+        sub = copy.copy(args)
+        sub.workload = wl
+        sub.steps = max(3, min(args.steps, 10))
+        sub.warmup = 3
+        sub.no_e2e = True
+        sub.no_cpu_baseline = True
+        _COLLECT = []
+        try:
+            {"lmhead-llama7b-16k": run_segloss, "attn-llama7b-16k": run_attention,
+             "predict-llama13b-32k": run_predict, "mlp-llama7b-16k": run_mlp}[wl](sub)
+            o = _COLLECT[-1]
+            r = o.get("roofline", {})
+            res[wl] = {"metric": o["metric"], "value": o["value"], "unit": o["unit"],
+                       "steps": o["steps"], "ms_per_step": o["ms_per_step"],
+                       "roofline": {k_: r.get(k_) for k_ in ("bound", "kernel", "achieved", "peak",
+                                                             "unit", "frac")},
+                       "kernels_us": o.get("kernels_us"), "clocks": o.get("clocks")}
+        except Exception as e:  # noqa: BLE001 - reported, not hidden
+            res[wl] = {"error": f"{type(e).__name__}: {e}"}
+        finally:
+            _COLLECT = None
+            torch.cuda.synchronize()
+            torch.cuda.empty_cache()
+    return res
 
 
 def naive_movement(x, y_out, layers, kept, fused_us, reps: int = 10):
@@ -690,12 +735,7 @@ def run_segloss(args):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = ext_cpu_baseline("lmhead-llama7b-16k", args.cpu_seconds)
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier(device_ids=[local])
-        dist.destroy_process_group()
-    if rank == 0:
-        print(json.dumps(out), flush=True)
+    _finish(out, world, local, rank)
 
 
 # ----------------------------------------------------------------------------
@@ -789,7 +829,13 @@ def torch_empty_pinned(shape, dtype):
     return torch.empty(shape, dtype=dtype).pin_memory()
 
 
+_COLLECT = None  # a list while the headline run gathers the extension lines
+
+
 def _finish(out, world, local, rank):
+    if _COLLECT is not None:  # an extension run inside the headline run (one rank)
+        _COLLECT.append(out)
+        return
     if world > 1:
         import torch.distributed as dist
         dist.barrier(device_ids=[local])
@@ -916,6 +962,108 @@ def run_attention(args):
                           lambda: call(dx.view(torch.bfloat16), bf(dq), bf(dk), bf(dv)))
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = ext_cpu_baseline("attn-llama7b-16k", args.cpu_seconds)
+    _finish(out, world, local, rank)
+
+
+SPLIT_METRIC = "tokens/sec per layer (score+select+gather+scatter), one sequence split over the GPUs"
+
+
+def run_split(args):
+    """One long sequence split over the ranks (strong scaling): each rank
+    scores the key blocks of its key tiles (lemo_score_blocks_shard), one
+    all-reduce of the block scores gives every rank the full scores, and each
+    rank selects, gathers and scatters the kept rows of its own token shard.
+    Q and K are replicated on every rank; the residual and the sublayer output
+    are sharded by tokens."""
+    import torch
+
+    from contextual_token_sparsity_b200 import lemo, split, synth
+    from contextual_token_sparsity_b200.pipeline import to_device_bf16
+
+    world, rank, local = dist_env()
+    dev, gpu_id = _setup_device(world, local)
+    lemo.load()
+    w = synth.WORKLOADS[args.workload]
+    if len(w.lengths) != 1:
+        raise ValueError("--split-sequence takes a workload of one sequence")
+    nl, L = w.layers, w.total_L
+    thetas = thresholds(args.workload, nl)
+    if thetas is None:
+        raise RuntimeError(f"stored thresholds tests/golden/{args.workload}.json are missing")
+    host = [synth.make_workload(args.workload, l, with_x=True) for l in range(nl)]
+    layers = [split.SplitLayer(L, w.H, w.dh, w.block, w.d, rank, world, pad_to=PAD_TO, device=dev)
+              for _ in range(nl)]
+    lo, hi = layers[0].lo, layers[0].hi
+    q = [to_device_bf16(h["q"], dev) for h in host]
+    k = [to_device_bf16(h["k"], dev) for h in host]
+    y = [to_device_bf16(np.ascontiguousarray(h["y_out"][lo:hi]), dev) for h in host]
+    x = to_device_bf16(np.ascontiguousarray(host[0]["x"][lo:hi]), dev)
+
+    def step(evs=None, qq=q, kk=k, xx=x, yy=y):
+        for l in range(nl):
+            sl = layers[l]
+            if evs is not None:
+                evs[4 * l].record()
+            sl.score(qq[l], kk[l])
+            if evs is not None:
+                evs[4 * l + 1].record()
+            sl.select(thetas[l])
+            if evs is not None:
+                evs[4 * l + 2].record()
+            sl.gather(xx)
+            sl.scatter(xx, yy[l])
+            if evs is not None:
+                evs[4 * l + 3].record()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = lemo.lemo_get_error()
+    if st != lemo.LEMO_OK:
+        raise RuntimeError(f"device error during warm-up: {lemo.STATUS.get(st, st)}")
+    kept_local = [int(sl.kept_total.item()) for sl in layers]
+    elapsed, clk, ev = _timed(step, args.steps, world, local, dev, gpu_id, 4 * nl)
+    st = lemo.lemo_get_error()
+    if st != lemo.LEMO_OK:
+        raise RuntimeError(f"device error in timed region: {lemo.STATUS.get(st, st)}")
+    step_s = max_over_ranks(elapsed, world, dev) / args.steps
+    us = {"score+allreduce": statistics.fmean(_mean_us(ev, 4 * l, 4 * l + 1) for l in range(nl)),
+          "select": statistics.fmean(_mean_us(ev, 4 * l + 1, 4 * l + 2) for l in range(nl)),
+          "gather+scatter": statistics.fmean(_mean_us(ev, 4 * l + 2, 4 * l + 3)
+                                             for l in range(nl))}
+    kept_all = [int(sl.offsets()[-1].item()) for sl in layers]
+    out = _header(SPLIT_METRIC, args, world, step_s, nl * L / step_s)
+    out["scaling"] = "strong"
+    out["config"] = {"workload": f"{args.workload}: {w.name}", "layers": nl, "seq_lens": [L],
+                     "heads": w.H, "head_dim": w.dh, "block": w.block, "d": w.d,
+                     "keep": list(w.keep), "kept_tokens": kept_all,
+                     "kept_tokens_this_rank": kept_local, "token_shard": [lo, hi],
+                     "parallelism": f"one sequence over {world} rank(s): key-tile shards of the "
+                                    "scoring (snake order), one all-reduce of the block scores "
+                                    "per layer, token shards of the movement; Q and K replicated",
+                     "l2": "not flushed; each step streams "
+                           f"{nl * 2 * L * w.H * w.dh * 2 / 1e9:.2f} GB of Q/K (> 126 MB L2)"}
+    out["kernels_us"] = {k_: round(v, 2) for k_, v in us.items()}
+    out["gpu_launches"] = 7 * nl * args.steps
+    out["clocks"] = clk
+    if not args.no_e2e:
+        pin = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).pin_memory()  # noqa
+        hq = [pin(h["q"]) for h in host]
+        hk = [pin(h["k"]) for h in host]
+        hy = [pin(h["y_out"][lo:hi]) for h in host]
+        hx = pin(host[0]["x"][lo:hi])
+        hx_out = torch_empty_pinned(hx.shape, hx.dtype)
+        dq = [torch.empty(t.shape, dtype=torch.int16, device=dev) for t in hq]
+        dk = [torch.empty(t.shape, dtype=torch.int16, device=dev) for t in hk]
+        dy = [torch.empty(t.shape, dtype=torch.int16, device=dev) for t in hy]
+        dx = torch.empty(hx.shape, dtype=torch.int16, device=dev)
+        bf = lambda ts: [t.view(torch.bfloat16) for t in ts]  # noqa: E731
+        out["e2e"] = _e2e(max(3, min(args.steps, args.e2e_steps)), world, local, dev, nl * L / world,
+                          list(zip(hq, dq)) + list(zip(hk, dk)) + list(zip(hy, dy)) + [(hx, dx)],
+                          [(dx, hx_out)],
+                          lambda: step(None, bf(dq), bf(dk), dx.view(torch.bfloat16), bf(dy)))
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(args.workload, budget_s=args.cpu_seconds)
     _finish(out, world, local, rank)
 
 
@@ -1417,6 +1565,11 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--no-extensions", action="store_true",
+                    help="skip the short runs of the extension workloads in the headline line")
+    ap.add_argument("--split-sequence", action="store_true",
+                    help="split each sequence over the ranks (strong scaling) instead of one "
+                         "replica per rank")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -1432,6 +1585,8 @@ def main(argv=None):
             extensions[args.workload](args)
     elif args.impl == "reference":
         run_reference(args)
+    elif args.split_sequence:
+        run_split(args)
     else:
         run_lemo(args)
 

@@ -31,6 +31,7 @@ std::mutex g_mu;
 int g_sms[kMaxDevices];              // 0 = not queried yet
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 int g_skip_publish_tile = -1;
+int g_predict_skip_cta = -1;
 int64_t g_spin_ns = kDefaultSpinNs;
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -231,8 +232,10 @@ lemo_status check_move(const void* x, int64_t ld_x, int64_t x_rows, int32_t d, c
 struct PredictLayout {
     lemo::WsLayout base;
     // byte offsets: block-mean images, split-K partials, hidden-activation
-    // images, Qhat / Khat images, head-group partial products, barrier words
-    size_t xb, part, hid, qk, ppart, sync, total;
+    // images, Qhat / Khat images, head-group partial products, barrier words,
+    // padded weight planes
+    size_t xb, part, hid, qk, ppart, sync, w1p, w2p, total;
+    int ldw1;        // row length of the padded W1 planes (rank rounded up to 8)
     int64_t tb;      // upper bound of the number of token blocks
     int rt, tba;     // row tiles of 128 token blocks
     int kc, kc2;     // 64-column chunks of d and of the rank
@@ -276,7 +279,7 @@ PredictLayout predict_layout(const lemo_shape* s, int d, int rank) {
     p.pt = (int)(pt < INT_MAX ? pt : INT_MAX);
     int64_t groups = (kTarget + pt - 1) / pt;
     if (groups > s->H) groups = s->H;
-    while (groups > 1 && groups * (int64_t)p.tba * p.tba * 4 > ((int64_t)64 << 20)) --groups;
+    while (groups > 1 && groups * (int64_t)p.tba * p.tba * 4 > ((int64_t)256 << 20)) --groups;
     if (groups < 1) groups = 1;
     p.hpg = (int)((s->H + groups - 1) / groups);
     p.groups = (s->H + p.hpg - 1) / p.hpg;
@@ -293,8 +296,10 @@ PredictLayout predict_layout(const lemo_shape* s, int d, int rank) {
     p.part = take(4 * (size_t)2 * p.zk * p.tba * p.ldr);
     p.hid = take((size_t)2 * rt * p.kc2 * 2 * pr::IMG);
     p.qk = take((size_t)2 * rt * s->H * p.dc * 2 * pr::IMG);
-    p.ppart = off;
-    if (p.groups > 1) off = lemo::align_up(off + 4 * (size_t)p.groups * p.tba * p.tba, 256);
+    p.ppart = take(4 * (size_t)p.groups * p.tba * p.tba);
+    p.ldw1 = (rank + 7) / 8 * 8;
+    p.w1p = take((size_t)2 * d * p.ldw1 * 2);
+    p.w2p = take((size_t)2 * rank * p.np * 2);
     p.total = off;
     return p;
 }
@@ -324,7 +329,9 @@ SegLayout seg_layout(int64_t T, int V, int seg_rows) {
     l.n_valid = off; off = lemo::align_up(off + 4, 256);
     l.token_loss = off; off = lemo::align_up(off + 4 * (size_t)(T > 0 ? T : 1), 256);
     l.z = off; off = lemo::align_up(off + 4 * (size_t)l.rows * l.ld, 256);
-    l.g = off; off = lemo::align_up(off + 2 * (size_t)l.rows * l.ld, 256);
+    // two segments of dz when there are several: dW is accumulated once per
+    // pair of segments (K = 2 segments), which halves its read-add-write
+    l.g = off; off = lemo::align_up(off + 2 * (size_t)(T > seg_rows ? 2 : 1) * l.rows * l.ld, 256);
     l.total = off;
     return l;
 }
@@ -364,6 +371,22 @@ bool encode_output(CUtensorMap* tm, void* base, int64_t rows, int64_t cols, int6
     const cuuint32_t estr[2] = {1, 1};
     return enc(tm, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base,
                dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+// 2-D tensor map of a bf16 weight matrix [rows, cols] (row stride ld
+// elements, 16-byte aligned rows), boxes of 64 columns x 64 rows with
+// 128-byte swizzle: the MN-major operand tiles of the predictor GEMMs.
+bool encode_weight(CUtensorMap* tm, const uint16_t* base, int64_t rows, int64_t cols, int64_t ld) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
+    const cuuint32_t box[2] = {64u, 64u};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(base), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
            CUDA_SUCCESS;
 }
@@ -810,11 +833,50 @@ lemo_status lemo_predict_scores(const lemo_shape* shape, int32_t d, const uint16
             g_prod_smem_set[dev] = true;
         }
     }
-    // block means, as hi / lo operand images (and the barrier words cleared)
+    // weights that TMA cannot read in place go through padded planes
+    const bool pad_w1 = !(rank % 8 == 0 && aligned(w1q, 16) && aligned(w1k, 16));
+    const bool pad_w2 = !(shape->dh % pr::KCH == 0 && aligned(w2q, 16) && aligned(w2k, 16));
+    uint16_t* w1p = reinterpret_cast<uint16_t*>(w + p.w1p);
+    uint16_t* w2p = reinterpret_cast<uint16_t*>(w + p.w2p);
+    pr::PadArgs pa = {};
+    pa.w1[0] = w1q;
+    pa.w1[1] = w1k;
+    pa.w2[0] = w2q;
+    pa.w2[1] = w2k;
+    if (pad_w1) {
+        pa.w1p[0] = w1p;
+        pa.w1p[1] = w1p + (size_t)d * p.ldw1;
+    }
+    if (pad_w2) {
+        pa.w2p[0] = w2p;
+        pa.w2p[1] = w2p + (size_t)rank * p.np;
+    }
+    pa.d = d;
+    pa.rank = rank;
+    pa.ldw1 = p.ldw1;
+    pa.H = shape->H;
+    pa.dh = shape->dh;
+    pa.dhp = p.dhp;
+    pa.w1_vec4 = rank % 2 == 0 && aligned(w1q, 4) && aligned(w1k, 4);
+    pa.w2_vec4 = shape->dh % 2 == 0 && aligned(w2q, 4) && aligned(w2k, 4);
+    pr::Maps maps;
+    for (int i = 0; i < 2; ++i) {
+        const bool ok1 = pad_w1 ? encode_weight(&maps.w1[i], pa.w1p[i], d, p.ldw1, p.ldw1)
+                                : encode_weight(&maps.w1[i], pa.w1[i], d, rank, rank);
+        const bool ok2 = pad_w2 ? encode_weight(&maps.w2[i], pa.w2p[i], rank, p.np, p.np)
+                                : encode_weight(&maps.w2[i], pa.w2[i], rank,
+                                                (int64_t)shape->H * shape->dh,
+                                                (int64_t)shape->H * shape->dh);
+        if (!ok1 || !ok2) return LEMO_ERR_CUDA;
+    }
+    // block means, as hi / lo operand images (and the barrier words cleared,
+    // the weight planes padded)
+    const int npad = (pad_w1 || pad_w2) ? pr::kPadCtas : 0;
     launch(pr::pool_kernel,
-           dim3((unsigned)p.tba, (unsigned)((p.kc * pr::KCH + pr::kPoolCols - 1) / pr::kPoolCols)),
-           pr::kPoolThreads, 0, st, x, ld_x, d, p.kc, shape->cu_seqlens, shape->batch,
-           shape->block, w, lay, reinterpret_cast<uint8_t*>(w + p.xb), sync);
+           dim3((unsigned)(npad + p.tba),
+                (unsigned)((p.kc * pr::KCH + pr::kPoolCols - 1) / pr::kPoolCols)),
+           pr::kPoolThreads, 0, st, x, ld_x, d, p.kc, npad, shape->cu_seqlens, shape->batch,
+           shape->block, w, lay, reinterpret_cast<uint8_t*>(w + p.xb), sync, pa);
     if ((e = launch_status()) != LEMO_OK) return e;
     pr::Args a;
     a.ws = w;
@@ -841,30 +903,20 @@ lemo_status lemo_predict_scores(const lemo_shape* shape, int32_t d, const uint16
     a.groups = p.groups;
     a.hpg = p.hpg;
     a.inv_h = 1.f / (float)shape->H;
-    a.w1[0] = w1q;
-    a.w1[1] = w1k;
-    a.w2[0] = w2q;
-    a.w2[1] = w2k;
-    a.w1_mode = (rank % 8 == 0 && aligned(w1q, 16) && aligned(w1k, 16))  ? pr::kW16
-                : (rank % 2 == 0 && aligned(w1q, 4) && aligned(w1k, 4)) ? pr::kW4
-                                                                         : pr::kW2;
-    a.w2_mode = (shape->dh % 8 == 0 && aligned(w2q, 16) && aligned(w2k, 16))  ? pr::kW16
-                : (shape->dh % 2 == 0 && aligned(w2q, 4) && aligned(w2k, 4)) ? pr::kW4
-                                                                              : pr::kW2;
     a.xb = reinterpret_cast<const uint8_t*>(w + p.xb);
     a.part = reinterpret_cast<float*>(w + p.part);
     a.hid = reinterpret_cast<uint8_t*>(w + p.hid);
     a.qk = reinterpret_cast<uint8_t*>(w + p.qk);
     a.ppart = reinterpret_cast<float*>(w + p.ppart);
-    a.P = reinterpret_cast<float*>(w + lay.mblk);
     a.sync = sync;
     a.scores = block_scores;
     {
         std::lock_guard<std::mutex> lk(g_mu);
         a.spin_limit_ns = (uint64_t)g_spin_ns;
+        a.skip_cta = g_predict_skip_cta;
     }
     // one persistent CTA per SM (the grid barriers need every CTA resident)
-    launch(pr::predict_kernel, (unsigned)sms, pr::THREADS, pr::SMEM_BYTES, st, a);
+    launch(pr::predict_kernel, (unsigned)sms, pr::THREADS, pr::SMEM_BYTES, st, maps, a);
     return launch_status();
 }
 
@@ -979,9 +1031,11 @@ lemo_status lemo_segment_loss(const uint16_t* h, int64_t ld_h, int64_t T, int32_
     lemo_status e = launch_status();
     if (e != LEMO_OK) return e;
     namespace gm = lemo::gemm;
-    for (int64_t s0 = 0; s0 < T; s0 += seg_rows) {
+    for (int64_t s0 = 0, si = 0; s0 < T; s0 += seg_rows, ++si) {
         const int S = (int)(T - s0 < seg_rows ? T - s0 : seg_rows);
         const uint16_t* hs = h + s0 * ld_h;
+        const int hb = (int)(si & 1);                     // which dz half this segment uses
+        uint16_t* gs = g + (size_t)hb * l.rows * l.ld;
         // z [S, V] = h_seg [S, d] . W [V, d]^T  (fp32, row stride l.ld)
         if ((e = run_gemm(dev, sms, st, hs, ld_h, false, w, ld_w, false, S, V, d, gm::kStoreF32, z,
                           l.ld, true)) != LEMO_OK)
@@ -989,7 +1043,7 @@ lemo_status lemo_segment_loss(const uint16_t* h, int64_t ld_h, int64_t T, int32_
         sl::RowArgs a;
         a.z = z;
         a.ldz = l.ld;
-        a.g = g;
+        a.g = gs;
         a.ldg = l.ld;
         a.y = targets + s0;
         a.token_loss = tl + s0;
@@ -999,13 +1053,20 @@ lemo_status lemo_segment_loss(const uint16_t* h, int64_t ld_h, int64_t T, int32_
         launch(sl::row_kernel, S, sl::kRowThreads, 0, st, a);
         if ((e = launch_status()) != LEMO_OK) return e;
         // dh_seg [S, d] = dz [S, V] . W [V, d]  (W read N-contiguous: MN-major B)
-        if (dh && (e = run_gemm(dev, sms, st, g, l.ld, false, w, ld_w, true, S, d, V,
+        if (dh && (e = run_gemm(dev, sms, st, gs, l.ld, false, w, ld_w, true, S, d, V,
                                 gm::kStoreBF16, dh + s0 * ld_dh, ld_dh, true)) != LEMO_OK)
             return e;
-        // dW [V, d] += dz^T [V, S] . h_seg [S, d]  (both read MN-major)
-        if (dw && (e = run_gemm(dev, sms, st, g, l.ld, true, hs, ld_h, true, V, d, S,
-                                gm::kAddF32, dw, ld_dw, false)) != LEMO_OK)
-            return e;
+        // dW [V, d] += dz^T [V, K] . h [K, d] over the rows of this segment and
+        // the one before it (the two dz halves are consecutive rows), both read
+        // MN-major; after every second segment and after the last one
+        const bool last = s0 + seg_rows >= T;
+        if (dw && (hb == 1 || last)) {
+            const int64_t p0 = hb == 1 ? s0 - seg_rows : s0;
+            const int K = (int)(s0 + S - p0);
+            if ((e = run_gemm(dev, sms, st, g, l.ld, true, h + p0 * ld_h, ld_h, true, V, d, K,
+                              gm::kAddF32, dw, ld_dw, false)) != LEMO_OK)
+                return e;
+        }
     }
     launch(sl::loss_kernel, 1, sl::kCountThreads, 0, st, tl, T, n_valid, loss);
     return launch_status();
@@ -1021,6 +1082,11 @@ lemo_status lemo_get_error(lemo_stream stream) {
         if (cudaMemcpyToSymbol(lemo::g_error, &z, sizeof(z)) != cudaSuccess) return LEMO_ERR_CUDA;
     }
     return static_cast<lemo_status>(v);
+}
+
+void lemo_set_predict_test_hook(int32_t skip_cta) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_predict_skip_cta = skip_cta < 0 ? -1 : skip_cta;
 }
 
 void lemo_set_test_hooks(int32_t select_skip_publish_tile, int64_t spin_limit_ns) {

@@ -10,15 +10,16 @@
 //
 //   pool_kernel     streams X once (bound by HBM bandwidth) and writes the
 //                   block means as bf16 hi / lo planes already laid out as
-//                   tensor-core operand tiles;
+//                   tensor-core operand tiles; a few extra CTAs copy weights
+//                   whose rows are not 16-byte aligned into padded planes;
 //   predict_kernel  one persistent CTA per SM runs everything else as
 //                   phases separated by grid-wide barriers:
 //                     A  split-K partial products xbar W1 (both predictors)
 //                     B  sum of the split-K partials, ReLU, hi / lo split
 //                     C  the hidden activations times W2 -> Qhat, Khat tiles
-//                     D  Eq. 3 block products, positive part per head
-//                     E  sum over head groups (when there are several), then
-//                        the column sums.
+//                     D  Eq. 3 block products, positive part, per head group
+//                     E  per token block: the head groups and the rows n >= m
+//                        summed in a fixed order -> the block score.
 //
 // Every contraction runs on the tensor cores: tcgen05.mma (cta_group::1,
 // M = 128, kind::f16, bf16 operands from shared memory, fp32 accumulators in
@@ -32,21 +33,21 @@
 // in the layout a 128-byte-swizzled TMA box would have: 8-row groups of 1024
 // bytes, row r at 128 (r % 8), its 16-byte chunk j at (j ^ (r % 8)) * 16.
 // Every intermediate is written by its producer directly in that layout, so
-// a consumer fetches a whole tile with one bulk copy (cp.async.bulk, no
-// tensor map).  The weights are read with plain loads (any 2-byte alignment)
-// into MN-major swizzled tiles: 64 rows of K, 64-column groups 8 KB apart.
+// a consumer fetches a whole tile with one bulk copy (cp.async.bulk).  The
+// weights arrive through TMA as MN-major 64 x 64 boxes (64 rows of K, 64
+// columns, 128-byte swizzle), four per 256-column tile.
 //
-// Per CTA: warp 0 issues the bulk copies into a 3-stage ring of 64 KB,
-// warp 1 issues the MMAs into two 256-column accumulators, warps 2-9 load
-// the weight tiles, run the epilogues and the reductions.  Sums are taken
-// in a fixed order everywhere (split-K partials, head groups, columns):
-// results are the same bits on every run.  Every wait - mbarriers and the
-// grid barriers - is bounded in time; a wait that runs out records
-// LEMO_ERR_TIMEOUT, raises a flag that makes every CTA skip the rest, and
-// each CTA drains what it issued and frees its tensor memory before it
+// Per CTA: warp 0 issues the copies into a 3-stage ring of 64 KB, warp 1 the
+// MMAs into two 256-column accumulators, warps 2-9 run the epilogues and the
+// reductions.  Sums are taken in a fixed order everywhere (split-K partials,
+// head groups, rows): results are the same bits on every run.  Every wait -
+// mbarriers and the grid barriers - is bounded in time; a wait that runs out
+// records LEMO_ERR_TIMEOUT, raises a flag that makes every CTA skip the rest,
+// and each CTA drains what it issued and frees its tensor memory before it
 // returns.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -68,28 +69,32 @@ using score::tmem_wait_ld;
 constexpr int TILE = 128;                 // rows of a row tile (MMA M, TMEM lanes)
 constexpr int KCH = 64;                   // K elements of one image (one 128-byte row)
 constexpr int IMG = TILE * KCH * 2;       // 16 KB
+constexpr int WBOX = 64 * 64 * 2;         // one 64 x 64 weight box: 8 KB
 constexpr int STAGES = 3;
 constexpr int STAGE_BYTES = 4 * IMG;      // A hi | A lo | B (hi) | B lo
-constexpr int LOAD_WARPS = 8;             // weight loaders + epilogue (warps 2..9)
-constexpr int THREADS = 32 * (2 + LOAD_WARPS);
+constexpr int EPI_WARPS = 8;              // epilogue / reduction warps (2..9)
+constexpr int THREADS = 32 * (2 + EPI_WARPS);
 constexpr int ACC_COLS = 256;
 constexpr int TMEM_COLS = 2 * ACC_COLS;
 constexpr int MAX_NT = 256;               // widest MMA N
 constexpr int kPoolThreads = 128;
 constexpr int kPoolCols = kPoolThreads * 8;  // columns of X per pooling CTA
+constexpr int kPadCtas = 148;                // CTAs of the weight-padding part
 
 // Grid-barrier words (in the workspace; zeroed by the pooling pass).
-constexpr int kSyncA = 0, kSyncB = 1, kSyncC = 2, kSyncD = 3, kSyncE = 4, kSyncAbort = 7;
+constexpr int kSyncA = 0, kSyncB = 1, kSyncC = 2, kSyncD = 3, kSyncAbort = 7;
 constexpr int kSyncWords = 8;
 
 struct Smem {
-    uint64_t full[STAGES];      // bulk bytes landed + every loader warp stored its part
+    uint64_t full[STAGES];      // the stage's copies landed
     uint64_t empty[STAGES];     // the MMAs reading the stage completed
     uint64_t acc_full[2];       // accumulator holds a finished product
     uint64_t acc_empty[2];      // the epilogue warps read the accumulator
     uint64_t done;              // every MMA of this CTA completed
     uint32_t tmem_base;
     int abort_flag;
+    float red[EPI_WARPS + 2];   // per-warp partial sums of phase E (first column)
+    float red2[EPI_WARPS + 2];  // (second column)
 };
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align slack*/ + (int)sizeof(Smem);
 static_assert(SMEM_BYTES <= 232448, "exceeds the 227 KB of shared memory per CTA");
@@ -98,12 +103,6 @@ static_assert(SMEM_BYTES <= 232448, "exceeds the 227 KB of shared memory per CTA
 __host__ __device__ __forceinline__ uint32_t img_off(int r, int e) {
     return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((((e >> 3) ^ (r & 7)) & 7) << 4) +
                       ((e & 7) << 1));
-}
-
-// Byte offset of the 16-byte chunk (row k, columns 8 j8 .. 8 j8 + 7 of 64-column
-// group grp) of an MN-major weight tile (64 rows of K, groups 8 KB apart).
-__device__ __forceinline__ uint32_t mn_off(int k, int grp, int j8) {
-    return (uint32_t)(grp * 8192 + (k >> 3) * 1024 + (k & 7) * 128 + (((j8 ^ (k & 7)) & 7) << 4));
 }
 
 __device__ __forceinline__ void split2(float v, uint16_t& hi, uint16_t& lo) {
@@ -124,14 +123,46 @@ __device__ __forceinline__ void split8(const float* v, uint4& a, uint4& b) {
     a.w = h[6] | ((uint32_t)h[7] << 16);  b.w = l[6] | ((uint32_t)l[7] << 16);
 }
 
+// 8 consecutive bf16 starting at src; elements at or past `valid` are zero.
+// vec4: src is 4-byte aligned (4-byte loads for whole pairs), else 2-byte loads.
+__device__ __forceinline__ uint4 load8_any(const uint16_t* src, int valid, bool vec4) {
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    if (vec4) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            if (2 * i + 1 < valid)
+                w[i] = __ldg(reinterpret_cast<const uint32_t*>(src) + i);
+            else if (2 * i < valid)
+                w[i] = __ldg(src + 2 * i);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (i < valid) w[i >> 1] |= (uint32_t)__ldg(src + i) << ((i & 1) * 16);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
 // ---------------------------------------------------------------------------
 // Pooling pass.  CTA (row g, column chunk y): block means of token block g
 // over columns [y*1024, +1024), each thread 8 consecutive columns (16-byte
 // loads, eight rows in flight, added in row order).  The means are written
 // as hi / lo images [row tile][64-column chunk][plane]; rows g >= TB and
 // columns >= d of the last tile / chunk are written as zeros.  CTA (0, 0)
-// also clears the grid-barrier words of predict_kernel.
+// also clears the grid-barrier words of predict_kernel.  The first `npad`
+// CTAs of column chunk 0 (scheduled first, beside the pooling CTAs) copy the
+// weights that TMA cannot read in place (rows not 16-byte aligned, or a head
+// dimension that is not a multiple of 64) into padded planes.
 // ---------------------------------------------------------------------------
+struct PadArgs {
+    const uint16_t* w1[2];   // [d, rank] sources
+    uint16_t* w1p[2];        // [d, ldw1] planes (null: not padded)
+    const uint16_t* w2[2];   // [rank, H dh] sources
+    uint16_t* w2p[2];        // [rank, H dhp] planes, head h at columns h dhp (null: not padded)
+    int d, rank, ldw1, H, dh, dhp;
+    int w1_vec4, w2_vec4;    // the source rows allow 4-byte loads
+};
+
 __device__ __forceinline__ void add_row(float* acc, const uint4 v) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -141,15 +172,45 @@ __device__ __forceinline__ void add_row(float* acc, const uint4 v) {
     }
 }
 
+__device__ __noinline__ void pad_weights(const PadArgs& pa, int cta, int nctas) {
+    const int64_t stride = (int64_t)nctas * kPoolThreads;
+    const int64_t t0 = (int64_t)cta * kPoolThreads + threadIdx.x;
+    const int64_t c1 = (int64_t)pa.d * (pa.ldw1 / 8);          // chunks of one W1 plane
+    const int64_t c2 = (int64_t)pa.rank * (pa.H * pa.dhp / 8);  // chunks of one W2 plane
+    for (int p = 0; p < 2; ++p) {
+        if (pa.w1p[p])
+            for (int64_t i = t0; i < c1; i += stride) {
+                const int64_t r = i / (pa.ldw1 / 8);
+                const int c = (int)(i % (pa.ldw1 / 8)) * 8;
+                *reinterpret_cast<uint4*>(pa.w1p[p] + r * pa.ldw1 + c) =
+                    load8_any(pa.w1[p] + r * pa.rank + c, pa.rank - c, pa.w1_vec4 != 0);
+            }
+        if (pa.w2p[p])
+            for (int64_t i = t0; i < c2; i += stride) {
+                const int64_t k = i / (pa.H * pa.dhp / 8);
+                const int n = (int)(i % (pa.H * pa.dhp / 8)) * 8;
+                const int h = n / pa.dhp, e = n - h * pa.dhp;
+                *reinterpret_cast<uint4*>(pa.w2p[p] + k * pa.H * pa.dhp + n) = load8_any(
+                    pa.w2[p] + k * (int64_t)pa.H * pa.dh + (int64_t)h * pa.dh + e, pa.dh - e,
+                    pa.w2_vec4 != 0);
+            }
+    }
+}
+
 __global__ void __launch_bounds__(kPoolThreads)
-    pool_kernel(const uint16_t* __restrict__ x, int64_t ld_x, int d, int kc, const int32_t* __restrict__ cu,
-                int batch, int block, const char* __restrict__ ws, WsLayout lay,
-                uint8_t* __restrict__ xb, uint32_t* __restrict__ sync) {
+    pool_kernel(const uint16_t* __restrict__ x, int64_t ld_x, int d, int kc, int npad,
+                const int32_t* __restrict__ cu, int batch, int block, const char* __restrict__ ws,
+                WsLayout lay, uint8_t* __restrict__ xb, uint32_t* __restrict__ sync,
+                const PadArgs pa) {
     pdl_entry();
     if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x < kSyncWords) sync[threadIdx.x] = 0u;
+    if ((int)blockIdx.x < npad) {
+        if (blockIdx.y == 0) pad_weights(pa, blockIdx.x, npad);
+        return;
+    }
     const PlanHeader* hdr = reinterpret_cast<const PlanHeader*>(ws + lay.hdr);
     if (!hdr->valid) return;
-    const int g = blockIdx.x;
+    const int g = blockIdx.x - npad;
     const int c0 = blockIdx.y * kPoolCols + threadIdx.x * 8;
     if (c0 >= kc * KCH) return;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -185,7 +246,10 @@ __global__ void __launch_bounds__(kPoolThreads)
 // ---------------------------------------------------------------------------
 // predict_kernel
 // ---------------------------------------------------------------------------
-enum WeightLoad : int { kW16 = 0, kW4 = 1, kW2 = 2 };  // 16-, 4- or 2-byte loads
+struct Maps {
+    CUtensorMap w1[2];   // [d rows, >= rank columns] bf16, boxes of 64 x 64
+    CUtensorMap w2[2];   // [rank rows, H dhp (padded) or H dh columns], boxes of 64 x 64
+};
 
 struct Args {
     const char* ws;
@@ -203,20 +267,16 @@ struct Args {
     int np, nj2;                   // H * dhp and its 256-column tiles
     int pt, groups, hpg;           // block-product tiles, head groups, heads per group
     float inv_h;
-    // inputs
-    const uint16_t* w1[2];
-    const uint16_t* w2[2];
-    int w1_mode, w2_mode;
     // workspace
     const uint8_t* xb;    // [rt][kc][2] images
     float* part;          // [2][zk][tba][ldr]
     uint8_t* hid;         // [2][rt][kc2][2] images
     uint8_t* qk;          // [2][rt][H][dc][2] images
-    float* ppart;         // [groups][tba][tba] (groups > 1)
-    float* P;             // per-sequence block-product matrices
+    float* ppart;         // [groups][tba m][tba n] positive parts per head group
     uint32_t* sync;
     float* scores;
     uint64_t spin_limit_ns;
+    int skip_cta;         // test hook: this CTA does not arrive at the first grid barrier (-1: off)
 };
 
 __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo) {
@@ -260,15 +320,16 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
         : "memory");
 }
 
-// `count` arrivals on a CTA-local mbarrier.
-__device__ __forceinline__ void mbar_arrive_cnt(uint64_t* bar, uint32_t count) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
-                 : "memory");
+// One 64 x 64 box of a weight tensor map at (column x, row y) into shared memory.
+__device__ __forceinline__ void tma_box(uint32_t dst, const CUtensorMap* tm, int x, int y,
+                                        uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
 }
 
-__device__ __forceinline__ void fence_proxy_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
 __device__ __forceinline__ void fence_proxy_global() {
     asm volatile("fence.proxy.async.global;" ::: "memory");
 }
@@ -335,7 +396,8 @@ __device__ __noinline__ bool grid_sync(const Args& a, Smem* sm, int word) {
         uint32_t* ctr = a.sync + word;
         const volatile uint32_t* abort_word = a.sync + kSyncAbort;
         fence_proxy_global();  // this CTA's stores -> later bulk copies of other CTAs
-        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
+        if (!(word == kSyncA && (int)blockIdx.x == a.skip_cta))
+            asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
         const uint64_t t0 = globaltimer_ns();
         for (uint32_t n = 1;; ++n) {
             uint32_t v;
@@ -417,112 +479,26 @@ __device__ __forceinline__ uint8_t* qk_img(const Args& a, int p, int R, int h, i
     return a.qk + ((size_t)(((p * a.rt + R) * a.H + h) * a.dc + c) * 2 + plane) * IMG;
 }
 
-// 8 consecutive bf16 of a weight row into a 16-byte chunk; elements whose
-// column is at or past `valid` are zero.  MODE picks the load width.
-template <int MODE>
-__device__ __forceinline__ uint4 load8(const uint16_t* src, int valid) {
-    uint4 o = make_uint4(0u, 0u, 0u, 0u);
-    if (valid <= 0) return o;
-    if (valid >= 8 && MODE == kW16) return __ldg(reinterpret_cast<const uint4*>(src));
-    uint32_t w[4] = {0u, 0u, 0u, 0u};
-    if (valid >= 8 && MODE == kW4) {
+// MMAs of one 64-deep K chunk of a GEMM unit: A hi / lo images at st, the
+// MN-major weight boxes at st + 2 IMG (64-column groups WBOX apart).
+__device__ __forceinline__ void mma_weight_chunk(uint32_t d_tmem, uint32_t st, uint32_t id,
+                                                 bool first) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) w[i] = __ldg(reinterpret_cast<const uint32_t*>(src) + i);
-    } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-            if (i < valid) w[i >> 1] |= (uint32_t)__ldg(src + i) << ((i & 1) * 16);
-    }
-    o.x = w[0]; o.y = w[1]; o.z = w[2]; o.w = w[3];
-    return o;
-}
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
-                 "r"(src_bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, uint32_t src_bytes) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src),
-                 "r"(src_bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
-// 8 consecutive bf16 of a weight row (columns at or past `valid` read as
-// zero) into the 16-byte chunk at shared address dst.  kW16 and kW4 issue
-// asynchronous copies (cp.async, zero fill past the source bytes); kW2 loads
-// and stores directly.
-template <int MODE>
-__device__ __forceinline__ void copy8(uint32_t dst, uint8_t* dst_ptr, const uint16_t* src,
-                                      const uint16_t* safe, int valid) {
-    if (MODE == kW16) {
-        const int v = valid < 0 ? 0 : (valid > 8 ? 8 : valid);
-        cp_async16(dst, v > 0 ? src : safe, (uint32_t)v * 2u);
-    } else if (MODE == kW4) {
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int e = 2 * u;
-            const uint32_t bytes = valid >= e + 2 ? 4u : (valid == e + 1 ? 2u : 0u);
-            cp_async4(dst + 4 * u, bytes ? src + e : safe, bytes);
-        }
-    } else {
-        *reinterpret_cast<uint4*>(dst_ptr) = load8<kW2>(src, valid);
+    for (int k = 0; k < 4; ++k) {
+        const uint64_t bd = sdesc(st + 2 * IMG + k * 2048, WBOX);
+        umma(d_tmem, sdesc(st + k * 32, 16), bd, id, (!first || k > 0) ? 1u : 0u);
+        umma(d_tmem, sdesc(st + IMG + k * 32, 16), bd, id, 1u);
     }
 }
 
-// W1[p] rows [64 c, +64) x columns [n0, n0 + nt) into an MN-major tile
-// (groups of 64 columns; columns past nt, rows past d, columns past rank: 0),
-// issued as asynchronous copies (the caller commits and waits).
-template <int MODE>
-__device__ __forceinline__ void issue_w1(const Args& a, uint8_t* dst, int p, int c, int n0, int nt,
-                                         int ltid) {
-    const uint16_t* w = p ? a.w1[1] : a.w1[0];
-    const uint32_t dsa = smem_u32(dst);
-    const int groups = (nt + 63) >> 6;
-    const int chunks = 64 * groups * 8;
-    for (int q = ltid; q < chunks; q += 32 * LOAD_WARPS) {
-        const int j8 = q & 7, grp = (q >> 3) % groups, k = (q >> 3) / groups;
-        const int kk = c * KCH + k, n = n0 + grp * 64 + j8 * 8;
-        int valid = min(a.rank - n, nt - (grp * 64 + j8 * 8));
-        if (kk >= a.d) valid = 0;
-        const uint32_t o = mn_off(k, grp, j8);
-        copy8<MODE>(dsa + o, dst + o, w + (size_t)kk * a.rank + n, w, valid);
-    }
-}
-
-// W2[p] rows [64 c, +64) (rank index) x padded columns [n0, n0 + nt) of
-// H * dhp (column h * dhp + e is W2 column h * dh + e for e < dh, else 0).
-template <int MODE>
-__device__ __forceinline__ void issue_w2(const Args& a, uint8_t* dst, int p, int c, int n0, int nt,
-                                         int ltid) {
-    const uint16_t* w = p ? a.w2[1] : a.w2[0];
-    const uint32_t dsa = smem_u32(dst);
-    const int groups = nt >> 6;
-    const int chunks = 64 * groups * 8;
-    const int64_t ldw = (int64_t)a.H * a.dh;
-    for (int q = ltid; q < chunks; q += 32 * LOAD_WARPS) {
-        const int j8 = q & 7, grp = (q >> 3) % groups, k = (q >> 3) / groups;
-        const int kk = c * KCH + k, n = n0 + grp * 64 + j8 * 8;
-        const int h = n / a.dhp, e = n - h * a.dhp;
-        const int valid = kk < a.rank ? a.dh - e : 0;
-        const uint32_t o = mn_off(k, grp, j8);
-        copy8<MODE>(dsa + o, dst + o, w + (size_t)kk * ldw + (int64_t)h * a.dh + e, w, valid);
-    }
-}
-
-__global__ void __launch_bounds__(THREADS, 1) predict_kernel(const Args a) {
+__global__ void __launch_bounds__(THREADS, 1)
+    predict_kernel(const __grid_constant__ Maps maps, const Args a) {
     pdl_entry();
     fence_proxy_global();  // the pooling pass's stores -> this kernel's bulk copies
     const PlanHeader* hdr = reinterpret_cast<const PlanHeader*>(a.ws + a.lay.hdr);
     if (!hdr->valid) return;  // every CTA leaves here, before any barrier
     const int TB = hdr->total_blocks;
     const int32_t* blk_prefix = reinterpret_cast<const int32_t*>(a.ws + a.lay.blk_prefix);
-    const int64_t* m_prefix = reinterpret_cast<const int64_t*>(a.ws + a.lay.m_prefix);
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* tiles = reinterpret_cast<uint8_t*>(
@@ -533,16 +509,20 @@ __global__ void __launch_bounds__(THREADS, 1) predict_kernel(const Args a) {
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&sm->full[s], 1 + LOAD_WARPS);
+            mbar_init(&sm->full[s], 1);
             mbar_init(&sm->empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm->acc_full[b], 1);
-            mbar_init(&sm->acc_empty[b], LOAD_WARPS);
+            mbar_init(&sm->acc_empty[b], EPI_WARPS);
         }
         mbar_init(&sm->done, 1);
         sm->abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        for (int i = 0; i < 2; ++i) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.w1[i])) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.w2[i])) : "memory");
+        }
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -555,12 +535,11 @@ __global__ void __launch_bounds__(THREADS, 1) predict_kernel(const Args a) {
     tc_fence_after();
     const uint32_t tmem = sm->tmem_base;
 
-    // Role state, carried across phases (every role counts the same chunks
-    // and accumulations).
+    // Role state, carried across phases (producer and MMA count the same
+    // stage uses; MMA and epilogue the same accumulations).
     uint32_t it = 0;      // stage uses
     uint32_t acc_it = 0;  // accumulations
     const uint32_t ring = smem_u32(tiles);
-    const int ltid = threadIdx.x - 64;  // loader / epilogue thread id (warps 2..9)
     const int q4 = warp & 3;            // TMEM lane quadrant of an epilogue warp
     const int hf = (warp - 2) >> 2;     // which half of the accumulator's columns
     const int erow = q4 * 32 + lane;    // row of the tile (TMEM lane) of this thread
@@ -572,12 +551,18 @@ __global__ void __launch_bounds__(THREADS, 1) predict_kernel(const Args a) {
         if (warp == 0 && lane == 0) {
             for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
                 const UnitA t = unit_a(a, u);
+                const int groups = (t.nt + 63) >> 6;
                 for (int ci = 0; ci < t.nc && ok; ++ci, ++it) {
                     const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
                     if (!(ok = wait(&sm->empty[s], ph ^ 1, sm, a.sync, lim))) break;
-                    mbar_arrive_expect_tx(&sm->full[s], 2 * IMG);
-                    bulk_load(ring + s * STAGE_BYTES, xb_img(a, t.R, t.c0 + ci, 0), IMG, &sm->full[s]);
-                    bulk_load(ring + s * STAGE_BYTES + IMG, xb_img(a, t.R, t.c0 + ci, 1), IMG, &sm->full[s]);
+                    const uint32_t st = ring + s * STAGE_BYTES;
+                    const int c = t.c0 + ci;
+                    mbar_arrive_expect_tx(&sm->full[s], 2 * IMG + groups * WBOX);
+                    bulk_load(st, xb_img(a, t.R, c, 0), IMG, &sm->full[s]);
+                    bulk_load(st + IMG, xb_img(a, t.R, c, 1), IMG, &sm->full[s]);
+                    for (int g = 0; g < groups; ++g)
+                        tma_box(st + 2 * IMG + g * WBOX, &maps.w1[t.p], t.n0 + 64 * g, c * KCH,
+                                &sm->full[s]);
                 }
             }
         } else if (warp == 1 && lane == 0) {
@@ -590,13 +575,7 @@ __global__ void __launch_bounds__(THREADS, 1) predict_kernel(const Args a) {
                     const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
                     if (!(ok = wait(&sm->full[s], ph, sm, a.sync, lim))) break;
                     tc_fence_after();
-                    const uint32_t st = ring + s * STAGE_BYTES;
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const uint64_t bd = sdesc(st + 2 * IMG + k * 2048, 8192);
-                        umma(tmem + b * ACC_COLS, sdesc(st + k * 32, 16), bd, id, (ci > 0 || k > 0) ? 1u : 0u);
-                        umma(tmem + b * ACC_COLS, sdesc(st + IMG + k * 32, 16), bd, id, 1u);
-                    }
+                    mma_weight_chunk(tmem + b * ACC_COLS, ring + s * STAGE_BYTES, id, ci == 0);
                     umma_commit(&sm->empty[s]);
                 }
                 if (!ok) break;
@@ -604,35 +583,9 @@ __global__ void __launch_bounds__(THREADS, 1) predict_kernel(const Args a) {
                 ++acc_it;
             }
         } else if (warp >= 2) {
+            // epilogue: the fp32 partial of rows [128 R, +128), columns [n0, n0 + nt)
             for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
                 const UnitA t = unit_a(a, u);
-                // the copies of chunk ci + 1 are issued before chunk ci is
-                // waited for: two chunks in flight per thread
-                uint32_t prev = 0;
-                for (int ci = 0; ci < t.nc && ok; ++ci, ++it) {
-                    const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
-                    if (!(ok = wait_warp(&sm->empty[s], ph ^ 1, sm, a.sync, lim))) break;
-                    uint8_t* dst = tiles + s * STAGE_BYTES + 2 * IMG;
-                    if (a.w1_mode == kW16) issue_w1<kW16>(a, dst, t.p, t.c0 + ci, t.n0, t.nt, ltid);
-                    else if (a.w1_mode == kW4) issue_w1<kW4>(a, dst, t.p, t.c0 + ci, t.n0, t.nt, ltid);
-                    else issue_w1<kW2>(a, dst, t.p, t.c0 + ci, t.n0, t.nt, ltid);
-                    cp_commit();
-                    if (ci > 0) {
-                        cp_wait<1>();
-                        fence_proxy_smem();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&sm->full[prev]);
-                    }
-                    prev = s;
-                }
-                cp_wait<0>();
-                if (!ok) break;
-                if (t.nc > 0) {
-                    fence_proxy_smem();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&sm->full[prev]);
-                }
-                // epilogue: the fp32 partial of rows [128 R, +128), columns [n0, n0 + nt)
                 const uint32_t b = acc_it & 1;
                 if (!(ok = wait_warp(&sm->acc_full[b], (acc_it >> 1) & 1, sm, a.sync, lim))) break;
                 tc_fence_after();
@@ -658,47 +611,61 @@ __global__ void __launch_bounds__(THREADS, 1) predict_kernel(const Args a) {
     ok = grid_sync(a, sm, kSyncA);
 
     // ================================================================ phase B
-    // hid[p][row][col] = relu(sum_z part[p][z][row][col]) (z in order), as
-    // hi / lo images; rows >= TB and columns >= rank are zero.
+    // hid[p][row][col] = relu(sum_z part[p][z][row][col]), as hi / lo images;
+    // rows >= TB and columns >= rank are zero.  Four lanes share an item of 8
+    // columns: lane j sums its quarter of z in order, then the quarters are
+    // added as (q0 + q1) + (q2 + q3) - a fixed order.
     if (ok) {
         const int chunks_per_row = a.kc2 * 8;
         const int64_t items = 2LL * a.tba * chunks_per_row;
-        for (int64_t i = blockIdx.x * (int64_t)THREADS + threadIdx.x; i < items;
-             i += (int64_t)gridDim.x * THREADS) {
+        const int zq = (a.zk + 3) / 4;
+        const int64_t span = (int64_t)gridDim.x * THREADS;
+        for (int64_t base = (int64_t)blockIdx.x * THREADS; base < items * 4; base += span) {
+            // every lane runs the loop the same number of times (the shuffles below)
+            const int64_t i4 = base + threadIdx.x;
+            const int64_t i = i4 >> 2;
+            const int quarter = (int)(i4 & 3);
             const int cj = (int)(i % chunks_per_row);
             const int row = (int)((i / chunks_per_row) % a.tba);
             const int p = (int)(i / ((int64_t)chunks_per_row * a.tba));
             const int col0 = cj * 8;
+            const bool live = i < items && row < TB && col0 < a.rank;
             float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            if (row < TB && col0 < a.rank) {
+            if (live) {
                 const float* src = a.part + ((size_t)p * a.zk * a.tba + row) * a.ldr + col0;
                 const size_t plane = (size_t)a.tba * a.ldr;
-                // z in increasing order, the loads of eight planes in flight
-                for (int z = 0; z < a.zk; z += 8) {
+                const int z0 = quarter * zq, z1 = min(a.zk, z0 + zq);
+                for (int z = z0; z < z1; z += 8) {
                     float4 t[16];
 #pragma unroll
-                    for (int uu = 0; uu < 8; ++uu) {
-                        if (z + uu < a.zk) {
+                    for (int uu = 0; uu < 8; ++uu)
+                        if (z + uu < z1) {
                             t[2 * uu] = *reinterpret_cast<const float4*>(src + (z + uu) * plane);
                             t[2 * uu + 1] = *reinterpret_cast<const float4*>(src + (z + uu) * plane + 4);
                         }
-                    }
 #pragma unroll
-                    for (int uu = 0; uu < 8; ++uu) {
-                        if (z + uu < a.zk) {
+                    for (int uu = 0; uu < 8; ++uu)
+                        if (z + uu < z1) {
                             v[0] += t[2 * uu].x; v[1] += t[2 * uu].y; v[2] += t[2 * uu].z; v[3] += t[2 * uu].w;
                             v[4] += t[2 * uu + 1].x; v[5] += t[2 * uu + 1].y; v[6] += t[2 * uu + 1].z; v[7] += t[2 * uu + 1].w;
                         }
-                    }
                 }
-#pragma unroll
-                for (int e = 0; e < 8; ++e) v[e] = (col0 + e < a.rank) ? fmaxf(v[e], 0.f) : 0.f;
             }
-            uint4 hi, lo;
-            split8(v, hi, lo);
-            uint8_t* im = hid_img(a, p, row / TILE, col0 / KCH, 0) + img_off(row % TILE, col0 % KCH);
-            *reinterpret_cast<uint4*>(im) = hi;
-            *reinterpret_cast<uint4*>(im + IMG) = lo;
+            // (q0 + q1) + (q2 + q3): the four lanes of an item are adjacent
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                v[e] += __shfl_xor_sync(0xffffffffu, v[e], 1);
+                v[e] += __shfl_xor_sync(0xffffffffu, v[e], 2);
+            }
+            if (quarter == 0 && i < items) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) v[e] = (live && col0 + e < a.rank) ? fmaxf(v[e], 0.f) : 0.f;
+                uint4 hi, lo;
+                split8(v, hi, lo);
+                uint8_t* im = hid_img(a, p, row / TILE, col0 / KCH, 0) + img_off(row % TILE, col0 % KCH);
+                *reinterpret_cast<uint4*>(im) = hi;
+                *reinterpret_cast<uint4*>(im + IMG) = lo;
+            }
         }
     }
     ok = grid_sync(a, sm, kSyncB);
@@ -711,12 +678,17 @@ __global__ void __launch_bounds__(THREADS, 1) predict_kernel(const Args a) {
         if (warp == 0 && lane == 0) {
             for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
                 const UnitC t = unit_c(a, u);
+                const int groups = t.nt >> 6;
                 for (int c = 0; c < a.kc2 && ok; ++c, ++it) {
                     const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
                     if (!(ok = wait(&sm->empty[s], ph ^ 1, sm, a.sync, lim))) break;
-                    mbar_arrive_expect_tx(&sm->full[s], 2 * IMG);
-                    bulk_load(ring + s * STAGE_BYTES, hid_img(a, t.p, t.R, c, 0), IMG, &sm->full[s]);
-                    bulk_load(ring + s * STAGE_BYTES + IMG, hid_img(a, t.p, t.R, c, 1), IMG, &sm->full[s]);
+                    const uint32_t st = ring + s * STAGE_BYTES;
+                    mbar_arrive_expect_tx(&sm->full[s], 2 * IMG + groups * WBOX);
+                    bulk_load(st, hid_img(a, t.p, t.R, c, 0), IMG, &sm->full[s]);
+                    bulk_load(st + IMG, hid_img(a, t.p, t.R, c, 1), IMG, &sm->full[s]);
+                    for (int g = 0; g < groups; ++g)
+                        tma_box(st + 2 * IMG + g * WBOX, &maps.w2[t.p], t.n0 + 64 * g, c * KCH,
+                                &sm->full[s]);
                 }
             }
         } else if (warp == 1 && lane == 0) {
@@ -729,13 +701,7 @@ __global__ void __launch_bounds__(THREADS, 1) predict_kernel(const Args a) {
                     const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
                     if (!(ok = wait(&sm->full[s], ph, sm, a.sync, lim))) break;
                     tc_fence_after();
-                    const uint32_t st = ring + s * STAGE_BYTES;
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const uint64_t bd = sdesc(st + 2 * IMG + k * 2048, 8192);
-                        umma(tmem + b * ACC_COLS, sdesc(st + k * 32, 16), bd, id, (c > 0 || k > 0) ? 1u : 0u);
-                        umma(tmem + b * ACC_COLS, sdesc(st + IMG + k * 32, 16), bd, id, 1u);
-                    }
+                    mma_weight_chunk(tmem + b * ACC_COLS, ring + s * STAGE_BYTES, id, c == 0);
                     umma_commit(&sm->empty[s]);
                 }
                 if (!ok) break;
@@ -745,41 +711,23 @@ __global__ void __launch_bounds__(THREADS, 1) predict_kernel(const Args a) {
         } else if (warp >= 2) {
             for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
                 const UnitC t = unit_c(a, u);
-                uint32_t prev = 0;
-                for (int c = 0; c < a.kc2 && ok; ++c, ++it) {
-                    const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
-                    if (!(ok = wait_warp(&sm->empty[s], ph ^ 1, sm, a.sync, lim))) break;
-                    uint8_t* dst = tiles + s * STAGE_BYTES + 2 * IMG;
-                    if (a.w2_mode == kW16) issue_w2<kW16>(a, dst, t.p, c, t.n0, t.nt, ltid);
-                    else if (a.w2_mode == kW4) issue_w2<kW4>(a, dst, t.p, c, t.n0, t.nt, ltid);
-                    else issue_w2<kW2>(a, dst, t.p, c, t.n0, t.nt, ltid);
-                    cp_commit();
-                    if (c > 0) {
-                        cp_wait<1>();
-                        fence_proxy_smem();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&sm->full[prev]);
-                    }
-                    prev = s;
-                }
-                cp_wait<0>();
-                if (!ok) break;
-                if (a.kc2 > 0) {
-                    fence_proxy_smem();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&sm->full[prev]);
-                }
                 const uint32_t b = acc_it & 1;
                 if (!(ok = wait_warp(&sm->acc_full[b], (acc_it >> 1) & 1, sm, a.sync, lim))) break;
                 tc_fence_after();
                 const int half = t.nt >> 1;
                 const uint32_t taddr = tmem + b * ACC_COLS + ((uint32_t)(q4 * 32) << 16) + hf * half;
-                for (int c = 0; c < half; c += 16) {
-                    uint32_t r[16];
-                    tmem_ld16(taddr + c, r);
+                for (int c = 0; c < half; c += 32) {
+                    uint32_t r[32];
+                    tmem_ld16(taddr + c, &r[0]);
+                    tmem_ld16(taddr + c + 16, &r[16]);
                     tmem_wait_ld();
+                    if (c + 32 >= half) {  // every read of the accumulator landed: free it
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&sm->acc_empty[b]);
+                    }
 #pragma unroll
-                    for (int i = 0; i < 16; i += 8) {
+                    for (int i = 0; i < 32; i += 8) {
                         const int n = t.n0 + hf * half + c + i;  // padded column (multiple of 8)
                         const int h = n / a.dhp, e = n - h * a.dhp;
                         float v[8];
@@ -792,9 +740,6 @@ __global__ void __launch_bounds__(THREADS, 1) predict_kernel(const Args a) {
                         *reinterpret_cast<uint4*>(im + IMG) = lo;
                     }
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sm->acc_empty[b]);
                 ++acc_it;
             }
         }
@@ -805,7 +750,7 @@ __global__ void __launch_bounds__(THREADS, 1) predict_kernel(const Args a) {
     // Block products of one lower-triangle tile (query row tile tn, key row
     // tile tm) for the heads of one group: per head 3 MMAs per K step (hi hi,
     // lo hi, hi lo), then the positive part is added into 64 running sums per
-    // thread.
+    // thread; the group's sums go to its plane of ppart.
     if (ok) {
         const int nunits = a.pt * a.groups;
         if (warp == 0 && lane == 0) {
@@ -817,10 +762,7 @@ __global__ void __launch_bounds__(THREADS, 1) predict_kernel(const Args a) {
                         if (!(ok = wait(&sm->empty[s], ph ^ 1, sm, a.sync, lim))) break;
                         const int h = t.h0 + hh;
                         const uint32_t st = ring + s * STAGE_BYTES;
-                        // the loader warps have nothing to load in this phase:
-                        // their arrivals are made here
                         mbar_arrive_expect_tx(&sm->full[s], 4 * IMG);
-                        mbar_arrive_cnt(&sm->full[s], LOAD_WARPS);
                         bulk_load(st, qk_img(a, 0, t.tn, h, c, 0), IMG, &sm->full[s]);
                         bulk_load(st + IMG, qk_img(a, 0, t.tn, h, c, 1), IMG, &sm->full[s]);
                         bulk_load(st + 2 * IMG, qk_img(a, 1, t.tm, h, c, 0), IMG, &sm->full[s]);
@@ -856,7 +798,6 @@ __global__ void __launch_bounds__(THREADS, 1) predict_kernel(const Args a) {
                 }
             }
         } else if (warp >= 2) {
-            // epilogue: the accumulations the MMA thread commits, one per head
             for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
                 const UnitD t = unit_d(a, u);
                 float tot[64];
@@ -867,99 +808,86 @@ __global__ void __launch_bounds__(THREADS, 1) predict_kernel(const Args a) {
                     if (!(ok = wait_warp(&sm->acc_full[b], (acc_it >> 1) & 1, sm, a.sync, lim))) break;
                     tc_fence_after();
                     const uint32_t taddr = tmem + b * ACC_COLS + ((uint32_t)(q4 * 32) << 16) + hf * 64;
-#pragma unroll
-                    for (int c = 0; c < 64; c += 16) {
-                        uint32_t r[16];
-                        tmem_ld16(taddr + c, r);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) tot[c + i] += fmaxf(__uint_as_float(r[i]), 0.f);
-                    }
+                    uint32_t r[64];
+                    tmem_ld16(taddr, &r[0]);
+                    tmem_ld16(taddr + 16, &r[16]);
+                    tmem_ld16(taddr + 32, &r[32]);
+                    tmem_ld16(taddr + 48, &r[48]);
+                    tmem_wait_ld();
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&sm->acc_empty[b]);
                     ++acc_it;
+#pragma unroll
+                    for (int i = 0; i < 64; ++i) tot[i] += fmaxf(__uint_as_float(r[i]), 0.f);
                 }
                 if (!ok) break;
+                // ppart[g][m][n]: the lanes of a warp hold consecutive n, so each
+                // store of the 64 columns m is one coalesced 128-byte row
                 const int n = t.tn * TILE + erow;
-                const int mb = t.tm * TILE + hf * 64;
-                if (a.groups == 1) {
-                    if (n < TB) {
-                        const int s = last_le(blk_prefix, a.batch + 1, n);
-                        const int b0 = blk_prefix[s], nb = blk_prefix[s + 1] - b0;
-                        float* row = a.P + m_prefix[s] + (int64_t)(n - b0) * nb - b0;
+                float* col = a.ppart + ((size_t)t.g * a.tba + t.tm * TILE + hf * 64) * a.tba + n;
 #pragma unroll
-                        for (int i = 0; i < 64; ++i) {
-                            const int m = mb + i;
-                            if (m >= b0 && m <= n) row[m] = tot[i] * a.inv_h;
-                        }
-                    }
-                } else {
-                    float* row = a.ppart + ((size_t)t.g * a.tba + n) * a.tba + mb;
-#pragma unroll
-                    for (int i = 0; i < 64; i += 4)
-                        *reinterpret_cast<float4*>(row + i) = make_float4(tot[i], tot[i + 1], tot[i + 2], tot[i + 3]);
-                }
+                for (int i = 0; i < 64; ++i) col[(size_t)i * a.tba] = tot[i];
             }
         }
     }
     ok = grid_sync(a, sm, kSyncD);
 
     // ================================================================ phase E
-    // P[n][m] = inv_h * sum_g ppart[g][n][m] (g in order) for the pairs of one
-    // sequence with n >= m, when the heads were split into groups ...
-    if (a.groups > 1) {
-      if (ok) {
-        const int64_t total = (int64_t)TB * TB;
-        const size_t plane = (size_t)a.tba * a.tba;
-        for (int64_t i = blockIdx.x * (int64_t)THREADS + threadIdx.x; i < total;
-             i += (int64_t)gridDim.x * THREADS) {
-            const int n = (int)(i / TB), m = (int)(i % TB);
-            if (m > n) continue;
-            const int s = last_le(blk_prefix, a.batch + 1, n);
-            const int b0 = blk_prefix[s];
-            if (m < b0) continue;
-            const float* src = a.ppart + (size_t)n * a.tba + m;
-            float v = 0.f;
-            // g in increasing order, sixteen loads in flight
-            for (int g = 0; g < a.groups; g += 16) {
-                float t[16];
-#pragma unroll
-                for (int uu = 0; uu < 16; ++uu)
-                    if (g + uu < a.groups) t[uu] = src[(g + uu) * plane];
-#pragma unroll
-                for (int uu = 0; uu < 16; ++uu)
-                    if (g + uu < a.groups) v += t[uu];
-            }
-            const int nb = blk_prefix[s + 1] - b0;
-            a.P[m_prefix[s] + (int64_t)(n - b0) * nb + (m - b0)] = v * a.inv_h;
-        }
-      }
-      ok = grid_sync(a, sm, kSyncE);
-    }
-    // ... then score[g] = sum_{n = m}^{N_b - 1} P[n][m] for the token block
-    // g = (seq, m): one warp per block, lane l adds rows m + l, m + l + 32, ...
-    // in increasing order, then a fixed butterfly.
+    // score[m] = sum_{n = m}^{end of m's sequence} P[n][m] with
+    // P[n][m] = (1/H) sum_g ppart[g][m][n].  One CTA per pair of block
+    // columns m1 = cp and m2 = TB-1-cp (so every CTA adds about TB + 1
+    // values): the rows of m1 then those of m2 are dealt to the threads in
+    // order, each thread adds the head groups of its rows in order into its
+    // share of either column, and the shares are combined by a fixed butterfly
+    // per warp and the ten warp sums in warp order.
     if (ok) {
-        const int nwarps = gridDim.x * (THREADS / 32);
-        for (int g = blockIdx.x * (THREADS / 32) + warp; g < TB; g += nwarps) {
-            const int s = last_le(blk_prefix, a.batch + 1, g);
-            const int m = g - blk_prefix[s];
-            const int nb = blk_prefix[s + 1] - blk_prefix[s];
-            const float* col = a.P + m_prefix[s] + m;
-            float sum = 0.f;
-            int n = m + lane;
-            for (; n + 96 < nb; n += 128) {
-                float t[4];
+        const size_t plane = (size_t)a.tba * a.tba;
+        const int ncols2 = (TB + 1) / 2;
+        for (int cp = blockIdx.x; cp < ncols2; cp += gridDim.x) {
+            const int m1 = cp, m2 = TB - 1 - cp;
+            const int e1 = blk_prefix[last_le(blk_prefix, a.batch + 1, m1) + 1];
+            const int e2 = blk_prefix[last_le(blk_prefix, a.batch + 1, m2) + 1];
+            const int c1 = e1 - m1, c2 = m2 != m1 ? e2 - m2 : 0;
+            float s1 = 0.f, s2 = 0.f;
+            for (int idx = threadIdx.x; idx < c1 + c2; idx += THREADS) {
+                const bool first = idx < c1;
+                const int m = first ? m1 : m2;
+                const int n = first ? m1 + idx : m2 + idx - c1;
+                const float* src = a.ppart + (size_t)m * a.tba + n;
+                float v = 0.f;
+                for (int g = 0; g < a.groups; g += 32) {
+                    float t[32];
 #pragma unroll
-                for (int uu = 0; uu < 4; ++uu) t[uu] = col[(int64_t)(n + 32 * uu) * nb];
+                    for (int uu = 0; uu < 32; ++uu)
+                        if (g + uu < a.groups) t[uu] = src[(g + uu) * plane];
 #pragma unroll
-                for (int uu = 0; uu < 4; ++uu) sum += t[uu];
+                    for (int uu = 0; uu < 32; ++uu)
+                        if (g + uu < a.groups) v += t[uu];
+                }
+                if (first) s1 += v * a.inv_h;
+                else s2 += v * a.inv_h;
             }
-            for (; n < nb; n += 32) sum += col[(int64_t)n * nb];
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-            if (lane == 0) a.scores[g] = sum;
+            for (int o = 16; o > 0; o >>= 1) {
+                s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+                s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+            }
+            if (lane == 0) {
+                sm->red[warp] = s1;
+                sm->red2[warp] = s2;
+            }
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                float t1 = 0.f, t2 = 0.f;
+                for (int w = 0; w < THREADS / 32; ++w) {
+                    t1 += sm->red[w];
+                    t2 += sm->red2[w];
+                }
+                a.scores[m1] = t1;
+                if (m2 != m1) a.scores[m2] = t2;
+            }
+            __syncthreads();
         }
     }
 

@@ -74,6 +74,7 @@ _SIGS = {
                                          _P, _P, _I64, _P, _I64, _P, ctypes.c_size_t, _P]),
     "lemo_get_error": (ctypes.c_int, [_P]),
     "lemo_set_test_hooks": (None, [_I32, _I64]),
+    "lemo_set_predict_test_hook": (None, [_I32]),
 }
 
 _lib = None
@@ -259,3 +260,7 @@ def lemo_get_error(stream=None) -> int:
 
 def lemo_set_test_hooks(select_skip_publish_tile: int = -1, spin_limit_ns: int = 0):
     load().lemo_set_test_hooks(int(select_skip_publish_tile), int(spin_limit_ns))
+
+
+def lemo_set_predict_test_hook(skip_cta: int = -1):
+    load().lemo_set_predict_test_hook(int(skip_cta))

@@ -425,10 +425,13 @@ LEMO_API lemo_status lemo_attention_kept(const lemo_shape* shape, const uint16_t
 /*
  * Workspace bytes of lemo_segment_loss for T tokens, vocabulary V and
  * segments of seg_rows tokens: the valid-token count, the per-token loss
- * terms and ONE segment's fp32 logits plus their bf16 gradient
- * (2 x min(seg_rows, T) x round_up(V, 8) elements).  That last part is the
- * activation peak that segmenting divides by T / seg_rows.  Returns 0 for
- * invalid arguments.  HOST-only computation.
+ * terms, ONE segment's fp32 logits and the bf16 logit gradients of TWO
+ * segments (one when T <= seg_rows): (4 + 2 x 2) x min(seg_rows, T) x
+ * round_up(V, 8) bytes.  That last part is the activation peak that
+ * segmenting divides by about T / seg_rows (it is 6 x T x round_up(V, 8)
+ * bytes unsegmented); the second gradient segment lets dW be accumulated
+ * once per pair of segments.  Returns 0 for invalid arguments.  HOST-only
+ * computation.
  */
 LEMO_API size_t lemo_segment_loss_workspace_size(int64_t T, int32_t V, int32_t seg_rows);
 
@@ -470,7 +473,8 @@ LEMO_API size_t lemo_segment_loss_workspace_size(int64_t T, int32_t V, int32_t s
  * The three GEMMs of a segment run on this library's tensor-core kernel
  * (tcgen05 on CTA pairs, bf16 inputs, fp32 accumulation in tensor memory;
  * the logits are stored in fp32, dh rounded once to bf16, dW accumulated in
- * fp32 segment after segment); the softmax / loss / gradient of each logit
+ * fp32 once per pair of segments, in segment order); the softmax / loss /
+ * gradient of each logit
  * row is a separate row kernel.  The loss is the fixed-order sum of the
  * per-token terms (deterministic); dz is rounded to bf16.
  */
@@ -497,6 +501,14 @@ LEMO_API lemo_status lemo_get_error(lemo_stream stream);
  * (0 restores the default of 2 s).
  */
 LEMO_API void lemo_set_test_hooks(int32_t select_skip_publish_tile, int64_t spin_limit_ns);
+
+/*
+ * Test hook of lemo_predict_scores (process-wide, not thread-safe): CTA
+ * `skip_cta` >= 0 of the persistent predictor kernel does not arrive at the
+ * grid barrier after its first phase, so every CTA's bounded wait there runs
+ * out and the call reports LEMO_ERR_TIMEOUT; -1 disables it.
+ */
+LEMO_API void lemo_set_predict_test_hook(int32_t skip_cta);
 
 #ifdef __cplusplus
 }

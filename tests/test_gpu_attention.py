@@ -197,7 +197,8 @@ def test_non_block_kept_set_is_reported():
 
 def test_llama7b_16k_layer_sampled_rows():
     """Llama-2-7B layer shape (L = 16384, H = 32, dh = 128, b = 64) with the
-    llama7b-16k layer-1 keep mask (50 %): sampled kept rows against the oracle."""
+    llama7b-16k layer-1 keep mask (50 %): sampled kept rows (at least one per
+    128-row query tile) against the oracle."""
     import json
     import os
     L, H, dh, b = 16384, 32, 128, 64
@@ -209,6 +210,13 @@ def test_llama7b_16k_layer_sampled_rows():
     cu, idx, cu_kept, K = kept_from_mask([L], b, mask)
     st, got, _ = run_attention([L], H, dh, b, q, k, v, idx, cu_kept, K)
     assert st == lemo.LEMO_OK
-    rows = [0, 63, 64, 127, 128, 4095, K // 2, K - 129, K - 1]
+    # one row in every 128-row query tile (at a seeded offset, so both query
+    # tiles of a CTA and every key-tile boundary position are reached) plus
+    # the tile edges and the last rows
+    rng = np.random.default_rng(5)
+    rows = sorted(set([0, 63, 64, 127, 128, 4095, K // 2, K - 129, K - 1] +
+                      [t * 128 + int(rng.integers(0, 128)) for t in range(K // 128)]))
+    rows = [r for r in rows if r < K]
+    assert len(rows) >= 64
     want = oracle.attention_kept_rows(q, k, v, idx, cu_kept, H, dh, rows)
     check_compact(got[rows], want, v, H, dh)

@@ -178,3 +178,34 @@ def test_predictor_llama13b_32k_against_stored_oracle():
     exact = np.array([float(v) for v in g["scores"]])
     rec = oracle.recall(mask_gpu, oracle.keep_mask(exact, float(g["theta"])))
     assert rec == pytest.approx(g["recall"], abs=2.0 / len(exact))
+
+
+def test_grid_barrier_times_out_and_recovers():
+    """One CTA of the persistent kernel withholds its arrival at the first
+    grid barrier (test hook): every CTA's bounded wait runs out, the call
+    reports LEMO_ERR_TIMEOUT and every CTA leaves (nothing hangs).  The next
+    call, without the hook, gives the oracle's scores."""
+    lengths, H, dh, b, d, rank = [1000, 300], 2, 64, 64, 128, 48
+    x = synth.normal_bf16(sum(lengths), d, 13, 7)
+    w1q, w2q, _ = synth.predictor_weights(d, rank, H * dh, 0.4, 13, 10)
+    w1k, w2k, _ = synth.predictor_weights(d, rank, H * dh, 0.4, 13, 11)
+    import torch
+    cu = np.zeros(len(lengths) + 1, dtype=np.int32)
+    cu[1:] = np.cumsum(lengths)
+    cu_d = torch.from_numpy(cu).cuda()
+    shape = lemo.make_shape(cu_d, int(cu[-1]), max(lengths), H, dh, b)
+    ws = torch.empty(lemo.lemo_predict_workspace_size(shape, d, rank), dtype=torch.uint8,
+                     device="cuda")
+    out = torch.zeros(32, dtype=torch.float32, device="cuda")
+    try:
+        lemo.lemo_set_test_hooks(-1, 50_000_000)
+        lemo.lemo_set_predict_test_hook(0)
+        lemo.lemo_predict_scores(shape, _dev(x), _dev(w1q), _dev(w2q), _dev(w1k), _dev(w2k),
+                                 out, ws)
+        assert lemo.lemo_get_error() == lemo.LEMO_ERR_TIMEOUT
+    finally:
+        lemo.lemo_set_predict_test_hook(-1)
+        lemo.lemo_set_test_hooks(-1, 0)
+    got, _ = run_predict(lengths, H, dh, b, x, w1q, w2q, w1k, w2k)
+    assert_scores_close(got, oracle_predict(lengths, H, dh, b, x, w1q, w2q, w1k, w2k),
+                        "predicted scores after a timed-out call")
