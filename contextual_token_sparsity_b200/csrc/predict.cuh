@@ -91,6 +91,7 @@ struct Smem {
     uint64_t acc_full[2];       // accumulator holds a finished product
     uint64_t acc_empty[2];      // the epilogue warps read the accumulator
     uint64_t done;              // every MMA of this CTA completed
+    uint64_t epi_bar;           // the epilogue warps finished a staged unit of phase C
     uint32_t tmem_base;
     int abort_flag;
     float red[EPI_WARPS + 2];   // per-warp partial sums of phase E (first column)
@@ -172,6 +173,41 @@ __device__ __forceinline__ void add_row(float* acc, const uint4 v) {
     }
 }
 
+// 8 bf16 of the contiguous matrix `src` starting at element e (any 2-byte
+// alignment of src + e), elements at or past `valid` zero: one or two aligned
+// 16-byte loads and a byte funnel shift.  Consecutive threads taking
+// consecutive chunks read consecutive 16-byte words (coalesced).  The second
+// load is made only when valid elements lie in it, so nothing past the last
+// element of the matrix is read.
+__device__ __forceinline__ uint4 load8_shifted(const uint16_t* src, int64_t e, int valid) {
+    if (valid <= 0) return make_uint4(0u, 0u, 0u, 0u);
+    const uintptr_t b = reinterpret_cast<uintptr_t>(src + e);
+    const uint32_t sh = (uint32_t)(b & 15u);  // even
+    const uint4* a0 = reinterpret_cast<const uint4*>(b - sh);
+    const int nbytes = (valid < 8 ? valid : 8) * 2;
+    const uint4 v0 = __ldg(a0);
+    const uint4 v1 = (int)sh + nbytes > 16 ? __ldg(a0 + 1) : make_uint4(0u, 0u, 0u, 0u);
+    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    const uint32_t q = sh >> 2, bits = (sh & 3u) * 8u;
+    uint32_t o[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        // words q + k and q + k + 1 (q <= 3), selected without local memory
+        uint32_t lo = w[k], hi = w[k + 1];
+        if (q == 1) { lo = w[k + 1]; hi = w[k + 2]; }
+        if (q == 2) { lo = w[k + 2]; hi = w[k + 3]; }
+        if (q == 3) { lo = w[k + 3]; hi = w[k + 4]; }
+        o[k] = __funnelshift_r(lo, hi, bits);
+    }
+    // zero the elements at or past `valid`
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        if (2 * k >= valid) o[k] = 0u;
+        else if (2 * k + 1 >= valid) o[k] &= 0xffffu;
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 __device__ __noinline__ void pad_weights(const PadArgs& pa, int cta, int nctas) {
     const int64_t stride = (int64_t)nctas * kPoolThreads;
     const int64_t t0 = (int64_t)cta * kPoolThreads + threadIdx.x;
@@ -183,7 +219,7 @@ __device__ __noinline__ void pad_weights(const PadArgs& pa, int cta, int nctas) 
                 const int64_t r = i / (pa.ldw1 / 8);
                 const int c = (int)(i % (pa.ldw1 / 8)) * 8;
                 *reinterpret_cast<uint4*>(pa.w1p[p] + r * pa.ldw1 + c) =
-                    load8_any(pa.w1[p] + r * pa.rank + c, pa.rank - c, pa.w1_vec4 != 0);
+                    load8_shifted(pa.w1[p], r * pa.rank + c, pa.rank - c);
             }
         if (pa.w2p[p])
             for (int64_t i = t0; i < c2; i += stride) {
@@ -330,6 +366,17 @@ __device__ __forceinline__ void tma_box(uint32_t dst, const CUtensorMap* tm, int
         : "memory");
 }
 
+// shared -> global bulk copy (bytes a multiple of 16, both addresses 16-byte aligned)
+__device__ __forceinline__ void bulk_store(void* dst, uint32_t src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
 __device__ __forceinline__ void fence_proxy_global() {
     asm volatile("fence.proxy.async.global;" ::: "memory");
 }
@@ -517,6 +564,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_init(&sm->acc_empty[b], EPI_WARPS);
         }
         mbar_init(&sm->done, 1);
+        mbar_init(&sm->epi_bar, EPI_WARPS);
         sm->abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         for (int i = 0; i < 2; ++i) {
@@ -583,7 +631,11 @@ __global__ void __launch_bounds__(THREADS, 1)
                 ++acc_it;
             }
         } else if (warp >= 2) {
-            // epilogue: the fp32 partial of rows [128 R, +128), columns [n0, n0 + nt)
+            // epilogue: the fp32 partial of rows [128 R, +128), columns [n0, n0 + nt).
+            // For the CTA's last unit of the phase the ring is idle (every load of
+            // the phase was consumed by the MMAs that completed before acc_full),
+            // so each thread stages its half row there and sends it with one bulk
+            // copy; otherwise it stores directly.
             for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
                 const UnitA t = unit_a(a, u);
                 const uint32_t b = acc_it & 1;
@@ -593,19 +645,33 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const uint32_t taddr = tmem + b * ACC_COLS + ((uint32_t)(q4 * 32) << 16) + hf * half;
                 float* dst = a.part + ((size_t)(t.p * a.zk + t.z) * a.tba + t.R * TILE + erow) * a.ldr +
                              t.n0 + hf * half;
+                const bool staged = u + (int)gridDim.x >= nunits;
+                // row pitch nt * 4 + 16 bytes: 16-byte stores of 32 rows hit distinct banks
+                uint8_t* srow = tiles + (size_t)erow * (t.nt * 4 + 16) + hf * half * 4;
                 for (int c = 0; c < half; c += 16) {
                     uint32_t r[16];
                     tmem_ld16(taddr + c, r);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 16; i += 4)
-                        *reinterpret_cast<uint4*>(dst + c + i) = make_uint4(r[i], r[i + 1], r[i + 2], r[i + 3]);
+                    for (int i = 0; i < 16; i += 4) {
+                        const uint4 v = make_uint4(r[i], r[i + 1], r[i + 2], r[i + 3]);
+                        if (staged)
+                            *reinterpret_cast<uint4*>(srow + (c + i) * 4) = v;
+                        else
+                            *reinterpret_cast<uint4*>(dst + c + i) = v;
+                    }
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm->acc_empty[b]);
                 ++acc_it;
+                if (staged) {
+                    fence_proxy_smem();
+                    bulk_store(dst, smem_u32(srow), (uint32_t)half * 4u);
+                    bulk_commit();
+                }
             }
+            bulk_wait_all();  // every staged copy landed (and read the ring) before the barrier
         }
     }
     ok = grid_sync(a, sm, kSyncA);
@@ -709,11 +775,15 @@ __global__ void __launch_bounds__(THREADS, 1)
                 ++acc_it;
             }
         } else if (warp >= 2) {
+            // For the CTA's last unit of the phase the output images are built in
+            // the idle ring (8 images of 16 KB at most) and sent with one bulk
+            // copy each; otherwise each thread stores its 16-byte chunks directly.
             for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
                 const UnitC t = unit_c(a, u);
                 const uint32_t b = acc_it & 1;
                 if (!(ok = wait_warp(&sm->acc_full[b], (acc_it >> 1) & 1, sm, a.sync, lim))) break;
                 tc_fence_after();
+                const bool staged = u + (int)gridDim.x >= nunits;
                 const int half = t.nt >> 1;
                 const uint32_t taddr = tmem + b * ACC_COLS + ((uint32_t)(q4 * 32) << 16) + hf * half;
                 for (int c = 0; c < half; c += 32) {
@@ -735,13 +805,33 @@ __global__ void __launch_bounds__(THREADS, 1)
                         for (int e8 = 0; e8 < 8; ++e8) v[e8] = __uint_as_float(r[i + e8]);
                         uint4 hi, lo;
                         split8(v, hi, lo);
-                        uint8_t* im = qk_img(a, t.p, t.R, h, e / KCH, 0) + img_off(erow, e % KCH);
+                        uint8_t* im = staged ? tiles + (size_t)((n - t.n0) / KCH) * 2 * IMG
+                                             : qk_img(a, t.p, t.R, h, e / KCH, 0);
+                        im += img_off(erow, e % KCH);
                         *reinterpret_cast<uint4*>(im) = hi;
                         *reinterpret_cast<uint4*>(im + IMG) = lo;
                     }
                 }
                 ++acc_it;
+                if (staged) {
+                    // every warp's part of the images is written: then one thread
+                    // sends them (a bounded wait, so a warp that gave up cannot
+                    // hold the others)
+                    fence_proxy_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sm->epi_bar);
+                    if (threadIdx.x == 64 && wait(&sm->epi_bar, 0, sm, a.sync, lim)) {
+                        for (int j = 0; j < t.nt / KCH; ++j) {
+                            const int n = t.n0 + j * KCH;
+                            const int h = n / a.dhp, e = n - h * a.dhp;
+                            bulk_store(qk_img(a, t.p, t.R, h, e / KCH, 0),
+                                       smem_u32(tiles + (size_t)j * 2 * IMG), 2 * IMG);
+                        }
+                        bulk_commit();
+                    }
+                }
             }
+            bulk_wait_all();  // every staged copy landed (and read the ring) before the barrier
         }
     }
     ok = grid_sync(a, sm, kSyncC);
