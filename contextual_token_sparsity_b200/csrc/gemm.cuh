@@ -97,6 +97,9 @@ struct Args {
     int M, N, K;
     int a_mn, b_mn;        // 1: the operand is MN-major (MN contiguous in memory)
     int epi;               // Epi (the output itself is the tensor map tm_c)
+    float2* stats;         // kStoreF32 only, optional: per row and 128-column half tile the
+                           // running (max, sum of 2^(u - max)) of u = C * log2(e), columns < N
+    int64_t ld_stats;      // float2 elements between the rows of stats (2 * tiles_n)
     int tiles_m, tiles_n;
     int m_fastest;         // 1: consecutive tiles step along M (they share a B tile)
     uint64_t spin_limit_ns;
@@ -372,6 +375,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             const int row0 = tm * TM + (int)rank * ROWS + q * 32;  // first output row of this warp
             const int col0 = tn * TN + colhalf * COLS_PER_THREAD;
             const uint32_t base = lane_addr + buf * ACC_COLS;
+            float st_m = -__int_as_float(0x7f800000), st_s = 0.f;  // this thread's row statistics
 #pragma unroll 1
             for (int ch = 0; ch < COLS_PER_THREAD; ch += chunk, ++nst) {
                 uint32_t r[64];
@@ -392,6 +396,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 #pragma unroll
                     for (int i = 0; i < 32; ++i)
                         r[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+                } else if (a.stats) {
+                    // online max / sum of 2^(u - max) over the columns < N of this chunk
+                    constexpr float kLog2e = 1.4426950408889634f;
+                    float cm = st_m;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (col0 + ch + i < a.N) cm = fmaxf(cm, __uint_as_float(r[i]) * kLog2e);
+                    if (cm > st_m) {
+                        st_s *= exp2f(st_m - cm);
+                        st_m = cm;
+                    }
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (col0 + ch + i < a.N) st_s += exp2f(__uint_as_float(r[i]) * kLog2e - st_m);
                 }
                 // the staging buffer used two boxes ago has been read by its TMA
                 const uint32_t sb = my_stg + (nst & 1) * STG_BYTES;
@@ -408,6 +426,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     bulk_commit();
                 }
             }
+            if (a.stats && !bf16_out && row0 + lane < a.M)
+                a.stats[(int64_t)(row0 + lane) * a.ld_stats + 2 * tn + colhalf] = make_float2(st_m, st_s);
         }
         if (lane == 0) bulk_wait_all();  // every store landed before the CTA exits
         __syncwarp();

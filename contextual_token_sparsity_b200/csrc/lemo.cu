@@ -316,7 +316,8 @@ lemo_status check_predict(const lemo_shape* s, int d, int rank) {
 
 // Workspace of lemo_segment_loss.
 struct SegLayout {
-    size_t n_valid, token_loss, z, g, total;
+    size_t n_valid, token_loss, z, g, stats, total;
+    int64_t nstats;   // partial (max, sum) pairs per logit row (two per 256-column tile)
     int64_t ld;    // row stride of the segment's logits and gradient
     int64_t rows;  // rows of one segment buffer
 };
@@ -332,6 +333,8 @@ SegLayout seg_layout(int64_t T, int V, int seg_rows) {
     // two segments of dz when there are several: dW is accumulated once per
     // pair of segments (K = 2 segments), which halves its read-add-write
     l.g = off; off = lemo::align_up(off + 2 * (size_t)(T > seg_rows ? 2 : 1) * l.rows * l.ld, 256);
+    l.nstats = 2 * (((int64_t)V + lemo::gemm::TN - 1) / lemo::gemm::TN);
+    l.stats = off; off = lemo::align_up(off + 8 * (size_t)l.rows * l.nstats, 256);
     l.total = off;
     return l;
 }
@@ -428,7 +431,7 @@ int gemm_pairs(int dev, int sms) {
 // a_mn / b_mn: the operand's M / N index is the contiguous one in memory.
 lemo_status run_gemm(int dev, int sms, cudaStream_t st, const uint16_t* A, int64_t lda, bool a_mn,
                      const uint16_t* B, int64_t ldb, bool b_mn, int M, int N, int K, int epi,
-                     void* out, int64_t ld_out, bool m_fastest) {
+                     void* out, int64_t ld_out, bool m_fastest, float2* stats = nullptr) {
     namespace gm = lemo::gemm;
     if (M <= 0 || N <= 0) return LEMO_OK;
     CUtensorMap ta, tb, tc;
@@ -445,6 +448,8 @@ lemo_status run_gemm(int dev, int sms, cudaStream_t st, const uint16_t* A, int64
     a.a_mn = a_mn ? 1 : 0;
     a.b_mn = b_mn ? 1 : 0;
     a.epi = epi;
+    a.stats = stats;
+    a.ld_stats = 2 * (int64_t)((N + gm::TN - 1) / gm::TN);
     a.tiles_m = (M + gm::TM - 1) / gm::TM;
     a.tiles_n = (N + gm::TN - 1) / gm::TN;
     a.m_fastest = m_fastest ? 1 : 0;
@@ -872,11 +877,12 @@ lemo_status lemo_predict_scores(const lemo_shape* shape, int32_t d, const uint16
     // block means, as hi / lo operand images (and the barrier words cleared,
     // the weight planes padded)
     const int npad = (pad_w1 || pad_w2) ? pr::kPadCtas : 0;
-    launch(pr::pool_kernel,
-           dim3((unsigned)(npad + p.tba),
-                (unsigned)((p.kc * pr::KCH + pr::kPoolCols - 1) / pr::kPoolCols)),
-           pr::kPoolThreads, 0, st, x, ld_x, d, p.kc, npad, shape->cu_seqlens, shape->batch,
-           shape->block, w, lay, reinterpret_cast<uint8_t*>(w + p.xb), sync, pa);
+    const int64_t pool_ctas =
+        (int64_t)p.tba * ((p.kc * pr::KCH + pr::kPoolCols - 1) / pr::kPoolCols);
+    if (npad + pool_ctas > INT_MAX) return LEMO_ERR_UNSUPPORTED;
+    launch(pr::pool_kernel, (unsigned)(npad + pool_ctas), pr::kPoolThreads, 0, st, x, ld_x, d, p.kc,
+           npad, p.tba, shape->cu_seqlens, shape->batch, shape->block, w, lay,
+           reinterpret_cast<uint8_t*>(w + p.xb), sync, pa);
     if ((e = launch_status()) != LEMO_OK) return e;
     pr::Args a;
     a.ws = w;
@@ -1037,12 +1043,15 @@ lemo_status lemo_segment_loss(const uint16_t* h, int64_t ld_h, int64_t T, int32_
         const int hb = (int)(si & 1);                     // which dz half this segment uses
         uint16_t* gs = g + (size_t)hb * l.rows * l.ld;
         // z [S, V] = h_seg [S, d] . W [V, d]^T  (fp32, row stride l.ld)
+        float2* stats = reinterpret_cast<float2*>(wsp + l.stats);
         if ((e = run_gemm(dev, sms, st, hs, ld_h, false, w, ld_w, false, S, V, d, gm::kStoreF32, z,
-                          l.ld, true)) != LEMO_OK)
+                          l.ld, true, stats)) != LEMO_OK)
             return e;
         sl::RowArgs a;
         a.z = z;
         a.ldz = l.ld;
+        a.stats = stats;
+        a.nstats = (int)l.nstats;
         a.g = gs;
         a.ldg = l.ld;
         a.y = targets + s0;

@@ -106,22 +106,21 @@ __host__ __device__ __forceinline__ uint32_t img_off(int r, int e) {
                       ((e & 7) << 1));
 }
 
-__device__ __forceinline__ void split2(float v, uint16_t& hi, uint16_t& lo) {
-    const __nv_bfloat16 h = __float2bfloat16_rn(v);
-    const __nv_bfloat16 l = __float2bfloat16_rn(v - __bfloat162float(h));
-    hi = *reinterpret_cast<const uint16_t*>(&h);
-    lo = *reinterpret_cast<const uint16_t*>(&l);
-}
-
-// Split 8 fp32 values into two 16-byte chunks (8 bf16 each).
+// Split 8 fp32 values into two 16-byte chunks (8 bf16 each): hi = bf16(v),
+// lo = bf16(v - hi), both rounded to nearest even, two values per conversion
+// instruction.
 __device__ __forceinline__ void split8(const float* v, uint4& a, uint4& b) {
-    uint16_t h[8], l[8];
+    uint32_t h[4], l[4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) split2(v[i], h[i], l[i]);
-    a.x = h[0] | ((uint32_t)h[1] << 16);  b.x = l[0] | ((uint32_t)l[1] << 16);
-    a.y = h[2] | ((uint32_t)h[3] << 16);  b.y = l[2] | ((uint32_t)l[3] << 16);
-    a.z = h[4] | ((uint32_t)h[5] << 16);  b.z = l[4] | ((uint32_t)l[5] << 16);
-    a.w = h[6] | ((uint32_t)h[7] << 16);  b.w = l[6] | ((uint32_t)l[7] << 16);
+    for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 hh = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+        const __nv_bfloat162 ll = __floats2bfloat162_rn(v[2 * i] - __low2float(hh),
+                                                        v[2 * i + 1] - __high2float(hh));
+        h[i] = *reinterpret_cast<const uint32_t*>(&hh);
+        l[i] = *reinterpret_cast<const uint32_t*>(&ll);
+    }
+    a = make_uint4(h[0], h[1], h[2], h[3]);
+    b = make_uint4(l[0], l[1], l[2], l[3]);
 }
 
 // 8 consecutive bf16 starting at src; elements at or past `valid` are zero.
@@ -145,13 +144,14 @@ __device__ __forceinline__ uint4 load8_any(const uint16_t* src, int valid, bool 
 }
 
 // ---------------------------------------------------------------------------
-// Pooling pass.  CTA (row g, column chunk y): block means of token block g
-// over columns [y*1024, +1024), each thread 8 consecutive columns (16-byte
+// Pooling pass.  CTA npad + y * tba + g (row g, column chunk y, so that the
+// grid is one wave of plain CTAs): block means of token block g over columns
+// [y*1024, +1024), each thread 8 consecutive columns (16-byte
 // loads, eight rows in flight, added in row order).  The means are written
 // as hi / lo images [row tile][64-column chunk][plane]; rows g >= TB and
 // columns >= d of the last tile / chunk are written as zeros.  CTA (0, 0)
 // also clears the grid-barrier words of predict_kernel.  The first `npad`
-// CTAs of column chunk 0 (scheduled first, beside the pooling CTAs) copy the
+// CTAs (scheduled first, beside the pooling CTAs) copy the
 // weights that TMA cannot read in place (rows not 16-byte aligned, or a head
 // dimension that is not a multiple of 64) into padded planes.
 // ---------------------------------------------------------------------------
@@ -234,20 +234,21 @@ __device__ __noinline__ void pad_weights(const PadArgs& pa, int cta, int nctas) 
 }
 
 __global__ void __launch_bounds__(kPoolThreads)
-    pool_kernel(const uint16_t* __restrict__ x, int64_t ld_x, int d, int kc, int npad,
+    pool_kernel(const uint16_t* __restrict__ x, int64_t ld_x, int d, int kc, int npad, int tba,
                 const int32_t* __restrict__ cu, int batch, int block, const char* __restrict__ ws,
                 WsLayout lay, uint8_t* __restrict__ xb, uint32_t* __restrict__ sync,
                 const PadArgs pa) {
     pdl_entry();
-    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x < kSyncWords) sync[threadIdx.x] = 0u;
+    if (blockIdx.x == 0 && threadIdx.x < kSyncWords) sync[threadIdx.x] = 0u;
     if ((int)blockIdx.x < npad) {
-        if (blockIdx.y == 0) pad_weights(pa, blockIdx.x, npad);
+        pad_weights(pa, blockIdx.x, npad);
         return;
     }
     const PlanHeader* hdr = reinterpret_cast<const PlanHeader*>(ws + lay.hdr);
     if (!hdr->valid) return;
-    const int g = blockIdx.x - npad;
-    const int c0 = blockIdx.y * kPoolCols + threadIdx.x * 8;
+    const int u = blockIdx.x - npad;
+    const int g = u % tba;
+    const int c0 = (u / tba) * kPoolCols + threadIdx.x * 8;
     if (c0 >= kc * KCH) return;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     if (g < hdr->total_blocks && c0 < d) {

@@ -15,10 +15,10 @@
 // the loss is the fixed-order sum of the per-token terms divided by n
 // (loss_kernel), so it does not depend on the segment size.
 //
-// row_kernel is one CTA per token row: an online (max, sum of exp) pass over
-// the fp32 logits, a block reduction, then a second pass that writes the bf16
-// gradient row.  Both passes stream the row with 16-byte loads; the segment's
-// logits were just written by the GEMM and are mostly still in L2.
+// row_kernel is one CTA per token row: the row's (max, sum of exp) - merged
+// from the partial pairs the logits GEMM's epilogue left for every 128-column
+// half tile, so the logits are read once - a block reduction, then a pass
+// that writes the bf16 gradient row (16-byte loads of the fp32 logits).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -65,6 +65,8 @@ __global__ void __launch_bounds__(kCountThreads)
 struct RowArgs {
     const float* z;        // segment logits, row r at z + r * ldz
     int64_t ldz;
+    const float2* stats;   // optional: per row, nstats partial (max, sum of 2^(u - max)) pairs
+    int nstats;            // (u = z log2(e)) from the logits GEMM, so pass 1 reads no logits
     uint16_t* g;           // bf16 gradient of the logits, row r at g + r * ldg
     int64_t ldg;
     const int32_t* y;      // targets of the segment's rows
@@ -108,9 +110,17 @@ __global__ void __launch_bounds__(kRowThreads) row_kernel(RowArgs a) {
         return;
     }
 
-    // pass 1: online max and sum of 2^(u - max)
+    // pass 1: online max and sum of 2^(u - max), from the GEMM's partial pairs
+    // of the row when it gave them, else from the logits
     float m = -CUDART_INF_F, s = 0.f;
     const float4* z4 = reinterpret_cast<const float4*>(zr);
+    if (a.stats) {
+        const float2* sr = a.stats + (int64_t)r * a.nstats;
+        for (int j = threadIdx.x; j < a.nstats; j += kRowThreads) {
+            const float2 p = sr[j];
+            lse_merge(m, s, p.x, p.y);
+        }
+    } else
     for (int j = threadIdx.x; j < nvec; j += kRowThreads) {
         const float4 v = z4[j];
         const float u0 = v.x * kLog2e, u1 = v.y * kLog2e, u2 = v.z * kLog2e, u3 = v.w * kLog2e;
@@ -121,6 +131,7 @@ __global__ void __launch_bounds__(kRowThreads) row_kernel(RowArgs a) {
         }
         s += exp2f(u0 - m) + exp2f(u1 - m) + exp2f(u2 - m) + exp2f(u3 - m);
     }
+    if (!a.stats)
     for (int v = 4 * nvec + threadIdx.x; v < V; v += kRowThreads) {
         const float u = zr[v] * kLog2e;
         if (u > m) {

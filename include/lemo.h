@@ -425,10 +425,11 @@ LEMO_API lemo_status lemo_attention_kept(const lemo_shape* shape, const uint16_t
 /*
  * Workspace bytes of lemo_segment_loss for T tokens, vocabulary V and
  * segments of seg_rows tokens: the valid-token count, the per-token loss
- * terms, ONE segment's fp32 logits and the bf16 logit gradients of TWO
- * segments (one when T <= seg_rows): (4 + 2 x 2) x min(seg_rows, T) x
- * round_up(V, 8) bytes.  That last part is the activation peak that
- * segmenting divides by about T / seg_rows (it is 6 x T x round_up(V, 8)
+ * terms, ONE segment's fp32 logits, the bf16 logit gradients of TWO
+ * segments (one when T <= seg_rows) and the rows' partial softmax
+ * statistics (8 bytes per 128 logits): about (4 + 2 x 2) x min(seg_rows, T)
+ * x round_up(V, 8) bytes.  That is the activation peak that segmenting
+ * divides by about 3/4 x T / seg_rows (it is about 6 x T x round_up(V, 8)
  * bytes unsegmented); the second gradient segment lets dW be accumulated
  * once per pair of segments.  Returns 0 for invalid arguments.  HOST-only
  * computation.
@@ -473,9 +474,11 @@ LEMO_API size_t lemo_segment_loss_workspace_size(int64_t T, int32_t V, int32_t s
  * The three GEMMs of a segment run on this library's tensor-core kernel
  * (tcgen05 on CTA pairs, bf16 inputs, fp32 accumulation in tensor memory;
  * the logits are stored in fp32, dh rounded once to bf16, dW accumulated in
- * fp32 once per pair of segments, in segment order); the softmax / loss /
- * gradient of each logit
- * row is a separate row kernel.  The loss is the fixed-order sum of the
+ * fp32 once per pair of segments, in segment order); the logits GEMM's
+ * epilogue also leaves each row's running (max, sum of exponentials) per
+ * 128 columns, from which a separate row kernel forms the softmax, the loss
+ * term and the bf16 gradient of each logit row, reading the logits once.
+ * The loss is the fixed-order sum of the
  * per-token terms (deterministic); dz is rounded to bf16.
  */
 LEMO_API lemo_status lemo_segment_loss(const uint16_t* h, int64_t ld_h, int64_t T, int32_t d,
