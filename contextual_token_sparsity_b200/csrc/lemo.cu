@@ -242,7 +242,7 @@ struct PredictLayout {
     int ldr, nj, nt; // rank padded to 32, n tiles of the first GEMM and their width
     int zk, cps;     // K splits of the first GEMM, chunks per split
     int dhp, dc;     // head dimension padded to 64, its chunks
-    int np, nj2;     // H * dhp and its 256-column tiles
+    int np, nc, nj2; // H * dhp, the second GEMM's unit width, its units per row tile
     int pt, groups, hpg;
     bool fits;       // every unit count fits in 32 bits
 };
@@ -274,7 +274,15 @@ PredictLayout predict_layout(const lemo_shape* s, int d, int rank) {
     p.dhp = (s->dh + pr::KCH - 1) / pr::KCH * pr::KCH;
     p.dc = p.dhp / pr::KCH;
     p.np = s->H * p.dhp;
-    p.nj2 = (p.np + pr::MAX_NT - 1) / pr::MAX_NT;
+    // second GEMM: units of nc columns, about one per SM of a B200
+    {
+        const int64_t cols = 2 * rt * (int64_t)p.np;
+        int64_t nc = ((cols + kTarget - 1) / kTarget + 15) / 16 * 16;
+        if (nc < 64) nc = 64;
+        if (nc > pr::MAX_NT) nc = pr::MAX_NT;
+        p.nc = (int)nc;
+    }
+    p.nj2 = (p.np + p.nc - 1) / p.nc;
     const int64_t pt = rt * (rt + 1) / 2;
     p.pt = (int)(pt < INT_MAX ? pt : INT_MAX);
     int64_t groups = (kTarget + pt - 1) / pt;
@@ -904,6 +912,7 @@ lemo_status lemo_predict_scores(const lemo_shape* shape, int32_t d, const uint16
     a.zk = p.zk;
     a.cps = p.cps;
     a.np = p.np;
+    a.nc = p.nc;
     a.nj2 = p.nj2;
     a.pt = p.pt;
     a.groups = p.groups;

@@ -16,7 +16,8 @@
 //                   phases separated by grid-wide barriers:
 //                     A  split-K partial products xbar W1 (both predictors)
 //                     B  sum of the split-K partials, ReLU, hi / lo split
-//                     C  the hidden activations times W2 -> Qhat, Khat tiles
+//                     C  the hidden activations times W2 -> Qhat, Khat tiles, in
+//                        column units sized to about one per SM
 //                     D  Eq. 3 block products, positive part, per head group
 //                     E  per token block: the head groups and the rows n >= m
 //                        summed in a fixed order -> the block score.
@@ -91,7 +92,6 @@ struct Smem {
     uint64_t acc_full[2];       // accumulator holds a finished product
     uint64_t acc_empty[2];      // the epilogue warps read the accumulator
     uint64_t done;              // every MMA of this CTA completed
-    uint64_t epi_bar;           // the epilogue warps finished a staged unit of phase C
     uint32_t tmem_base;
     int abort_flag;
     float red[EPI_WARPS + 2];   // per-warp partial sums of phase E (first column)
@@ -301,7 +301,7 @@ struct Args {
     int ldr;                       // rank padded to 32 (columns of the split-K partials)
     int nj, nt;                    // n tiles of the first GEMM and their width
     int zk, cps;                   // K splits of the first GEMM and chunks per split
-    int np, nj2;                   // H * dhp and its 256-column tiles
+    int np, nc, nj2;               // H * dhp, the second GEMM's unit width and units per row tile
     int pt, groups, hpg;           // block-product tiles, head groups, heads per group
     float inv_h;
     // workspace
@@ -380,6 +380,13 @@ __device__ __forceinline__ void fence_proxy_smem() {
 }
 __device__ __forceinline__ void fence_proxy_global() {
     asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t* r) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                   "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
 }
 
 __device__ __forceinline__ bool aborted(const Smem* sm) {
@@ -488,7 +495,7 @@ __device__ __forceinline__ UnitA unit_a(const Args& a, int u) {
     t.nt = min(a.nt, a.ldr - t.n0);
     return t;
 }
-struct UnitC {  // one 256-column tile of the second GEMM
+struct UnitC {  // nc columns (a multiple of 16, at most 256) of the second GEMM
     int p, R, j, n0, nt;
 };
 __device__ __forceinline__ UnitC unit_c(const Args& a, int u) {
@@ -497,8 +504,8 @@ __device__ __forceinline__ UnitC unit_c(const Args& a, int u) {
     const int v = u / a.nj2;
     t.R = v % a.rt;
     t.p = v / a.rt;
-    t.n0 = t.j * MAX_NT;
-    t.nt = min(MAX_NT, a.np - t.n0);
+    t.n0 = t.j * a.nc;
+    t.nt = min(a.nc, a.np - t.n0);
     return t;
 }
 struct UnitD {  // lower-triangle tile (tn >= tm) of block pairs, one head group
@@ -565,7 +572,6 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_init(&sm->acc_empty[b], EPI_WARPS);
         }
         mbar_init(&sm->done, 1);
-        mbar_init(&sm->epi_bar, EPI_WARPS);
         sm->abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         for (int i = 0; i < 2; ++i) {
@@ -738,14 +744,15 @@ __global__ void __launch_bounds__(THREADS, 1)
     ok = grid_sync(a, sm, kSyncB);
 
     // ================================================================ phase C
-    // Qhat / Khat tiles: hid[p] (hi, lo) x W2[p], written as hi / lo images
-    // per (row tile, head, 64-column chunk of dhp).
+    // Qhat / Khat: hid[p] (hi, lo) x W2[p] in units of nc columns (about one
+    // unit per SM), written as hi / lo images per (row tile, head, 64-column
+    // chunk of dhp); a unit's columns need not start at an image boundary.
     if (ok) {
         const int nunits = 2 * a.rt * a.nj2;
         if (warp == 0 && lane == 0) {
             for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
                 const UnitC t = unit_c(a, u);
-                const int groups = t.nt >> 6;
+                const int groups = (t.nt + 63) >> 6;
                 for (int c = 0; c < a.kc2 && ok; ++c, ++it) {
                     const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
                     if (!(ok = wait(&sm->empty[s], ph ^ 1, sm, a.sync, lim))) break;
@@ -776,63 +783,43 @@ __global__ void __launch_bounds__(THREADS, 1)
                 ++acc_it;
             }
         } else if (warp >= 2) {
-            // For the CTA's last unit of the phase the output images are built in
-            // the idle ring (8 images of 16 KB at most) and sent with one bulk
-            // copy each; otherwise each thread stores its 16-byte chunks directly.
+            // The unit's 8-column chunks are split between the two warp
+            // groups; each thread loads four chunks of its row at a time.
             for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
                 const UnitC t = unit_c(a, u);
                 const uint32_t b = acc_it & 1;
                 if (!(ok = wait_warp(&sm->acc_full[b], (acc_it >> 1) & 1, sm, a.sync, lim))) break;
                 tc_fence_after();
-                const bool staged = u + (int)gridDim.x >= nunits;
-                const int half = t.nt >> 1;
-                const uint32_t taddr = tmem + b * ACC_COLS + ((uint32_t)(q4 * 32) << 16) + hf * half;
-                for (int c = 0; c < half; c += 32) {
+                const int nch = t.nt >> 3, mine = nch >> 1, ch0 = hf * mine;
+                const uint32_t taddr = tmem + b * ACC_COLS + ((uint32_t)(q4 * 32) << 16) + ch0 * 8;
+                for (int c = 0; c < mine; c += 4) {
                     uint32_t r[32];
-                    tmem_ld16(taddr + c, &r[0]);
-                    tmem_ld16(taddr + c + 16, &r[16]);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        if (c + q < mine) tmem_ld8(taddr + (c + q) * 8, &r[8 * q]);
                     tmem_wait_ld();
-                    if (c + 32 >= half) {  // every read of the accumulator landed: free it
+                    if (c + 4 >= mine) {  // every read of the accumulator landed: free it
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&sm->acc_empty[b]);
                     }
 #pragma unroll
-                    for (int i = 0; i < 32; i += 8) {
-                        const int n = t.n0 + hf * half + c + i;  // padded column (multiple of 8)
+                    for (int q = 0; q < 4; ++q) {
+                        if (c + q >= mine) break;
+                        const int n = t.n0 + (ch0 + c + q) * 8;  // padded column (multiple of 8)
                         const int h = n / a.dhp, e = n - h * a.dhp;
                         float v[8];
 #pragma unroll
-                        for (int e8 = 0; e8 < 8; ++e8) v[e8] = __uint_as_float(r[i + e8]);
+                        for (int e8 = 0; e8 < 8; ++e8) v[e8] = __uint_as_float(r[8 * q + e8]);
                         uint4 hi, lo;
                         split8(v, hi, lo);
-                        uint8_t* im = staged ? tiles + (size_t)((n - t.n0) / KCH) * 2 * IMG
-                                             : qk_img(a, t.p, t.R, h, e / KCH, 0);
-                        im += img_off(erow, e % KCH);
+                        uint8_t* im = qk_img(a, t.p, t.R, h, e / KCH, 0) + img_off(erow, e % KCH);
                         *reinterpret_cast<uint4*>(im) = hi;
                         *reinterpret_cast<uint4*>(im + IMG) = lo;
                     }
                 }
                 ++acc_it;
-                if (staged) {
-                    // every warp's part of the images is written: then one thread
-                    // sends them (a bounded wait, so a warp that gave up cannot
-                    // hold the others)
-                    fence_proxy_smem();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&sm->epi_bar);
-                    if (threadIdx.x == 64 && wait(&sm->epi_bar, 0, sm, a.sync, lim)) {
-                        for (int j = 0; j < t.nt / KCH; ++j) {
-                            const int n = t.n0 + j * KCH;
-                            const int h = n / a.dhp, e = n - h * a.dhp;
-                            bulk_store(qk_img(a, t.p, t.R, h, e / KCH, 0),
-                                       smem_u32(tiles + (size_t)j * 2 * IMG), 2 * IMG);
-                        }
-                        bulk_commit();
-                    }
-                }
             }
-            bulk_wait_all();  // every staged copy landed (and read the ring) before the barrier
         }
     }
     ok = grid_sync(a, sm, kSyncC);
