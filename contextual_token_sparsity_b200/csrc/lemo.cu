@@ -870,7 +870,6 @@ lemo_status lemo_predict_scores(const lemo_shape* shape, int32_t d, const uint16
     pa.H = shape->H;
     pa.dh = shape->dh;
     pa.dhp = p.dhp;
-    pa.w1_vec4 = rank % 2 == 0 && aligned(w1q, 4) && aligned(w1k, 4);
     pa.w2_vec4 = shape->dh % 2 == 0 && aligned(w2q, 4) && aligned(w2k, 4);
     pr::Maps maps;
     for (int i = 0; i < 2; ++i) {

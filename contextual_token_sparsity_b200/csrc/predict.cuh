@@ -161,7 +161,7 @@ struct PadArgs {
     const uint16_t* w2[2];   // [rank, H dh] sources
     uint16_t* w2p[2];        // [rank, H dhp] planes, head h at columns h dhp (null: not padded)
     int d, rank, ldw1, H, dh, dhp;
-    int w1_vec4, w2_vec4;    // the source rows allow 4-byte loads
+    int w2_vec4;             // the W2 source rows allow 4-byte loads
 };
 
 __device__ __forceinline__ void add_row(float* acc, const uint4 v) {
@@ -208,28 +208,94 @@ __device__ __forceinline__ uint4 load8_shifted(const uint16_t* src, int64_t e, i
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+// Thread t of T copies the 16-byte chunks t, t + T, ... of both padded W1
+// planes, then of both padded W2 planes, with eight loads in flight per
+// thread (consecutive threads take consecutive chunks of a row).  Chunk
+// indices are kept as (row, chunk) pairs advanced by T, so no integer
+// division runs per chunk.
+struct PadCursor {
+    int64_t r;  // row (of one plane; rows of the second plane follow the first's)
+    int c;      // 16-byte chunk within the row
+};
+__device__ __forceinline__ PadCursor pad_cursor(int64_t i, int cpr) {
+    PadCursor k;
+    k.r = i / cpr;
+    k.c = (int)(i - k.r * cpr);
+    return k;
+}
+__device__ __forceinline__ void pad_advance(PadCursor& k, int dr, int dc, int cpr) {
+    k.r += dr;
+    k.c += dc;
+    if (k.c >= cpr) {
+        k.c -= cpr;
+        ++k.r;
+    }
+}
+
 __device__ __noinline__ void pad_weights(const PadArgs& pa, int cta, int nctas) {
-    const int64_t stride = (int64_t)nctas * kPoolThreads;
-    const int64_t t0 = (int64_t)cta * kPoolThreads + threadIdx.x;
-    const int64_t c1 = (int64_t)pa.d * (pa.ldw1 / 8);          // chunks of one W1 plane
-    const int64_t c2 = (int64_t)pa.rank * (pa.H * pa.dhp / 8);  // chunks of one W2 plane
-    for (int p = 0; p < 2; ++p) {
-        if (pa.w1p[p])
-            for (int64_t i = t0; i < c1; i += stride) {
-                const int64_t r = i / (pa.ldw1 / 8);
-                const int c = (int)(i % (pa.ldw1 / 8)) * 8;
-                *reinterpret_cast<uint4*>(pa.w1p[p] + r * pa.ldw1 + c) =
-                    load8_shifted(pa.w1[p], r * pa.rank + c, pa.rank - c);
+    const int64_t T = (int64_t)nctas * kPoolThreads;
+    const int64_t t = (int64_t)cta * kPoolThreads + threadIdx.x;
+    if (pa.w1p[0]) {
+        // rows 0 .. 2d-1: plane p = row / d
+        const int cpr = pa.ldw1 / 8;
+        const int64_t rows = 2 * (int64_t)pa.d;
+        const int dr = (int)(T / cpr), dc = (int)(T % cpr);
+        PadCursor k = pad_cursor(t, cpr);
+        while (k.r < rows) {
+            PadCursor kk = k;
+            uint4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const bool live = kk.r < rows;
+                const int p = kk.r >= pa.d ? 1 : 0;
+                const int64_t r = kk.r - (int64_t)p * pa.d;
+                const int c = kk.c * 8;
+                v[u] = live ? load8_shifted(pa.w1[p], r * pa.rank + c, pa.rank - c)
+                            : make_uint4(0u, 0u, 0u, 0u);
+                pad_advance(kk, dr, dc, cpr);
             }
-        if (pa.w2p[p])
-            for (int64_t i = t0; i < c2; i += stride) {
-                const int64_t k = i / (pa.H * pa.dhp / 8);
-                const int n = (int)(i % (pa.H * pa.dhp / 8)) * 8;
-                const int h = n / pa.dhp, e = n - h * pa.dhp;
-                *reinterpret_cast<uint4*>(pa.w2p[p] + k * pa.H * pa.dhp + n) = load8_any(
-                    pa.w2[p] + k * (int64_t)pa.H * pa.dh + (int64_t)h * pa.dh + e, pa.dh - e,
-                    pa.w2_vec4 != 0);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                if (k.r < rows) {
+                    const int p = k.r >= pa.d ? 1 : 0;
+                    const int64_t r = k.r - (int64_t)p * pa.d;
+                    *reinterpret_cast<uint4*>(pa.w1p[p] + r * pa.ldw1 + k.c * 8) = v[u];
+                }
+                pad_advance(k, dr, dc, cpr);
             }
+        }
+    }
+    if (pa.w2p[0]) {
+        // rows 0 .. 2 rank - 1: plane p = row / rank
+        const int cpr = pa.H * pa.dhp / 8;
+        const int64_t rows = 2 * (int64_t)pa.rank;
+        const int dr = (int)(T / cpr), dc = (int)(T % cpr);
+        PadCursor k = pad_cursor(t, cpr);
+        while (k.r < rows) {
+            PadCursor kk = k;
+            uint4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const bool live = kk.r < rows;
+                const int p = kk.r >= pa.rank ? 1 : 0;
+                const int64_t r = kk.r - (int64_t)p * pa.rank;
+                const int nn = kk.c * 8;
+                const int h = nn / pa.dhp, e = nn - h * pa.dhp;
+                v[u] = live ? load8_any(pa.w2[p] + r * pa.H * pa.dh + (int64_t)h * pa.dh + e,
+                                        pa.dh - e, pa.w2_vec4 != 0)
+                            : make_uint4(0u, 0u, 0u, 0u);
+                pad_advance(kk, dr, dc, cpr);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                if (k.r < rows) {
+                    const int p = k.r >= pa.rank ? 1 : 0;
+                    const int64_t r = k.r - (int64_t)p * pa.rank;
+                    *reinterpret_cast<uint4*>(pa.w2p[p] + r * pa.H * pa.dhp + k.c * 8) = v[u];
+                }
+                pad_advance(k, dr, dc, cpr);
+            }
+        }
     }
 }
 
