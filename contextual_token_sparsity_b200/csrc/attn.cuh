@@ -90,6 +90,7 @@ constexpr int KV_SLOTS = 10;
 constexpr int TMEM_COLS = 512;   // S_0 [0,128), S_1 [128,256), O_0 [256,+dh), O_1 [384,+dh)
 constexpr int O_COL = 256;
 constexpr float kRescaleLog2 = 8.f;  // rescale O only when the max grows by more
+constexpr int HEAD_GROUP = 16;       // heads whose query-tile pairs are interleaved
 
 // shared memory: Q_0 | Q_1 | KV ring | barriers
 constexpr int OFF_Q = 0;
@@ -400,8 +401,18 @@ __global__ void __launch_bounds__(THREADS, 1)
     const WsHeader* hdr = reinterpret_cast<const WsHeader*>(a.ws);
     const int32_t* prefix = reinterpret_cast<const int32_t*>(a.ws + kWsPrefix);
     if (!hdr->valid) return;
-    const int item = blockIdx.x / a.H, h = blockIdx.x % a.H;
-    if (item >= hdr->total_items) return;
+    // Order: heads in groups of HEAD_GROUP; inside a group, query-tile pairs
+    // heaviest first with the group's heads side by side.  The heavy pairs
+    // still start first, and the K / V rows read at a time (one group's
+    // heads) fit in L2.
+    const int ti = hdr->total_items;
+    const int hg = min(a.H, HEAD_GROUP);
+    const int64_t per_group = (int64_t)ti * hg;
+    if (ti <= 0 || (int64_t)blockIdx.x >= per_group * ((a.H + hg - 1) / hg)) return;
+    const int grp = (int)(blockIdx.x / per_group);
+    const int rem = (int)(blockIdx.x - grp * per_group);
+    const int item = rem / hg, h = grp * hg + rem % hg;
+    if (h >= a.H) return;
     const int s = last_le(prefix, a.batch + 1, item);
     const int npairs = prefix[s + 1] - prefix[s];
     const int pair = npairs - 1 - (item - prefix[s]);  // heaviest pairs first

@@ -1003,7 +1003,11 @@ lemo_status lemo_attention_kept(const lemo_shape* shape, const uint16_t* q, cons
         std::lock_guard<std::mutex> lk(g_mu);
         a.spin_limit_ns = (uint64_t)g_spin_ns;
     }
-    launch(at::attn_kernel, (unsigned)(items * shape->H), at::THREADS, at::SMEM_BYTES, st, tq, tk,
+    // heads are taken in groups of HEAD_GROUP: the grid covers whole groups
+    const int hg = shape->H < at::HEAD_GROUP ? shape->H : at::HEAD_GROUP;
+    const int64_t heads = (int64_t)(shape->H + hg - 1) / hg * hg;
+    if (items * heads > INT_MAX) return LEMO_ERR_UNSUPPORTED;
+    launch(at::attn_kernel, (unsigned)(items * heads), at::THREADS, at::SMEM_BYTES, st, tq, tk,
            tv, a);
     return launch_status();
 }
