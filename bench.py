@@ -730,7 +730,9 @@ def run_segloss(args):
                      "algorithmic_flops_per_call": flops},
         "peak_memory": {"workspace_bytes": ws.numel(), "unsegmented_workspace_bytes": full_ws},
         "loss": float(loss.item()),
-        "gpu_launches": (2 + 4 * -(-T // S)) * args.steps,
+        # count + loss kernels; per segment the logits GEMM, the row kernel and
+        # the dh GEMM; one dW GEMM per pair of segments
+        "gpu_launches": (2 + 3 * -(-T // S) + -(-(-(-T // S)) // 2)) * args.steps,
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -1157,10 +1159,10 @@ def run_predict(args):
     out["movement"] = {"gather_gbs": round(g_b / (us["gather"] * 1e-6) / 1e9, 1),
                        "scatter_gbs": round(s_b / (us["scatter"] * 1e-6) / 1e9, 1),
                        "hbm_peak_gbs": bw}
-    # predict: plan, pool, both predictors' first GEMM, split-K reduce, both
-    # second GEMMs, block products, head-group reduce, column sum; select:
-    # plan, select; gather; scatter
-    out["gpu_launches"] = 12 * args.steps
+    # predict: (plan,) pooling pass, persistent predictor kernel - a batch of
+    # one sequence has its plan written by the pooling pass; select: plan,
+    # select; gather; scatter
+    out["gpu_launches"] = ((2 if len(w.lengths) == 1 else 3) + 4) * args.steps
     out["clocks"] = clk
     if not args.no_e2e:
         pin = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).pin_memory()  # noqa

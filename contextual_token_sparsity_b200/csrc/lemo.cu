@@ -828,8 +828,12 @@ lemo_status lemo_predict_scores(const lemo_shape* shape, int32_t d, const uint16
     const lemo::WsLayout& lay = p.base;
     uint32_t* sync = reinterpret_cast<uint32_t*>(w + p.sync);
 
-    launch_plan(shape, w, lay, nullptr, st);
-    if ((e = launch_status()) != LEMO_OK) return e;
+    // one sequence: the pooling pass writes the plan itself (one launch less)
+    const bool own_plan = shape->batch == 1 && shape->total_L > 0;
+    if (!own_plan) {
+        launch_plan(shape, w, lay, nullptr, st);
+        if ((e = launch_status()) != LEMO_OK) return e;
+    }
     if (shape->total_L == 0) return LEMO_OK;
     {
         std::lock_guard<std::mutex> lk(g_mu);
@@ -888,8 +892,9 @@ lemo_status lemo_predict_scores(const lemo_shape* shape, int32_t d, const uint16
         (int64_t)p.tba * ((p.kc * pr::KCH + pr::kPoolCols - 1) / pr::kPoolCols);
     if (npad + pool_ctas > INT_MAX) return LEMO_ERR_UNSUPPORTED;
     launch(pr::pool_kernel, (unsigned)(npad + pool_ctas), pr::kPoolThreads, 0, st, x, ld_x, d, p.kc,
-           npad, p.tba, shape->cu_seqlens, shape->batch, shape->block, w, lay,
-           reinterpret_cast<uint8_t*>(w + p.xb), sync, pa);
+           npad, p.tba, shape->cu_seqlens, shape->batch, shape->total_L, shape->max_seqlen,
+           shape->block, w, lay, reinterpret_cast<uint8_t*>(w + p.xb), sync, pa,
+           own_plan ? 1 : 0);
     if ((e = launch_status()) != LEMO_OK) return e;
     pr::Args a;
     a.ws = w;

@@ -149,8 +149,10 @@ __device__ __forceinline__ uint4 load8_any(const uint16_t* src, int valid, bool 
 // [y*1024, +1024), each thread 8 consecutive columns (16-byte
 // loads, eight rows in flight, added in row order).  The means are written
 // as hi / lo images [row tile][64-column chunk][plane]; rows g >= TB and
-// columns >= d of the last tile / chunk are written as zeros.  CTA (0, 0)
-// also clears the grid-barrier words of predict_kernel.  The first `npad`
+// columns >= d of the last tile / chunk are written as zeros.  CTA 0 also
+// clears the grid-barrier words of predict_kernel and, for a batch of one
+// sequence (`own_plan`), writes the plan itself (no separate plan launch;
+// the pooling CTAs then take block g as rows [g b, g b + b)).  The first `npad`
 // CTAs (scheduled first, beside the pooling CTAs) copy the
 // weights that TMA cannot read in place (rows not 16-byte aligned, or a head
 // dimension that is not a multiple of 64) into padded planes.
@@ -301,28 +303,46 @@ __device__ __noinline__ void pad_weights(const PadArgs& pa, int cta, int nctas) 
 
 __global__ void __launch_bounds__(kPoolThreads)
     pool_kernel(const uint16_t* __restrict__ x, int64_t ld_x, int d, int kc, int npad, int tba,
-                const int32_t* __restrict__ cu, int batch, int block, const char* __restrict__ ws,
-                WsLayout lay, uint8_t* __restrict__ xb, uint32_t* __restrict__ sync,
-                const PadArgs pa) {
+                const int32_t* __restrict__ cu, int batch, int total_L, int max_seqlen, int block,
+                char* __restrict__ ws, WsLayout lay, uint8_t* __restrict__ xb,
+                uint32_t* __restrict__ sync, const PadArgs pa, int own_plan) {
     pdl_entry();
-    if (blockIdx.x == 0 && threadIdx.x < kSyncWords) sync[threadIdx.x] = 0u;
+    if (blockIdx.x == 0) {
+        if (threadIdx.x < kSyncWords) sync[threadIdx.x] = 0u;
+        // one sequence: this CTA writes the plan (read by predict_kernel); the
+        // pooling CTAs below do not need it
+        if (own_plan)
+            plan_body(cu, batch, total_L, max_seqlen, block, ws, lay, nullptr, nullptr, 0, 1);
+    }
     if ((int)blockIdx.x < npad) {
         pad_weights(pa, blockIdx.x, npad);
         return;
     }
-    const PlanHeader* hdr = reinterpret_cast<const PlanHeader*>(ws + lay.hdr);
-    if (!hdr->valid) return;
+    int nblocks;
+    const int32_t* blk_prefix = reinterpret_cast<const int32_t*>(ws + lay.blk_prefix);
+    if (own_plan) {
+        nblocks = (total_L + block - 1) / block;
+    } else {
+        const PlanHeader* hdr = reinterpret_cast<const PlanHeader*>(ws + lay.hdr);
+        if (!hdr->valid) return;
+        nblocks = hdr->total_blocks;
+    }
     const int u = blockIdx.x - npad;
     const int g = u % tba;
     const int c0 = (u / tba) * kPoolCols + threadIdx.x * 8;
     if (c0 >= kc * KCH) return;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    if (g < hdr->total_blocks && c0 < d) {
-        const int32_t* blk_prefix = reinterpret_cast<const int32_t*>(ws + lay.blk_prefix);
-        const int s = last_le(blk_prefix, batch + 1, g);
-        const int m = g - blk_prefix[s];
-        const int64_t r0 = (int64_t)cu[s] + (int64_t)m * block;
-        const int64_t r1 = min((int64_t)cu[s + 1], r0 + block);
+    if (g < nblocks && c0 < d) {
+        int64_t r0, r1;
+        if (own_plan) {  // one sequence of total_L rows
+            r0 = (int64_t)g * block;
+            r1 = min((int64_t)total_L, r0 + block);
+        } else {
+            const int s = last_le(blk_prefix, batch + 1, g);
+            const int m = g - blk_prefix[s];
+            r0 = (int64_t)cu[s] + (int64_t)m * block;
+            r1 = min((int64_t)cu[s + 1], r0 + block);
+        }
         const uint16_t* p = x + r0 * ld_x + c0;
         int64_t r = r0;
         for (; r + 8 <= r1; r += 8, p += 8 * ld_x) {

@@ -46,14 +46,13 @@ __device__ __forceinline__ T block_scan_incl(T v, T* warp_sums, T* total) {
 // `zero_word` (optional) is set to 0 first, so that a compaction that gives
 // up leaves K = 0 behind rather than a stale count.  `zero_blocks` (optional)
 // gets its first total_blocks entries cleared (the host only knows an upper
-// bound of that count).
+// bound of that count).  plan_body() is the work of one CTA of any size
+// (every thread calls it); plan_kernel is that CTA on its own.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ cu, int batch,
-                                                    int total_L, int max_seqlen, int block,
-                                                    char* __restrict__ ws, WsLayout lay,
-                                                    int32_t* zero_word, float* zero_blocks,
-                                                    int shard, int nshards) {
-    pdl_entry();
+__device__ __noinline__ void plan_body(const int32_t* __restrict__ cu, int batch, int total_L,
+                                       int max_seqlen, int block, char* __restrict__ ws,
+                                       WsLayout lay, int32_t* zero_word, float* zero_blocks,
+                                       int shard, int nshards) {
     PlanHeader* hdr = reinterpret_cast<PlanHeader*>(ws + lay.hdr);
     int64_t* tile_prefix = reinterpret_cast<int64_t*>(ws + lay.tile_prefix);
     int32_t* blk_prefix = reinterpret_cast<int32_t*>(ws + lay.blk_prefix);
@@ -117,6 +116,16 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
         hdr->select_ticket = 0;
         if (bad) raise_error(LEMO_ERR_INVALID_ARG);
     }
+}
+
+__global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ cu, int batch,
+                                                    int total_L, int max_seqlen, int block,
+                                                    char* __restrict__ ws, WsLayout lay,
+                                                    int32_t* zero_word, float* zero_blocks,
+                                                    int shard, int nshards) {
+    pdl_entry();
+    plan_body(cu, batch, total_L, max_seqlen, block, ws, lay, zero_word, zero_blocks, shard,
+              nshards);
 }
 
 // ---------------------------------------------------------------------------

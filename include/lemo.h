@@ -352,8 +352,10 @@ LEMO_API size_t lemo_predict_workspace_size(const lemo_shape* shape, int32_t d, 
  * block_scores DEVICE fp32 [total_blocks].
  * ws, ws_bytes DEVICE workspace of lemo_predict_workspace_size bytes,
  *              256-byte aligned.
- * Three launches: the plan, a pass that streams x once (bound by HBM
- * bandwidth) and writes the block means, and one persistent kernel (one CTA
+ * Two launches for a batch of one sequence, three otherwise: the plan
+ * (written by the pooling pass itself for one sequence), a pass that streams
+ * x once (bound by HBM bandwidth) and writes the block means, and one
+ * persistent kernel (one CTA
  * per SM, grid-wide barriers between its phases) that runs both predictor
  * GEMMs, the Eq. 3 block products and the column sums on the tensor cores
  * (tcgen05, fp32 accumulation in tensor memory).  fp32 accuracy: every fp32
