@@ -731,8 +731,8 @@ def run_segloss(args):
         "peak_memory": {"workspace_bytes": ws.numel(), "unsegmented_workspace_bytes": full_ws},
         "loss": float(loss.item()),
         # count + loss kernels; per segment the logits GEMM, the row kernel and
-        # the dh GEMM; one dW GEMM per pair of segments
-        "gpu_launches": (2 + 3 * -(-T // S) + -(-(-(-T // S)) // 2)) * args.steps,
+        # the dh GEMM; one dW GEMM per four segments
+        "gpu_launches": (2 + 3 * -(-T // S) + -(-(-(-T // S)) // 4)) * args.steps,
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

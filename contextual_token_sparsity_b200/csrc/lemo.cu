@@ -328,19 +328,27 @@ struct SegLayout {
     int64_t nstats;   // partial (max, sum) pairs per logit row (two per 256-column tile)
     int64_t ld;    // row stride of the segment's logits and gradient
     int64_t rows;  // rows of one segment buffer
+    int64_t dz_segs;  // segments of dz held (dW is accumulated once per that many)
 };
+
+constexpr int64_t kDwSegs = 4;  // segments per dW GEMM
 
 SegLayout seg_layout(int64_t T, int V, int seg_rows) {
     SegLayout l;
     l.ld = ((int64_t)V + 7) / 8 * 8;
     l.rows = T < seg_rows ? (T > 0 ? T : 1) : seg_rows;
+    {
+        const int64_t nseg = T > 0 ? (T + seg_rows - 1) / seg_rows : 1;
+        l.dz_segs = nseg < kDwSegs ? nseg : kDwSegs;
+    }
     size_t off = 0;
     l.n_valid = off; off = lemo::align_up(off + 4, 256);
     l.token_loss = off; off = lemo::align_up(off + 4 * (size_t)(T > 0 ? T : 1), 256);
     l.z = off; off = lemo::align_up(off + 4 * (size_t)l.rows * l.ld, 256);
-    // two segments of dz when there are several: dW is accumulated once per
-    // pair of segments (K = 2 segments), which halves its read-add-write
-    l.g = off; off = lemo::align_up(off + 2 * (size_t)(T > seg_rows ? 2 : 1) * l.rows * l.ld, 256);
+    // up to kDwSegs segments of dz: dW is accumulated once per kDwSegs
+    // segments (K = kDwSegs segment rows), which divides its fp32
+    // read-add-write of the weight gradient by kDwSegs
+    l.g = off; off = lemo::align_up(off + 2 * (size_t)l.dz_segs * l.rows * l.ld, 256);
     l.nstats = 2 * (((int64_t)V + lemo::gemm::TN - 1) / lemo::gemm::TN);
     l.stats = off; off = lemo::align_up(off + 8 * (size_t)l.rows * l.nstats, 256);
     l.total = off;
@@ -1057,7 +1065,7 @@ lemo_status lemo_segment_loss(const uint16_t* h, int64_t ld_h, int64_t T, int32_
     for (int64_t s0 = 0, si = 0; s0 < T; s0 += seg_rows, ++si) {
         const int S = (int)(T - s0 < seg_rows ? T - s0 : seg_rows);
         const uint16_t* hs = h + s0 * ld_h;
-        const int hb = (int)(si & 1);                     // which dz half this segment uses
+        const int hb = (int)(si % l.dz_segs);             // which dz slot this segment uses
         uint16_t* gs = g + (size_t)hb * l.rows * l.ld;
         // z [S, V] = h_seg [S, d] . W [V, d]^T  (fp32, row stride l.ld)
         float2* stats = reinterpret_cast<float2*>(wsp + l.stats);
@@ -1083,11 +1091,12 @@ lemo_status lemo_segment_loss(const uint16_t* h, int64_t ld_h, int64_t T, int32_
                                 gm::kStoreBF16, dh + s0 * ld_dh, ld_dh, true)) != LEMO_OK)
             return e;
         // dW [V, d] += dz^T [V, K] . h [K, d] over the rows of this segment and
-        // the one before it (the two dz halves are consecutive rows), both read
-        // MN-major; after every second segment and after the last one
+        // the ones before it since the last dW GEMM (the dz slots hold
+        // consecutive rows), both read MN-major; after every kDwSegs-th
+        // segment and after the last one
         const bool last = s0 + seg_rows >= T;
-        if (dw && (hb == 1 || last)) {
-            const int64_t p0 = hb == 1 ? s0 - seg_rows : s0;
+        if (dw && (hb == l.dz_segs - 1 || last)) {
+            const int64_t p0 = s0 - (int64_t)hb * seg_rows;
             const int K = (int)(s0 + S - p0);
             if ((e = run_gemm(dev, sms, st, g, l.ld, true, h + p0 * ld_h, ld_h, true, V, d, K,
                               gm::kAddF32, dw, ld_dw, false)) != LEMO_OK)

@@ -427,14 +427,14 @@ LEMO_API lemo_status lemo_attention_kept(const lemo_shape* shape, const uint16_t
 /*
  * Workspace bytes of lemo_segment_loss for T tokens, vocabulary V and
  * segments of seg_rows tokens: the valid-token count, the per-token loss
- * terms, ONE segment's fp32 logits, the bf16 logit gradients of TWO
- * segments (one when T <= seg_rows) and the rows' partial softmax
- * statistics (8 bytes per 128 logits): about (4 + 2 x 2) x min(seg_rows, T)
- * x round_up(V, 8) bytes.  That is the activation peak that segmenting
- * divides by about 3/4 x T / seg_rows (it is about 6 x T x round_up(V, 8)
- * bytes unsegmented); the second gradient segment lets dW be accumulated
- * once per pair of segments.  Returns 0 for invalid arguments.  HOST-only
- * computation.
+ * terms, ONE segment's fp32 logits, the bf16 logit gradients of up to FOUR
+ * segments (as many as there are, at most four) and the rows' partial
+ * softmax statistics (8 bytes per 128 logits): about (4 + 2 x 4) x
+ * min(seg_rows, T) x round_up(V, 8) bytes.  That is the activation peak that
+ * segmenting divides by about T / (2 seg_rows) (it is about 6 x T x
+ * round_up(V, 8) bytes unsegmented); the extra gradient segments let dW be
+ * accumulated once per four segments.  Returns 0 for invalid arguments.
+ * HOST-only computation.
  */
 LEMO_API size_t lemo_segment_loss_workspace_size(int64_t T, int32_t V, int32_t seg_rows);
 
@@ -476,7 +476,7 @@ LEMO_API size_t lemo_segment_loss_workspace_size(int64_t T, int32_t V, int32_t s
  * The three GEMMs of a segment run on this library's tensor-core kernel
  * (tcgen05 on CTA pairs, bf16 inputs, fp32 accumulation in tensor memory;
  * the logits are stored in fp32, dh rounded once to bf16, dW accumulated in
- * fp32 once per pair of segments, in segment order); the logits GEMM's
+ * fp32 once per four segments, in segment order); the logits GEMM's
  * epilogue also leaves each row's running (max, sum of exponentials) per
  * 128 columns, from which a separate row kernel forms the softmax, the loss
  * term and the bf16 gradient of each logit row, reading the logits once.
