@@ -634,13 +634,6 @@ __device__ __forceinline__ void mma_weight_chunk(uint32_t d_tmem, uint32_t st, u
 
 __global__ void __launch_bounds__(THREADS, 1)
     predict_kernel(const __grid_constant__ Maps maps, const Args a) {
-    pdl_entry();
-    fence_proxy_global();  // the pooling pass's stores -> this kernel's bulk copies
-    const PlanHeader* hdr = reinterpret_cast<const PlanHeader*>(a.ws + a.lay.hdr);
-    if (!hdr->valid) return;  // every CTA leaves here, before any barrier
-    const int TB = hdr->total_blocks;
-    const int32_t* blk_prefix = reinterpret_cast<const int32_t*>(a.ws + a.lay.blk_prefix);
-
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* tiles = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -675,6 +668,24 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm->tmem_base;
+
+    // Nothing above reads what the pooling pass writes, so it overlaps that
+    // pass's tail; from here on the pass has completed.
+    pdl_entry();
+    fence_proxy_global();  // the pooling pass's stores -> this kernel's bulk copies
+    const PlanHeader* hdr = reinterpret_cast<const PlanHeader*>(a.ws + a.lay.hdr);
+    if (!hdr->valid) {  // the same in every CTA: leave before any barrier
+        tc_fence_before();
+        __syncthreads();
+        if (warp == 1) {
+            tc_fence_after();
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                         "r"(TMEM_COLS));
+        }
+        return;
+    }
+    const int TB = hdr->total_blocks;
+    const int32_t* blk_prefix = reinterpret_cast<const int32_t*>(a.ws + a.lay.blk_prefix);
 
     // Role state, carried across phases (producer and MMA count the same
     // stage uses; MMA and epilogue the same accumulations).
@@ -772,41 +783,46 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ================================================================ phase B
     // hid[p][row][col] = relu(sum_z part[p][z][row][col]), as hi / lo images;
     // rows >= TB and columns >= rank are zero.  Four lanes share an item of 8
-    // columns: lane j sums its quarter of z in order, then the quarters are
-    // added as (q0 + q1) + (q2 + q3) - a fixed order.
+    // columns below the rank: lane j sums its quarter of z in order, then the
+    // quarters are added as (q0 + q1) + (q2 + q3) - a fixed order.  The
+    // chunks of padding columns past the rank take one lane each (zeros), so
+    // that every item fits in one pass of the grid.
     if (ok) {
-        const int chunks_per_row = a.kc2 * 8;
-        const int64_t items = 2LL * a.tba * chunks_per_row;
+        const int cpr = a.kc2 * 8;            // 8-column chunks of a hid row
+        const int lcpr = (a.rank + 7) / 8;    // chunks holding columns below the rank
+        const int64_t live4 = 4LL * 2 * a.tba * lcpr;
+        const int64_t lanes = live4 + 2LL * a.tba * (cpr - lcpr);
         const int zq = (a.zk + 3) / 4;
         const int64_t span = (int64_t)gridDim.x * THREADS;
-        for (int64_t base = (int64_t)blockIdx.x * THREADS; base < items * 4; base += span) {
+        for (int64_t base = (int64_t)blockIdx.x * THREADS; base < lanes; base += span) {
             // every lane runs the loop the same number of times (the shuffles below)
-            const int64_t i4 = base + threadIdx.x;
-            const int64_t i = i4 >> 2;
-            const int quarter = (int)(i4 & 3);
-            const int cj = (int)(i % chunks_per_row);
-            const int row = (int)((i / chunks_per_row) % a.tba);
-            const int p = (int)(i / ((int64_t)chunks_per_row * a.tba));
+            const int64_t t = base + threadIdx.x;
+            const bool is_live = t < live4;  // groups of four lanes never straddle live4
+            const int64_t i = t >> 2;
+            const int quarter = (int)(t & 3);
+            const int cj = (int)(i % lcpr);
+            const int row = (int)((i / lcpr) % a.tba);
+            const int p = (int)(i / ((int64_t)lcpr * a.tba));
             const int col0 = cj * 8;
-            const bool live = i < items && row < TB && col0 < a.rank;
+            const bool live = is_live && row < TB;
             float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
             if (live) {
                 const float* src = a.part + ((size_t)p * a.zk * a.tba + row) * a.ldr + col0;
                 const size_t plane = (size_t)a.tba * a.ldr;
                 const int z0 = quarter * zq, z1 = min(a.zk, z0 + zq);
                 for (int z = z0; z < z1; z += 8) {
-                    float4 t[16];
+                    float4 tt[16];
 #pragma unroll
                     for (int uu = 0; uu < 8; ++uu)
                         if (z + uu < z1) {
-                            t[2 * uu] = *reinterpret_cast<const float4*>(src + (z + uu) * plane);
-                            t[2 * uu + 1] = *reinterpret_cast<const float4*>(src + (z + uu) * plane + 4);
+                            tt[2 * uu] = *reinterpret_cast<const float4*>(src + (z + uu) * plane);
+                            tt[2 * uu + 1] = *reinterpret_cast<const float4*>(src + (z + uu) * plane + 4);
                         }
 #pragma unroll
                     for (int uu = 0; uu < 8; ++uu)
                         if (z + uu < z1) {
-                            v[0] += t[2 * uu].x; v[1] += t[2 * uu].y; v[2] += t[2 * uu].z; v[3] += t[2 * uu].w;
-                            v[4] += t[2 * uu + 1].x; v[5] += t[2 * uu + 1].y; v[6] += t[2 * uu + 1].z; v[7] += t[2 * uu + 1].w;
+                            v[0] += tt[2 * uu].x; v[1] += tt[2 * uu].y; v[2] += tt[2 * uu].z; v[3] += tt[2 * uu].w;
+                            v[4] += tt[2 * uu + 1].x; v[5] += tt[2 * uu + 1].y; v[6] += tt[2 * uu + 1].z; v[7] += tt[2 * uu + 1].w;
                         }
                 }
             }
@@ -816,7 +832,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 v[e] += __shfl_xor_sync(0xffffffffu, v[e], 1);
                 v[e] += __shfl_xor_sync(0xffffffffu, v[e], 2);
             }
-            if (quarter == 0 && i < items) {
+            if (is_live && quarter == 0) {
 #pragma unroll
                 for (int e = 0; e < 8; ++e) v[e] = (live && col0 + e < a.rank) ? fmaxf(v[e], 0.f) : 0.f;
                 uint4 hi, lo;
@@ -824,6 +840,15 @@ __global__ void __launch_bounds__(THREADS, 1)
                 uint8_t* im = hid_img(a, p, row / TILE, col0 / KCH, 0) + img_off(row % TILE, col0 % KCH);
                 *reinterpret_cast<uint4*>(im) = hi;
                 *reinterpret_cast<uint4*>(im + IMG) = lo;
+            } else if (!is_live && t < lanes) {
+                const int64_t dd = t - live4;
+                const int dcnt = cpr - lcpr;
+                const int dcol0 = (lcpr + (int)(dd % dcnt)) * 8;
+                const int drow = (int)((dd / dcnt) % a.tba);
+                const int dp = (int)(dd / ((int64_t)dcnt * a.tba));
+                uint8_t* im = hid_img(a, dp, drow / TILE, dcol0 / KCH, 0) + img_off(drow % TILE, dcol0 % KCH);
+                *reinterpret_cast<uint4*>(im) = make_uint4(0u, 0u, 0u, 0u);
+                *reinterpret_cast<uint4*>(im + IMG) = make_uint4(0u, 0u, 0u, 0u);
             }
         }
     }
