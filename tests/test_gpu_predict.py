@@ -77,9 +77,10 @@ def oracle_predict(lengths, H, dh, b, x_bits, w1q, w2q, w1k, w2k):
 
 CASES = [([300, 0, 517, 64, 1], 2, 64, 64, 64, 48),
          ([1000], 3, 128, 128, 256, 40),
-         ([2049, 640], 4, 32, 64, 136, 100),   # rank % 8 != 0: W1 rows read 4 bytes at a time
+         ([2049, 640], 4, 32, 64, 136, 100),   # rank % 8 != 0: W1 copied into padded planes
          ([700, 130], 3, 20, 64, 64, 37),       # odd rank and dh % 8 != 0: padded weight copies
-         ([513], 2, 24, 128, 40, 6)]
+         ([513], 2, 24, 128, 40, 6),
+         ([777], 2, 64, 64, 64, 24)]            # one sequence, b = 64: the pooling pass writes the plan
 
 
 @pytest.mark.parametrize("lengths,H,dh,b,d,rank", CASES, ids=[str(c[0]) for c in CASES])
