@@ -6,7 +6,8 @@
 //   P[n][m]  = (1/H) sum_h max(Qhat_n^h . Khat_m^h, 0),  n >= m          (block products)
 //   score[m] = sum_{n >= m} P[n][m]                                      (column sum)
 //
-// Two kernels after the per-call plan:
+// Two kernels (after the per-call plan kernel when the batch has several
+// sequences; for one sequence the pooling pass writes the plan itself):
 //
 //   pool_kernel     streams X once (bound by HBM bandwidth) and writes the
 //                   block means as bf16 hi / lo planes already laid out as
