@@ -900,7 +900,7 @@ lemo_status lemo_predict_scores(const lemo_shape* shape, int32_t d, const uint16
         (int64_t)p.tba * ((p.kc * pr::KCH + pr::kPoolCols - 1) / pr::kPoolCols);
     if (npad + pool_ctas > INT_MAX) return LEMO_ERR_UNSUPPORTED;
     launch(pr::pool_kernel, (unsigned)(npad + pool_ctas), pr::kPoolThreads, 0, st, x, ld_x, d, p.kc,
-           npad, p.tba, shape->cu_seqlens, shape->batch, shape->total_L, shape->max_seqlen,
+           npad, shape->cu_seqlens, shape->batch, shape->total_L, shape->max_seqlen,
            shape->block, w, lay, reinterpret_cast<uint8_t*>(w + p.xb), sync, pa,
            own_plan ? 1 : 0);
     if ((e = launch_status()) != LEMO_OK) return e;

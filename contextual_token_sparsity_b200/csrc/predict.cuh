@@ -145,8 +145,8 @@ __device__ __forceinline__ uint4 load8_any(const uint16_t* src, int valid, bool 
 }
 
 // ---------------------------------------------------------------------------
-// Pooling pass.  CTA npad + y * tba + g (row g, column chunk y, so that the
-// grid is one wave of plain CTAs): block means of token block g over columns
+// Pooling pass.  CTA npad + g * nch + y (block g, column chunk y of nch, so
+// that the grid is one wave of plain CTAs): block means of token block g over columns
 // [y*1024, +1024), each thread 8 consecutive columns (16-byte
 // loads, eight rows in flight, added in row order).  The means are written
 // as hi / lo images [row tile][64-column chunk][plane]; rows g >= TB and
@@ -303,7 +303,7 @@ __device__ __noinline__ void pad_weights(const PadArgs& pa, int cta, int nctas) 
 }
 
 __global__ void __launch_bounds__(kPoolThreads)
-    pool_kernel(const uint16_t* __restrict__ x, int64_t ld_x, int d, int kc, int npad, int tba,
+    pool_kernel(const uint16_t* __restrict__ x, int64_t ld_x, int d, int kc, int npad,
                 const int32_t* __restrict__ cu, int batch, int total_L, int max_seqlen, int block,
                 char* __restrict__ ws, WsLayout lay, uint8_t* __restrict__ xb,
                 uint32_t* __restrict__ sync, const PadArgs pa, int own_plan) {
@@ -328,9 +328,12 @@ __global__ void __launch_bounds__(kPoolThreads)
         if (!hdr->valid) return;
         nblocks = hdr->total_blocks;
     }
+    // neighbouring CTAs take the column chunks of the same block, so the
+    // 128 rows are read whole at about the same time (DRAM page locality)
     const int u = blockIdx.x - npad;
-    const int g = u % tba;
-    const int c0 = (u / tba) * kPoolCols + threadIdx.x * 8;
+    const int nch = (kc * KCH + kPoolCols - 1) / kPoolCols;
+    const int g = u / nch;
+    const int c0 = (u % nch) * kPoolCols + threadIdx.x * 8;
     if (c0 >= kc * KCH) return;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     if (g < nblocks && c0 < d) {
